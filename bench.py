@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Benchmark of the MoT world-action-model chunk on B200.
+
+Default workload: the Fast-WAM-shaped one-step model (28 blocks per expert,
+video width 1536 / action width 768, 24 x 64 heads, FFN 6144 / 3072,
+64 + 1024 video-expert tokens, 32 action tokens of dim 30, batch 1, S = 1),
+bf16, CEWP schedule replayed from a CUDA graph.  One "step" = one chunk
+(video expert once + S action Euler steps) on synthetic seeded inputs that
+are resident in HBM.
+
+Prints one JSON line (rank 0).  --impl reference times the CPU oracle (the
+plain float64 definition) on the host cores instead, on a bounded sample of
+the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ms per action chunk (1-step, CEWP, bs=1); achieved HBM GB/s & TC % of peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "_kind": "fallback"}
+
+WORKLOADS = {
+    2: "Fast-WAM-shaped one-step MoT: 28 blocks/expert, d 1536/768, 24x64 heads, FFN 6144/3072, "
+       "64+1024 video tokens, 32 action tokens x 30, batch 1",
+    3: "teacher-style 10-step: config-2 shapes, S=10 uniform grid",
+    4: "throughput batch: config-2 architecture, batch 8, 64+2048 video tokens, 32 action tokens",
+}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--config", type=int, default=2, choices=[2, 3, 4])
+    p.add_argument("--schedule", default="cewp", choices=["cewp", "sequential"])
+    p.add_argument("--no-graph", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--seed", type=int, default=0)
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        d["_kind"] = "measured"
+        return d
+    except Exception:
+        return dict(FALLBACK_PEAKS)
+
+
+# ---------------------------------------------------------------- work model
+def work_model(c, S):
+    """Algorithmic FLOPs and HBM bytes of one chunk (what the method must do).
+
+    GEMM FLOPs 2*M*N*K; attention 4*Lq*Lk*Dh per (sample, head).  The video
+    expert runs once and skips its last block's attention and remainder (no
+    video output); the action expert runs S times.  Bytes: every weight read
+    once per use, activations in/out once per kernel, K/V written once and
+    read by every consumer."""
+    N, dv, da, A, Fv, Fa = c.n_blocks, c.d_video, c.d_action, c.n_heads * c.head_dim, c.ffn_video, c.ffn_action
+    Lv, La, B, H, Dh, P = c.l_cond + c.l_video, c.l_action, c.batch, c.n_heads, c.head_dim, c.action_dim
+    Mv, Ma = B * Lv, B * La
+    e = 2  # bf16
+    w = {}
+    # per-launch GEMM work of each class: (flops, bytes)
+    w["video_qkv"] = (2 * Mv * dv * 3 * A, e * (3 * A * dv + Mv * dv + 3 * Mv * A))
+    w["video_oproj"] = (2 * Mv * A * dv, e * (A * dv + Mv * A) + 8 * Mv * dv)
+    w["video_ffn_up"] = (2 * Mv * dv * Fv, e * (Fv * dv + Mv * dv + Mv * Fv))
+    w["video_ffn_down"] = (2 * Mv * Fv * dv, e * (Fv * dv + Mv * Fv) + 8 * Mv * dv)
+    w["video_attn"] = (4 * B * H * Lv * Lv * Dh, e * B * H * Dh * 4 * Lv)
+    w["action_qkv"] = (2 * Ma * da * 3 * A, e * (3 * A * da + Ma * da + 3 * Ma * A))
+    w["action_oproj"] = (2 * Ma * A * da, e * (A * da + Ma * A) + 8 * Ma * da)
+    w["action_ffn_up"] = (2 * Ma * da * Fa, e * (Fa * da + Ma * da + Ma * Fa))
+    w["action_ffn_down"] = (2 * Ma * Fa * da, e * (Fa * da + Ma * Fa) + 8 * Ma * da)
+    w["action_attn"] = (4 * B * H * La * (Lv + La) * Dh, e * B * H * Dh * (2 * (Lv + La) + 2 * La))
+    counts = {"video_qkv": N, "video_oproj": N - 1, "video_ffn_up": N - 1, "video_ffn_down": N - 1,
+              "video_attn": N - 1, "action_qkv": N * S, "action_oproj": N * S, "action_ffn_up": N * S,
+              "action_ffn_down": N * S, "action_attn": N * S}
+    flops = sum(w[k][0] * counts[k] for k in w)
+    # chunk bytes: weights once per use + activations (above) + small terms
+    bytes_ = sum(w[k][1] * counts[k] for k in w)
+    bytes_ += e * (N * (6 * dv * dv) + S * N * 0) + 4 * (Mv * dv + Ma * P * 2)
+    return w, counts, flops, bytes_
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------- CPU baseline
+def cpu_oracle_sample(cfg_id, seed, blocks=2, reps=3, budget_s=25.0):
+    """The oracle, as it stands, on a bounded sample of the workload: the first
+    `blocks` blocks of each expert (parameters generated outside the timing),
+    scaled to the full depth.  Returns (ms per chunk, sample description)."""
+    import numpy as np  # noqa: F401
+
+    import synthetic
+    from oracle import model as M
+    from oracle import params as PR
+    from oracle.config import preset as opreset
+    full = opreset(cfg_id)
+    oc = full.with_(n_blocks=blocks)
+    S = full.default_steps
+    P = PR.generate_params(oc, seed)
+    inp = synthetic.make_inputs(seed, batch=oc.batch, l_cond=oc.l_cond, l_video=oc.l_video,
+                                video_width=oc.d_video, l_action=oc.l_action, action_dim=oc.action_dim)
+    times = []
+    t_start = time.perf_counter()
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        M.infer_chunk(oc, P, inp, S=S)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_start > budget_s:
+            break
+    scale = full.n_blocks / blocks
+    ms = statistics.median(times) * 1e3 * scale
+    sample = (f"oracle float64 forward of the first {blocks} of {full.n_blocks} blocks per expert "
+              f"(S={S}), median of {len(times)} runs, x{scale:g} to the full depth; parameter "
+              f"generation excluded")
+    return ms, sample
+
+
+def cpu_info():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+# ------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    cfg_id = args.config
+    times = []
+    sample = None
+    for i in range(args.warmup + args.steps):
+        ms, sample = cpu_oracle_sample(cfg_id, args.seed, blocks=1, reps=1, budget_s=1e9)
+        if i >= args.warmup:
+            times.append(ms)
+    v = statistics.mean(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "ms", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOADS[cfg_id], "global_batch": 1 if cfg_id != 4 else 8,
+                   "seq_len": 1088 + 32 if cfg_id != 4 else 2112 + 32, "parallelism": "replicas",
+                   "schedule": "sequential (oracle)"},
+        "cpu_baseline": {"value": round(v, 3), "unit": "ms", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": sample + f"; one sample per step, {cpu_info()}"},
+        "e2e": {"value": round(v, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import mot_dit_b200 as W
+    import synthetic
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    c = W.preset(args.config)
+    S = 10 if args.config == 3 else 1
+    mode = W.CEWP if args.schedule == "cewp" else W.SEQUENTIAL
+    wam = W.Wam(c, seed=args.seed + rank)
+    inp = synthetic.make_inputs(args.seed + rank, batch=c.batch, l_cond=c.l_cond, l_video=c.l_video,
+                                video_width=c.d_video, l_action=c.l_action, action_dim=c.action_dim)
+    video = torch.from_numpy(inp["video"]).to(dev)
+    cond = torch.from_numpy(inp["cond"]).to(dev)
+    noise = torch.from_numpy(inp["noise"]).to(dev)
+    out = torch.empty_like(noise)
+    sv = torch.cuda.Stream(device=dev, priority=0)
+    sa = torch.cuda.Stream(device=dev, priority=-1)
+    use_graph = not args.no_graph
+
+    def step():
+        wam.infer_chunk(video, cond, noise, out, S=S, mode=mode, use_graph=use_graph,
+                        stream_video=sv, stream_action=sa)
+
+    def barrier():
+        if dist:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    sv.synchronize()
+    wam.check_device_status()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(sv)
+    for _ in range(args.steps):
+        step()
+    e1.record(sv)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    wam.check_device_status()
+    elapsed = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+    ms_per_step = elapsed / args.steps
+    launches_per_chunk = wam.chunk_kernel_count(S)
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    hv = torch.from_numpy(inp["video"]).pin_memory()
+    hc = torch.from_numpy(inp["cond"]).pin_memory()
+    hn = torch.from_numpy(inp["noise"]).pin_memory()
+    ho = torch.empty(hn.shape, dtype=torch.float32).pin_memory()
+
+    def step_host():
+        wam.infer_chunk_host(hv.data_ptr(), hc.data_ptr(), hn.data_ptr(), ho.data_ptr(), S=S, mode=mode,
+                             use_graph=use_graph, stream_video=sv, stream_action=sa)
+
+    for _ in range(3):
+        step_host()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(sv)
+    for _ in range(args.steps):
+        step_host()
+    e1.record(sv)
+    torch.cuda.synchronize()
+    e2e_elapsed = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_elapsed = float(t.item())
+    assert np.array_equal(ho.numpy(), out.cpu().numpy()), "host entry point disagrees with the device one"
+    h2d = 4 * (hv.numel() + hc.numel() + hn.numel())
+    d2h = 4 * ho.numel()
+
+    # live per-class launch timing (eager, sequential, CUDA events on the launching stream)
+    prof = None
+    for _ in range(2):  # second pass is warm
+        prof = wam.profile_chunk(video, cond, noise, out, S=S, stream=sv)
+    wam.check_device_status()
+
+    if dist:
+        dist.barrier()
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return 0
+
+    peaks = load_peaks()
+    w, counts, flops, bytes_ = work_model(c, S)
+    gemm = ["video_qkv", "video_oproj", "video_ffn_up", "video_ffn_down"]
+    g_flops = sum(w[k][0] * counts[k] for k in gemm)
+    g_ms = sum(prof[k][0] for k in gemm)
+    g_launch = sum(prof[k][1] for k in gemm)
+    achieved = g_flops / (g_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    breakdown = {}
+    for k, (ms, n) in prof.items():
+        if n == 0:
+            continue
+        ent = {"us_per_chunk": round(ms * 1e3, 1), "launches": n}
+        if k in w:
+            f_, b_ = w[k]
+            ent["tflops"] = round(f_ * counts[k] / (ms * 1e-3) / 1e12, 1)
+            ent["gbs"] = round(b_ * counts[k] / (ms * 1e-3) / 1e9, 1)
+        breakdown[k] = ent
+    t_tc = flops / (float(peaks["bf16_tflops"]) * 1e12) * 1e3
+    t_hbm = bytes_ / (float(peaks["hbm_gbs"]) * 1e9) * 1e3
+    chunk_roof = max(t_tc, t_hbm)
+
+    line = {
+        "metric": METRIC, "value": round(ms_per_step / world, 4), "unit": "ms", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOADS[args.config], "global_batch": c.batch * world,
+                   "seq_len": c.l_cond + c.l_video + c.l_action, "steps_S": S,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "schedule": args.schedule + ("+graph" if use_graph else "+eager"),
+                   "l2": "no flush: each chunk streams 2.1 GB of weights, > 126 MB L2"},
+        "chunks_per_s": round(1e3 * world / ms_per_step, 2),
+        "actions_per_s": round(1e3 * world * c.batch * c.l_action / ms_per_step, 1),
+        "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMM, video expert (QKV/out/FFN)",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_kind": f"{peaks['_kind']} bf16 sustained",
+                     "launches_timed": g_launch, "method": "CUDA events around each launch, eager sequential chunk"},
+        "chunk_roofline": {"ms": round(chunk_roof, 4), "t_tensor_ms": round(t_tc, 4), "t_hbm_ms": round(t_hbm, 4),
+                           "flops": flops, "bytes": bytes_, "frac": round(chunk_roof / ms_per_step, 4)},
+        "breakdown": breakdown,
+        "e2e": {"value": round(e2e_elapsed / args.steps / world, 4), "unit": "ms", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_chunk * args.steps,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        ms_cpu, sample = cpu_oracle_sample(args.config, args.seed)
+        line["cpu_baseline"] = {"value": round(ms_cpu, 1), "unit": "ms", "cores": os.cpu_count(), "kind": "oracle",
+                                "sample": sample + f"; {cpu_info()}"}
+    print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,219 @@
+/*
+ * wam.h -- C ABI of the B200 (sm_100a) MoT world-action-model forward.
+ *
+ * What is computed.  A Mixture-of-Transformers world-action model has a
+ * video expert and an action expert, each a stack of N DiT blocks; block i
+ * of the action expert attends over the concatenation [K^v_i; K^a_i],
+ * [V^v_i; V^a_i] of the video expert's block-i keys/values and its own, so
+ * the video expert runs once per chunk and publishes z = {(K^v_i, V^v_i)}
+ * (RealtimeWAM summary page, section 前置知识: "Mixture-of-Transformers",
+ * "KV 缓存").  The action chunk is then integrated by Euler flow matching,
+ * a_{t_{j-1}} = a_{t_j} - (t_j - t_{j-1}) v(a_{t_j}, t_j), whose one-step form
+ * from t is the endpoint f = a_t - t v (section 前置知识, "流匹配与速度场去噪").
+ * The two experts overlap as the Cross-Expert Wavefront Pipeline: video
+ * stream P^v_i -> record(e_i) -> Attn^v_i -> R^v_i, action stream P^a_i ->
+ * wait(e_i) -> Attn^a_i -> R^a_i (sections 核心方法 and 方法步骤详情; the
+ * tokendh.com article, CEWP section).  The joint one-step variant adds the SNR
+ * time shift, the consistency endpoints and an unmerged LoRA on the action
+ * expert (Flash-WAM close reading, sections 概念 / 方法 / 数据与训练流程).
+ *
+ * Conventions of every entry point.
+ *   - Pointers named dev_* are device pointers on the context's device; the
+ *     caller owns them and keeps them alive until the enqueued work finishes.
+ *     Pointers named host_* are host pointers (pageable or pinned).
+ *   - Streams are cudaStream_t values passed as void* (NULL = legacy default
+ *     stream).  All calls only enqueue work and return; synchronise on the
+ *     stream named in each call's comment.
+ *   - Layouts are row-major, C-contiguous, fp32 unless stated.
+ *   - Errors: argument errors return WAM_ERR_INVALID_ARG before anything is
+ *     enqueued; CUDA errors return WAM_ERR_CUDA (text: wam_last_error); a
+ *     device-side bounded wait that gave up is reported as WAM_ERR_TIMEOUT by
+ *     wam_check_device_status.  No call aborts the process.
+ *   - One context per host thread; a context is bound to the device that was
+ *     current at wam_init.
+ */
+#ifndef MOT_DIT_B200_WAM_H
+#define MOT_DIT_B200_WAM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WAM_OK = 0,
+  WAM_ERR_INVALID_ARG = 1,
+  WAM_ERR_UNSUPPORTED = 2,
+  WAM_ERR_OOM = 3,
+  WAM_ERR_CUDA = 4,
+  WAM_ERR_TIMEOUT = 5,
+  WAM_ERR_STATE = 6
+} wam_status;
+
+typedef enum { WAM_FP32 = 0, WAM_BF16 = 1 } wam_dtype;
+typedef enum { WAM_SCHED_SEQUENTIAL = 0, WAM_SCHED_CEWP = 1 } wam_sched;
+
+/* Model shapes.  N blocks per expert; widths d_video / d_action; n_heads x
+ * head_dim attention (A = n_heads * head_dim, shared by both experts); FFN
+ * widths; l_cond + l_video video-expert tokens (L_v) and l_action action
+ * tokens of dimension action_dim per sample; batch samples.
+ * video_patch_dim > 0 selects patch-vector video input (joint variant).
+ * lora_rank > 0 adds an unmerged LoRA (scale lora_scale) to the action
+ * expert's QKV / out / FFN projections.  video_has_output: the video expert's
+ * last block and output map run (joint variant).  dtype: WAM_BF16 (bf16
+ * weights and GEMM operands, fp32 accumulation and residual stream, head_dim
+ * 64) or WAM_FP32 (fp32 everywhere, debug precision). */
+typedef struct {
+  int n_blocks, d_video, d_action, n_heads, head_dim, ffn_video, ffn_action;
+  int l_cond, l_video, l_action, action_dim, video_patch_dim;
+  int batch, lora_rank;
+  float lora_scale;
+  int video_has_output;
+  int dtype;
+} wam_config;
+
+typedef struct wam_ctx wam_ctx;
+
+/* Fill *out with synthetic preset k (1: tiny fp32; 2: Fast-WAM-shaped bf16,
+ * 28 blocks, 1536/768 widths, 64+1024 video tokens, 32 action tokens;
+ * 3: as 2 (the 10-step teacher schedule is chosen per call); 4: as 2 with
+ * batch 8 and 2048 video tokens; 5: joint one-step, 30 blocks at 1536,
+ * 1024 patch tokens of dim 192, 16 action tokens, LoRA rank 128).
+ * Returns WAM_ERR_INVALID_ARG for an unknown k. */
+wam_status wam_preset(int k, wam_config* out);
+
+/* Create a context on the current device: generates the seeded parameters
+ * on the device (parameter p, element e: SplitMix64 counters
+ * (seed XOR p*0x9E3779B97F4A7C15) + 2e + {0,1}, Box-Muller, N(0, 0.02) for
+ * weights / biases / modulation tables / LoRA factors, 1 for norm gains;
+ * rounded to bf16 for bf16 models), allocates the K/V cache, the
+ * activations and the workspaces, and creates the per-block events.
+ * Synchronous.  *out is set only on WAM_OK. */
+wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out);
+
+/* Release everything the context owns (device memory, events, graphs).
+ * Synchronises the device first.  NULL is a no-op. */
+void wam_destroy(wam_ctx* ctx);
+
+/* Video expert of one chunk on `stream`: x = [cond; video] per sample, N DiT
+ * blocks at timestep t_video; block i publishes K^v_i / V^v_i into the cache
+ * and records its ready event right after its projection.  The last block's
+ * attention and remainder run only when the model has a video output.
+ * dev_video: [B, l_video, d_video]; dev_cond: [B, l_cond, d_video] (NULL iff
+ * l_cond == 0).  Before overwriting block i's K/V it waits for the previous
+ * chunk's action attention of block i. */
+wam_status wam_video_forward(wam_ctx* ctx, const float* dev_video, const float* dev_cond, float t_video,
+                             void* stream);
+
+/* One Euler step of the action expert on `stream`, in place on
+ * dev_actions [B, l_action, action_dim]: a <- a - (t_from - t_to) v(a, t_from).
+ * Block i waits for the video expert's block-i event before its attention.
+ * Requires a wam_video_forward on this context first (else WAM_ERR_STATE).
+ * t_from > t_to, both in [0, 1], else WAM_ERR_INVALID_ARG. */
+wam_status wam_action_step(wam_ctx* ctx, float* dev_actions, float t_from, float t_to, void* stream);
+
+/* Whole chunk: video expert once (at t = 0) and S Euler steps from the noise
+ * dev_noise [B, l_action, action_dim] along host_t_sched (S + 1 values,
+ * t_S = first > ... > t_0 = last, within [0, 1]; NULL = uniform j/S), result
+ * in dev_actions_out.  mode: WAM_SCHED_CEWP runs the experts on stream_video
+ * and stream_action with one event per block (action attention i waits only
+ * for video block i); WAM_SCHED_SEQUENTIAL runs everything on stream_video.
+ * Both produce bitwise-identical results.  use_graph: capture the chunk once
+ * per (S, mode) into a CUDA graph and replay it (pointers and the schedule
+ * are read from device memory, so later calls may change them).  The work
+ * starts after all work previously enqueued on both streams and completes on
+ * stream_video.  1 <= S <= 64. */
+wam_status wam_infer_chunk(wam_ctx* ctx, const float* dev_video, const float* dev_cond, const float* dev_noise,
+                           float* dev_actions_out, int S, const float* host_t_sched, int mode, int use_graph,
+                           void* stream_video, void* stream_action);
+
+/* Same as wam_infer_chunk with host buffers: copies host_video / host_cond /
+ * host_noise into context-owned device buffers on stream_video, runs the
+ * chunk, copies the actions back into host_actions_out and synchronises
+ * stream_video before returning. */
+wam_status wam_infer_chunk_host(wam_ctx* ctx, const float* host_video, const float* host_cond,
+                                const float* host_noise, float* host_actions_out, int S, const float* host_t_sched,
+                                int mode, int use_graph, void* stream_video, void* stream_action);
+
+/* Joint one-step variant (1 video step, 1 action step): sigma_v / sigma_a
+ * from the unshifted levels u_video / u_action by sigma = s u / (1 + (s-1) u);
+ * x_sigma = (1 - sigma_v) x_0 + sigma_v eps_v, a_sigma = (1 - sigma_a) a_0 +
+ * sigma_a eps_a; outputs the action endpoint f^a = a_sigma - sigma_a v^a and
+ * the video endpoint f^v = c_skip x_sigma + c_out (x_sigma - sigma_v v^v),
+ * c_skip = sd^2/(sigma^2+sd^2), c_out = sigma sd / sqrt(sigma^2+sd^2),
+ * sd = 0.5.  Requires video_patch_dim > 0 and video_has_output.
+ * dev_video_clean / dev_video_eps: [B, l_video, video_patch_dim];
+ * dev_action_clean / dev_action_eps: [B, l_action, action_dim];
+ * outputs of the same shapes.  Streams, mode and use_graph as in
+ * wam_infer_chunk. */
+wam_status wam_joint_one_step(wam_ctx* ctx, const float* dev_video_clean, const float* dev_video_eps,
+                              const float* dev_action_clean, const float* dev_action_eps, float u_video,
+                              float u_action, float shift_video, float shift_action, float* dev_video_out,
+                              float* dev_action_out, int mode, int use_graph, void* stream_video,
+                              void* stream_action);
+
+/* Copy every parameter, in generation order, as fp32 into host_buf (matrix
+ * padding removed).  With host_buf == NULL only *nbytes is set.  Synchronous.
+ * WAM_ERR_INVALID_ARG if *nbytes is too small. */
+wam_status wam_export_params(wam_ctx* ctx, float* host_buf, size_t* nbytes);
+
+/* Overwrite every parameter from host_buf (same order and size as
+ * wam_export_params; values are rounded to bf16 for bf16 models).  Synchronous. */
+wam_status wam_import_params(wam_ctx* ctx, const float* host_buf, size_t nbytes);
+
+/* Copy block `block`'s K (which = 0) or V (which = 1) cache, [B, H,
+ * l_cond + l_video + l_action, head_dim], as fp32 into host_buf (size
+ * checked against *nbytes; NULL: report size).  Synchronous. */
+wam_status wam_read_kv(wam_ctx* ctx, int block, int which, float* host_buf, size_t* nbytes);
+
+/* Synchronise the context's device and report device-side failures of the
+ * bounded waits (WAM_ERR_TIMEOUT, then clears the flag) or CUDA errors. */
+wam_status wam_check_device_status(wam_ctx* ctx);
+
+/* Number of kernel launches one chunk enqueues for (S, mode) (graph or not). */
+int wam_chunk_kernel_count(wam_ctx* ctx, int S);
+
+/* Kernel classes of wam_profile_chunk. */
+typedef enum {
+  WAM_PROF_VIDEO_NORM = 0, WAM_PROF_VIDEO_QKV, WAM_PROF_VIDEO_ATTN, WAM_PROF_VIDEO_OPROJ,
+  WAM_PROF_VIDEO_FFN_UP, WAM_PROF_VIDEO_FFN_DOWN, WAM_PROF_VIDEO_TEMB, WAM_PROF_VIDEO_IO,
+  WAM_PROF_ACTION_NORM, WAM_PROF_ACTION_QKV, WAM_PROF_ACTION_ATTN, WAM_PROF_ACTION_OPROJ,
+  WAM_PROF_ACTION_FFN_UP, WAM_PROF_ACTION_FFN_DOWN, WAM_PROF_ACTION_TEMB, WAM_PROF_ACTION_IO,
+  WAM_PROF_CLASSES
+} wam_prof_class;
+
+/* Measurement: run one chunk (S uniform steps) eagerly with the sequential
+ * schedule on `stream`, with a CUDA event pair around every launch, and
+ * return per class the summed launch durations host_ms[WAM_PROF_CLASSES] and
+ * the launch counts host_counts[WAM_PROF_CLASSES].  Synchronises `stream`.
+ * Arguments as in wam_infer_chunk.  (QKV and the action in / out projections
+ * count the whole projection; the fp32 path's QK-norm kernel is part of QKV.) */
+wam_status wam_profile_chunk(wam_ctx* ctx, const float* dev_video, const float* dev_cond, const float* dev_noise,
+                             float* dev_actions_out, int S, void* stream, float* host_ms, int* host_counts);
+
+const char* wam_status_str(wam_status s);
+const char* wam_last_error(wam_ctx* ctx);
+
+/* ---- single-operation entry points (tests and measurement) ------------ */
+
+/* C[M, N] = X[M, K] W[N, K]^T + bias (fp32 out), X / W bf16 (dtype WAM_BF16)
+ * on the tcgen05 path or fp32 (WAM_FP32) on the SIMT path.  swap selects
+ * the few-token orientation (weight on the 128-row MMA operand), splits its
+ * split-K factor.  K must be a multiple of 64 and ld of X / W equal K on the
+ * bf16 path.  Uses a private workspace; enqueued on `stream`. */
+wam_status wam_op_linear(int dtype, const void* dev_x, const void* dev_w, const float* dev_bias, float* dev_out,
+                         int M, int N, int K, int swap, int splits, void* stream);
+
+/* out[B*Lq, H*Dh] = softmax(q k^T / sqrt(Dh)) v per (sample, head) over
+ * cache rows [0, Lk); q [B, H, Lq, Dh], k / v [B, H, Lcache, Dh]; bf16
+ * (Dh = 64, split-KV when splits > 1) or fp32.  Enqueued on `stream`. */
+wam_status wam_op_attention(int dtype, const void* dev_q, const void* dev_k, const void* dev_v, void* dev_out,
+                            int B, int H, int Dh, int Lq, int Lk, int Lcache, int splits, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOT_DIT_B200_WAM_H */

@@ -1,0 +1,161 @@
+// Internal launcher interface of the MoT world-action-model kernels.
+// Host code (the C ABI, the schedules) calls only these functions; each one
+// enqueues kernels on the given stream and returns the launch error code.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace wam {
+
+constexpr int kMaxSteps = 64;  // Euler steps per chunk held in the device schedule
+
+// Per-call inputs read by the first/last kernels of a chunk.  They live in
+// device memory so a captured CUDA graph reads the current call's pointers and
+// timestep schedule instead of baked-in values.
+struct VideoIo {
+  const float* video;   // [B, L_vid, d_v] (or patch vectors [B, L_vid, P_v])
+  const float* cond;    // [B, L_c, d_v] or null
+  const float* eps;     // joint variant: video noise [B, L_vid, P_v]
+  float* video_out;     // joint variant: video endpoint [B, L_vid, P_v]
+  float t;              // video timestep (noise level) of the chunk
+  float u;              // joint variant: unshifted level; shift applied on device
+  float shift;          // joint variant: SNR shift s_v (0: use t as is)
+};
+struct ActionIo {
+  const float* a_in;    // chunk start [B, L_a, P_a] (noise, or the caller's state)
+  const float* a_clean; // joint variant: clean action to noise
+  float* a_out;         // result [B, L_a, P_a]
+  float sched[kMaxSteps + 1];  // t_S, ..., t_0
+  int steps;
+  float u;              // joint variant: unshifted action level
+  float shift;          // joint variant: SNR shift s_a (0: not the joint variant)
+};
+
+enum Epi : int {
+  kEpiStoreF32 = 0,  // out_f32[m, n] = acc + bias[n]
+  kEpiGateRes = 1,   // out_f32[m, n] += gate[n] * (acc + bias[n])
+  kEpiGelu = 2,      // out_act[m, n] = gelu_tanh(acc + bias[n])
+  kEpiQkv = 3,       // bias, per-head QK-RMSNorm with gains, RoPE, scatter to Q and the KV cache
+  kEpiEuler = 4,     // a[m, n] -= (t_j - t_{j-1}) * (acc + bias[n]); also writes the next in-proj input
+  kEpiVideoOut = 5,  // joint variant: video endpoint f^v = c_skip x + c_out (x - sigma v)
+};
+
+struct EpiArgs {
+  int kind = 0;
+  const float* bias = nullptr;
+  const float* gate = nullptr;
+  float* out_f32 = nullptr;
+  void* out_act = nullptr;
+  int ld_out = 0;
+  // QKV scatter
+  const float* gq = nullptr;
+  const float* gk = nullptr;
+  const float* rope_cos = nullptr;  // [cache_len][Dh/2]
+  const float* rope_sin = nullptr;
+  void* q_out = nullptr;            // [B, H, seq_len, Dh]
+  void* k_cache = nullptr;          // [B, H, cache_len, Dh] (block base)
+  void* v_cache = nullptr;
+  int seq_len = 0, cache_len = 0, cache_off = 0, n_heads = 0, head_dim = 0, attn_dim = 0;
+  // Euler / endpoints
+  const ActionIo* aio = nullptr;
+  const VideoIo* vio = nullptr;
+  int step = 0;
+  void* a_next = nullptr;           // next in-proj input (act dtype), ld = a_next_ld
+  int a_next_ld = 0;
+  const float* x_sigma = nullptr;   // joint variant: noised video patches
+};
+
+// C[m, n] = sum_k X[m, k] W[n, k] (+ epilogue), bf16 operands via TMA into
+// tcgen05 tiles.  `swap`: the weight is the 128-row MMA operand (features on
+// TMEM lanes) and the tokens are the N operand -- used when there are few tokens.
+struct TcGemm {
+  const CUtensorMap* map_a;  // A operand: [rows_a, K] (3-D: z = matrix index)
+  const CUtensorMap* map_b;  // B operand: [rows_b, K]
+  int rows_a, rows_b, K;
+  int z_a, z_b;              // matrix index (block) of each operand
+  int bn;                    // N tile (32, 64, 128, 256)
+  int splits;                // split-K factor (swap only)
+  bool swap;
+  float* ws;                 // split-K partials, splits * tiles * 128 * bn floats
+  int* tickets;              // one per output tile, zero on entry, left zero
+  unsigned* status;
+};
+
+cudaError_t launch_tc_gemm(const TcGemm& g, const EpiArgs& e, cudaStream_t s);
+// Sets the kernels' shared-memory attributes; call once per device before any
+// launch (and never during stream capture).
+cudaError_t prepare_tc_gemm();
+
+// fp32 SIMT GEMM (debug precision): C = X W^T + epilogue; X [M, K] (ld = K), W [N, K].
+cudaError_t launch_f32_gemm(const float* X, const float* W, int M, int N, int K, const EpiArgs& e,
+                            cudaStream_t s);
+
+// fp32 path: per-head QK-RMSNorm + RoPE + scatter of a raw projection [M, 3A].
+cudaError_t launch_qkv_post_f32(const float* qkv, int M, const EpiArgs& e, cudaStream_t s);
+
+// h[m, :] = rms(x[m, :]) * (gain ? gain : 1 + scale) + (shift ? shift : 0)
+cudaError_t launch_norm_mod(const float* x, void* h, bool h_bf16, int M, int d, const float* scale,
+                            const float* shift, const float* gain, cudaStream_t s);
+
+// Timestep conditioning of one expert: tau(t) -> c -> m, then mod[i] = m + T_i
+// for every block.  t = io_t[0] (device scalar); weights in `bf16` or fp32.
+struct TembArgs {
+  const float* t;       // device scalar
+  const void* w1; const float* b1;   // [d, 256]
+  const void* w2; const float* b2;   // [d, d]
+  const void* wm; const float* bm;   // [6d, d]
+  const float* T0; size_t T_stride;  // block tables (fp32, [6, d] each, stride in floats)
+  float* mod;                        // [N, 6d]
+  float* scratch;                    // 256 + 2d floats
+  int d, n_blocks;
+  bool bf16;
+};
+cudaError_t launch_temb(const TembArgs& a, cudaStream_t s);
+
+// Attention.  q: [B, H, Lq, Dh]; keys/values are rows [0, Lk) of the cache
+// [B, H, Lcache, Dh]; out: [B*Lq, H*Dh].  Video: keys = video tokens only;
+// action: keys = [video; action] (rows [0, L_v + L_a)), split over key blocks.
+struct AttnArgs {
+  const void* q; const void* k; const void* v; void* out;
+  int B, H, Dh, Lq, Lk, Lcache;
+  int splits;        // key splits (1 = single pass)
+  float* ws;         // partial O / m / l when splits > 1
+  int* tickets;      // B*H counters, zero on entry, left zero
+};
+cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s);
+cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t s);
+size_t attention_ws_floats(int B, int H, int Dh, int Lq, int splits);
+
+// Chunk input/output movers.
+cudaError_t launch_init_video(const VideoIo* io, float* x, int B, int Lc, int Lvid, int d,
+                              cudaStream_t s);
+cudaError_t launch_init_action(const ActionIo* io, float* a_state, void* a_in, bool a_in_bf16,
+                               int M, int P, int ld_in, cudaStream_t s);
+cudaError_t launch_copy_out(const ActionIo* io, const float* a_state, int n, cudaStream_t s);
+cudaError_t launch_set_video_io(VideoIo* dst, const VideoIo& v, cudaStream_t s);
+cudaError_t launch_set_action_io(ActionIo* dst, const ActionIo& v, cudaStream_t s);
+
+// Joint variant input construction: x_sigma = (1 - sigma) x0 + sigma eps with the
+// SNR-shifted sigma computed on device from the io block.
+cudaError_t launch_noise_video(const VideoIo* io, float* x_sigma, void* x_act, bool act_bf16,
+                               int n_rows, int P, int ld_act, cudaStream_t s);
+cudaError_t launch_noise_action(const ActionIo* io, float* a_state, void* a_in, bool a_in_bf16,
+                                int M, int P, int ld_in, cudaStream_t s);
+
+// Seeded parameters (counter-based SplitMix64 + Box-Muller, see wam.h).
+// Element e of a [rows, cols] parameter is stored at out[(e / cols) * ld + e % cols].
+cudaError_t launch_gen_param(uint64_t seed, uint64_t pid, size_t count, double stdv, bool ones,
+                             bool round_bf16, void* out, bool out_bf16, int cols, int ld, cudaStream_t s);
+cudaError_t launch_rope_table(float* cos_t, float* sin_t, int L, int Dh, cudaStream_t s);
+// dst[e] = src[(e / cols) * ld + e % cols] as fp32.
+cudaError_t launch_to_f32(const void* src, bool src_bf16, float* dst, size_t n, int cols, int ld, cudaStream_t s);
+
+// TMA tensor-map creation (driver entry point resolved at run time).
+bool make_tmap_3d(CUtensorMap* map, const void* base, int K, int rows, int nmat, size_t mat_stride_bytes,
+                  int box_rows);
+
+}  // namespace wam

@@ -1,0 +1,1276 @@
+// C ABI of the MoT world-action-model forward: context, seeded parameters,
+// the sequential and Cross-Expert Wavefront Pipeline (CEWP) schedules, CUDA
+// graph capture, and the single-operation entry points.
+//
+// Schedules (RealtimeWAM summary page, sections 核心方法 / 方法步骤详情;
+// tokendh.com article, CEWP section).  A DiT block splits into P_i (norm +
+// merged QKV projection with QK-norm, RoPE and the K/V publish fused into its
+// epilogue), Attn_i and R_i (out-projection + FFN).  CEWP puts the video
+// expert on one stream and the action expert on another: the video stream
+// records event e_i right after P^v_i, the action stream waits on e_i right
+// before Attn^a_i and on nothing else.  The sequential schedule enqueues the
+// same kernels, with the same launch configurations, on one stream -- the two
+// differ only in order, so their results are bitwise identical (every kernel
+// is deterministic; split reductions use a fixed order).
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <memory>
+#include <string>
+#include <vector>
+
+#include "../../include/wam.h"
+#include "kernels.h"
+
+using namespace wam;
+
+namespace {
+
+struct PEntry {
+  std::string name;
+  int rows, cols, ld;
+  bool matrix, ones;
+  size_t off;  // elements into wmat (matrix) or wvec (vector)
+  size_t count() const { return (size_t)rows * cols; }
+};
+
+// Per-block entry order (must match the generation order below).
+enum BlkLocal {
+  kT = 0, kQkvW, kQkvB, kQnG, kKnG, kOW, kOB, kF1W, kF1B, kF2W, kF2B,
+  kQkvLa, kQkvLb, kOLa, kOLb, kF1La, kF1Lb, kF2La, kF2Lb
+};
+
+struct ExpertIdx {
+  int t1w, t1b, t2w, t2b, modw, modb;
+  int inw = -1, inb = -1, fng = -1, outw = -1, outb = -1;
+  int blk0 = -1, per_blk = 0;
+};
+
+struct Dims {
+  int N, dv, da, H, Dh, A, Fv, Fa, Lc, Lvid, Lv, La, Pa, Pv, B, r, Ltot, Mv, Ma, Kin;
+  bool bf16;
+};
+
+struct GemmPlan {
+  int bn = 128, splits = 1;
+};
+
+}  // namespace
+
+struct wam_ctx {
+  wam_config cfg{};
+  Dims d{};
+  int device = 0;
+  std::vector<PEntry> params;
+  ExpertIdx ev{}, ea{};
+  void* wmat = nullptr;
+  float* wvec = nullptr;
+  size_t wmat_elems = 0, wvec_elems = 0;
+  size_t esz = 2;  // bytes per activation / matrix element
+
+  // activations
+  float *x_v = nullptr, *x_a = nullptr, *a_state = nullptr, *x_sigma = nullptr;
+  void *h_v = nullptr, *q_v = nullptr, *o_v = nullptr, *f_v = nullptr, *x_vin = nullptr;
+  void *h_a = nullptr, *q_a = nullptr, *o_a = nullptr, *f_a = nullptr, *a_in = nullptr;
+  float *qkv_tmp_v = nullptr, *qkv_tmp_a = nullptr;  // fp32 path only
+  void* kv = nullptr;                                 // [N][2][B][H][Ltot][Dh]
+  float *mod_v = nullptr, *mod_a = nullptr, *temb_v = nullptr, *temb_a = nullptr;
+  float *rope_cos = nullptr, *rope_sin = nullptr;
+  float* ws_gemm = nullptr;
+  int* tk_gemm = nullptr;
+  float* ws_attn = nullptr;
+  int* tk_attn = nullptr;
+  unsigned* status = nullptr;
+  VideoIo *vio_chunk = nullptr, *vio_eager = nullptr;
+  ActionIo *aio_chunk = nullptr, *aio_eager = nullptr;
+  VideoIo vio_shadow{};
+  ActionIo aio_shadow{};
+  bool vio_valid = false, aio_valid = false;
+  float *h_video = nullptr, *h_cond = nullptr, *h_noise = nullptr, *h_out = nullptr;  // host-API staging
+  float *j_vout = nullptr, *j_aout = nullptr;
+
+  // plans
+  GemmPlan p_v_qkv, p_v_o, p_v_f1, p_v_f2, p_v_in, p_v_out;
+  GemmPlan p_a_in, p_a_qkv, p_a_o, p_a_f1, p_a_f2, p_a_out;
+  int attn_splits = 1;
+
+  // TMA maps
+  CUtensorMap m_hv, m_ov, m_fv, m_xvin, m_w_qkv_v, m_w_o_v, m_w_f1_v, m_w_f2_v, m_w_vin, m_w_vout;
+  CUtensorMap m_w_in, m_w_qkv_a, m_w_o_a, m_w_f1_a, m_w_f2_a, m_w_out, m_ain, m_ha, m_oa, m_fa;
+
+  // events and streams
+  std::vector<cudaEvent_t> ev_kv, ev_kv_cap, ev_used;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_pre = nullptr, ev_post = nullptr;
+  cudaStream_t cap_v = nullptr, cap_a = nullptr;
+  std::map<long long, cudaGraphExec_t> graphs;
+  std::map<long long, int> launch_counts;
+  bool video_done = false;
+  int launches = 0;
+  std::string last_error;
+
+  // per-launch timing (wam_profile_chunk)
+  bool prof_on = false;
+  int cur_cls = 0;
+  struct ProfRec {
+    int cls;
+    cudaEvent_t a, b;
+  };
+  std::vector<ProfRec> prof;
+  std::vector<cudaEvent_t> prof_pool;
+  size_t prof_next = 0;
+};
+
+namespace {
+
+wam_status fail(wam_ctx* c, wam_status s, const char* fmt, ...) {
+  if (c) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    c->last_error = buf;
+  }
+  return s;
+}
+
+#define CK(expr)                                                                              \
+  do {                                                                                        \
+    cudaError_t e_ = (expr);                                                                  \
+    if (e_ != cudaSuccess) return fail(c, WAM_ERR_CUDA, "%s: %s (%s:%d)", #expr,              \
+                                       cudaGetErrorString(e_), __FILE__, __LINE__);           \
+  } while (0)
+
+// Records a timing event pair around the launches inside its scope when the
+// context is profiling (eager, one stream), tagged with the current class.
+struct ProfScope {
+  wam_ctx* c;
+  cudaStream_t s;
+  cudaEvent_t b = nullptr;
+  ProfScope(wam_ctx* c_, cudaStream_t s_) : c(c_), s(s_) {
+    if (!c->prof_on) return;
+    while (c->prof_pool.size() < c->prof_next + 2) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return;
+      c->prof_pool.push_back(e);
+    }
+    cudaEvent_t a = c->prof_pool[c->prof_next++];
+    b = c->prof_pool[c->prof_next++];
+    cudaEventRecord(a, s);
+    c->prof.push_back({c->cur_cls, a, b});
+  }
+  ~ProfScope() {
+    if (b) cudaEventRecord(b, s);
+  }
+};
+
+// ------------------------------------------------------------ parameters --
+void add_expert(wam_ctx* c, bool video) {
+  const Dims& d = c->d;
+  const int dm = video ? d.dv : d.da, F = video ? d.Fv : d.Fa, A = d.A;
+  const std::string p = video ? "video." : "action.";
+  ExpertIdx& ix = video ? c->ev : c->ea;
+  auto add = [&](const std::string& n, int rows, int cols, bool matrix, bool ones) {
+    PEntry e;
+    e.name = n;
+    e.rows = rows;
+    e.cols = cols;
+    e.matrix = matrix;
+    e.ones = ones;
+    e.ld = (matrix && d.bf16) ? (cols + 63) / 64 * 64 : cols;
+    e.off = 0;
+    c->params.push_back(e);
+    return (int)c->params.size() - 1;
+  };
+  ix.t1w = add(p + "t1.w", dm, 256, true, false);
+  ix.t1b = add(p + "t1.b", 1, dm, false, false);
+  ix.t2w = add(p + "t2.w", dm, dm, true, false);
+  ix.t2b = add(p + "t2.b", 1, dm, false, false);
+  ix.modw = add(p + "mod.w", 6 * dm, dm, true, false);
+  ix.modb = add(p + "mod.b", 1, 6 * dm, false, false);
+  if (video && d.Pv > 0) {
+    ix.inw = add(p + "in.w", dm, d.Pv, true, false);
+    ix.inb = add(p + "in.b", 1, dm, false, false);
+  }
+  if (!video) {
+    ix.inw = add(p + "in.w", dm, d.Pa, true, false);
+    ix.inb = add(p + "in.b", 1, dm, false, false);
+  }
+  const bool lora = !video && d.r > 0;
+  for (int i = 0; i < d.N; ++i) {
+    const std::string b = p + "blk" + std::to_string(i) + ".";
+    const int first = add(b + "T", 6, dm, false, false);
+    if (i == 0) ix.blk0 = first;
+    add(b + "qkv.w", 3 * A, dm, true, false);
+    add(b + "qkv.b", 1, 3 * A, false, false);
+    add(b + "qn.g", 1, A, false, true);
+    add(b + "kn.g", 1, A, false, true);
+    add(b + "o.w", dm, A, true, false);
+    add(b + "o.b", 1, dm, false, false);
+    add(b + "ffn1.w", F, dm, true, false);
+    add(b + "ffn1.b", 1, F, false, false);
+    add(b + "ffn2.w", dm, F, true, false);
+    add(b + "ffn2.b", 1, dm, false, false);
+    if (lora) {
+      add(b + "qkv.la", d.r, dm, true, false);
+      add(b + "qkv.lb", 3 * A, d.r, true, false);
+      add(b + "o.la", d.r, A, true, false);
+      add(b + "o.lb", dm, d.r, true, false);
+      add(b + "ffn1.la", d.r, dm, true, false);
+      add(b + "ffn1.lb", F, d.r, true, false);
+      add(b + "ffn2.la", d.r, F, true, false);
+      add(b + "ffn2.lb", dm, d.r, true, false);
+    }
+    if (i == 0) ix.per_blk = (int)c->params.size() - first;
+  }
+  if (video && c->cfg.video_has_output) {
+    ix.fng = add(p + "fn.g", 1, dm, false, true);
+    ix.outw = add(p + "out.w", d.Pv, dm, true, false);
+    ix.outb = add(p + "out.b", 1, d.Pv, false, false);
+  }
+  if (!video) {
+    ix.fng = add(p + "fn.g", 1, dm, false, true);
+    ix.outw = add(p + "out.w", d.Pa, dm, true, false);
+    ix.outb = add(p + "out.b", 1, d.Pa, false, false);
+  }
+}
+
+void layout_params(wam_ctx* c) {
+  size_t om = 0, ov = 0;
+  for (auto& e : c->params) {
+    if (e.matrix) {
+      e.off = om;
+      om += ((size_t)e.rows * e.ld + 127) / 128 * 128;
+    } else {
+      e.off = ov;
+      ov += (e.count() + 63) / 64 * 64;
+    }
+  }
+  c->wmat_elems = om;
+  c->wvec_elems = ov;
+}
+
+inline int blk(const ExpertIdx& x, int i, int local) { return x.blk0 + i * x.per_blk + local; }
+inline void* matp(wam_ctx* c, int idx) { return (char*)c->wmat + c->params[idx].off * c->esz; }
+inline float* vecp(wam_ctx* c, int idx) { return c->wvec + c->params[idx].off; }
+inline size_t blk_stride_bytes(wam_ctx* c, const ExpertIdx& x, int local) {
+  if (c->d.N < 2) return 0;
+  return (c->params[blk(x, 1, local)].off - c->params[blk(x, 0, local)].off) * c->esz;
+}
+inline void* kcache(wam_ctx* c, int i) {
+  const size_t per = (size_t)c->d.B * c->d.H * c->d.Ltot * c->d.Dh;
+  return (char*)c->kv + (size_t)(2 * i) * per * c->esz;
+}
+inline void* vcache(wam_ctx* c, int i) {
+  const size_t per = (size_t)c->d.B * c->d.H * c->d.Ltot * c->d.Dh;
+  return (char*)c->kv + (size_t)(2 * i + 1) * per * c->esz;
+}
+
+// ------------------------------------------------------------- planning ---
+GemmPlan plan_swap(int rows_w, int tokens, int K, int bn) {
+  GemmPlan p;
+  p.bn = bn;
+  const int tiles = ((rows_w + 127) / 128) * ((tokens + bn - 1) / bn);
+  const int kb = (K + 63) / 64;
+  int s = (148 + tiles - 1) / tiles;
+  const int min_kb = 3;  // keep each split a few k-blocks deep
+  if (s > kb / min_kb) s = kb / min_kb;
+  if (s < 1) s = 1;
+  p.splits = s;
+  return p;
+}
+
+size_t ws_floats(const GemmPlan& p, int rows_w, int tokens) {
+  if (p.splits <= 1) return 0;
+  const int tiles = ((rows_w + 127) / 128) * ((tokens + p.bn - 1) / p.bn);
+  return (size_t)tiles * p.splits * 128 * p.bn;
+}
+
+int tiles_of(const GemmPlan& p, int rows_w, int tokens) {
+  return ((rows_w + 127) / 128) * ((tokens + p.bn - 1) / p.bn);
+}
+
+// --------------------------------------------------------- GEMM wrappers --
+wam_status run_tc(wam_ctx* c, const CUtensorMap& A, const CUtensorMap& Bm, int rows_a, int rows_b, int K, int z_a,
+                  int z_b, const GemmPlan& p, bool swap, const EpiArgs& e, cudaStream_t s) {
+  TcGemm g;
+  g.map_a = &A;
+  g.map_b = &Bm;
+  g.rows_a = rows_a;
+  g.rows_b = rows_b;
+  g.K = K;
+  g.z_a = z_a;
+  g.z_b = z_b;
+  g.bn = p.bn;
+  g.splits = p.splits;
+  g.swap = swap;
+  g.ws = c->ws_gemm;
+  g.tickets = c->tk_gemm;
+  g.status = c->status;
+  c->launches++;
+  CK(launch_tc_gemm(g, e, s));
+  return WAM_OK;
+}
+
+EpiArgs epi_base(int kind, const float* bias, float* out_f32, void* out_act, int ld) {
+  EpiArgs e;
+  e.kind = kind;
+  e.bias = bias;
+  e.out_f32 = out_f32;
+  e.out_act = out_act;
+  e.ld_out = ld;
+  return e;
+}
+
+EpiArgs epi_qkv(wam_ctx* c, bool video, int i) {
+  const Dims& d = c->d;
+  const ExpertIdx& x = video ? c->ev : c->ea;
+  EpiArgs e = epi_base(kEpiQkv, vecp(c, blk(x, i, kQkvB)), nullptr, nullptr, 0);
+  e.gq = vecp(c, blk(x, i, kQnG));
+  e.gk = vecp(c, blk(x, i, kKnG));
+  e.rope_cos = c->rope_cos;
+  e.rope_sin = c->rope_sin;
+  e.q_out = video ? c->q_v : c->q_a;
+  e.k_cache = kcache(c, i);
+  e.v_cache = vcache(c, i);
+  e.seq_len = video ? d.Lv : d.La;
+  e.cache_len = d.Ltot;
+  e.cache_off = video ? 0 : d.Lv;
+  e.n_heads = d.H;
+  e.head_dim = d.Dh;
+  e.attn_dim = d.A;
+  return e;
+}
+
+// Linear layer of expert `video` block i (or a non-block layer when i < 0),
+// dispatched to the tcgen05 path (bf16) or the SIMT path (fp32).
+struct Lin {
+  const CUtensorMap* map_w;  // weight map (bf16)
+  const CUtensorMap* map_x;  // activation map (bf16)
+  const void* w;             // fp32 path: weight pointer
+  const void* x;             // fp32 path: activation pointer
+  int n_out, K;              // output features, reduction length
+  int z;                     // block index in the weight map
+  const GemmPlan* plan;
+};
+
+wam_status linear(wam_ctx* c, bool video, const Lin& L, int M, const EpiArgs& e_in, float* qkv_tmp, cudaStream_t s) {
+  const Dims& d = c->d;
+  ProfScope ps(c, s);
+  if (d.bf16) {
+    if (video)  // tokens on TMEM lanes
+      return run_tc(c, *L.map_x, *L.map_w, M, L.n_out, L.K, 0, L.z, *L.plan, false, e_in, s);
+    return run_tc(c, *L.map_w, *L.map_x, L.n_out, M, L.K, L.z, 0, *L.plan, true, e_in, s);
+  }
+  if (e_in.kind == kEpiQkv) {
+    EpiArgs st = epi_base(kEpiStoreF32, e_in.bias, qkv_tmp, nullptr, 3 * d.A);
+    c->launches++;
+    CK(launch_f32_gemm((const float*)L.x, (const float*)L.w, M, L.n_out, L.K, st, s));
+    c->launches++;
+    CK(launch_qkv_post_f32(qkv_tmp, M, e_in, s));
+    return WAM_OK;
+  }
+  c->launches++;
+  CK(launch_f32_gemm((const float*)L.x, (const float*)L.w, M, L.n_out, L.K, e_in, s));
+  return WAM_OK;
+}
+
+wam_status norm(wam_ctx* c, const float* x, void* h, int M, int dm, const float* sc, const float* sh, const float* g,
+                cudaStream_t s) {
+  c->launches++;
+  ProfScope ps(c, s);
+  CK(launch_norm_mod(x, h, c->d.bf16, M, dm, sc, sh, g, s));
+  return WAM_OK;
+}
+
+wam_status temb(wam_ctx* c, bool video, const float* t, cudaStream_t s) {
+  const ExpertIdx& x = video ? c->ev : c->ea;
+  TembArgs a;
+  a.t = t;
+  a.w1 = matp(c, x.t1w);
+  a.b1 = vecp(c, x.t1b);
+  a.w2 = matp(c, x.t2w);
+  a.b2 = vecp(c, x.t2b);
+  a.wm = matp(c, x.modw);
+  a.bm = vecp(c, x.modb);
+  a.T0 = vecp(c, blk(x, 0, kT));
+  a.T_stride = c->d.N > 1 ? c->params[blk(x, 1, kT)].off - c->params[blk(x, 0, kT)].off : 0;
+  a.mod = video ? c->mod_v : c->mod_a;
+  a.scratch = video ? c->temb_v : c->temb_a;
+  a.d = video ? c->d.dv : c->d.da;
+  a.n_blocks = c->d.N;
+  a.bf16 = c->d.bf16;
+  c->launches += 3;
+  ProfScope ps(c, s);
+  CK(launch_temb(a, s));
+  return WAM_OK;
+}
+
+wam_status attention(wam_ctx* c, bool video, int i, cudaStream_t s) {
+  const Dims& d = c->d;
+  AttnArgs a;
+  a.q = video ? c->q_v : c->q_a;
+  a.k = kcache(c, i);
+  a.v = vcache(c, i);
+  a.out = video ? c->o_v : c->o_a;
+  a.B = d.B;
+  a.H = d.H;
+  a.Dh = d.Dh;
+  a.Lq = video ? d.Lv : d.La;
+  a.Lk = video ? d.Lv : d.Lv + d.La;
+  a.Lcache = d.Ltot;
+  a.splits = video ? 1 : c->attn_splits;
+  a.ws = c->ws_attn;
+  a.tickets = c->tk_attn;
+  c->launches++;
+  ProfScope ps(c, s);
+  CK(d.bf16 ? launch_attention_bf16(a, s) : launch_attention_f32(a, s));
+  return WAM_OK;
+}
+
+#define RET(expr)                       \
+  do {                                  \
+    wam_status r_ = (expr);             \
+    if (r_ != WAM_OK) return r_;        \
+  } while (0)
+
+// ------------------------------------------------------------- experts ----
+// Video expert: P^v_i -> record(e_i) -> Attn^v_i -> R^v_i for every block.
+wam_status enqueue_video(wam_ctx* c, cudaStream_t s, const VideoIo* io, bool joint, cudaEvent_t* ev_ready,
+                         bool war_waits) {
+  const Dims& d = c->d;
+  const ExpertIdx& x = c->ev;
+  const bool has_out = c->cfg.video_has_output != 0;
+  c->cur_cls = WAM_PROF_VIDEO_IO;
+  if (joint) {
+    c->launches++;
+    ProfScope ps(c, s);
+    CK(launch_noise_video(io, c->x_sigma, d.bf16 ? c->x_vin : c->x_sigma, d.bf16, d.Mv, d.Pv, d.Pv, s));
+    Lin L{&c->m_w_vin, &c->m_xvin, matp(c, x.inw), c->x_sigma, d.dv, d.Pv, 0, &c->p_v_in};
+    RET(linear(c, true, L, d.Mv, epi_base(kEpiStoreF32, vecp(c, x.inb), c->x_v, nullptr, d.dv), nullptr, s));
+  } else {
+    c->launches++;
+    ProfScope ps(c, s);
+    CK(launch_init_video(io, c->x_v, d.B, d.Lc, d.Lvid, d.dv, s));
+  }
+  c->cur_cls = WAM_PROF_VIDEO_TEMB;
+  RET(temb(c, true, &io->t, s));
+  for (int i = 0; i < d.N; ++i) {
+    const float* mod = c->mod_v + (size_t)i * 6 * d.dv;
+    if (war_waits) CK(cudaStreamWaitEvent(s, c->ev_used[i], 0));
+    c->cur_cls = WAM_PROF_VIDEO_NORM;
+    RET(norm(c, c->x_v, c->h_v, d.Mv, d.dv, mod + d.dv, mod, nullptr, s));
+    c->cur_cls = WAM_PROF_VIDEO_QKV;
+    Lin Lq{&c->m_w_qkv_v, &c->m_hv, matp(c, blk(x, i, kQkvW)), c->h_v, 3 * d.A, d.dv, i, &c->p_v_qkv};
+    RET(linear(c, true, Lq, d.Mv, epi_qkv(c, true, i), c->qkv_tmp_v, s));
+    if (ev_ready) CK(cudaEventRecord(ev_ready[i], s));
+    if (i == d.N - 1 && !has_out) break;
+    c->cur_cls = WAM_PROF_VIDEO_ATTN;
+    RET(attention(c, true, i, s));
+    c->cur_cls = WAM_PROF_VIDEO_OPROJ;
+    EpiArgs eo = epi_base(kEpiGateRes, vecp(c, blk(x, i, kOB)), c->x_v, nullptr, d.dv);
+    eo.gate = mod + 2 * d.dv;
+    Lin Lo{&c->m_w_o_v, &c->m_ov, matp(c, blk(x, i, kOW)), c->o_v, d.dv, d.A, i, &c->p_v_o};
+    RET(linear(c, true, Lo, d.Mv, eo, nullptr, s));
+    c->cur_cls = WAM_PROF_VIDEO_NORM;
+    RET(norm(c, c->x_v, c->h_v, d.Mv, d.dv, mod + 4 * d.dv, mod + 3 * d.dv, nullptr, s));
+    c->cur_cls = WAM_PROF_VIDEO_FFN_UP;
+    Lin L1{&c->m_w_f1_v, &c->m_hv, matp(c, blk(x, i, kF1W)), c->h_v, d.Fv, d.dv, i, &c->p_v_f1};
+    RET(linear(c, true, L1, d.Mv, epi_base(kEpiGelu, vecp(c, blk(x, i, kF1B)), nullptr, c->f_v, d.Fv), nullptr, s));
+    c->cur_cls = WAM_PROF_VIDEO_FFN_DOWN;
+    EpiArgs e2 = epi_base(kEpiGateRes, vecp(c, blk(x, i, kF2B)), c->x_v, nullptr, d.dv);
+    e2.gate = mod + 5 * d.dv;
+    Lin L2{&c->m_w_f2_v, &c->m_fv, matp(c, blk(x, i, kF2W)), c->f_v, d.dv, d.Fv, i, &c->p_v_f2};
+    RET(linear(c, true, L2, d.Mv, e2, nullptr, s));
+  }
+  if (joint) {
+    c->cur_cls = WAM_PROF_VIDEO_IO;
+    RET(norm(c, c->x_v, c->h_v, d.Mv, d.dv, nullptr, nullptr, vecp(c, x.fng), s));
+    EpiArgs eo = epi_base(kEpiVideoOut, vecp(c, x.outb), nullptr, nullptr, d.Pv);
+    eo.vio = io;
+    eo.x_sigma = c->x_sigma;
+    Lin Lout{&c->m_w_vout, &c->m_hv, matp(c, x.outw), c->h_v, d.Pv, d.dv, 0, &c->p_v_out};
+    RET(linear(c, true, Lout, d.Mv, eo, nullptr, s));
+  }
+  return WAM_OK;
+}
+
+// One Euler step j of the action expert: P^a_i -> wait(e_i) -> Attn^a_i -> R^a_i.
+wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, int j, const cudaEvent_t* ev_wait,
+                               bool record_used) {
+  const Dims& d = c->d;
+  const ExpertIdx& x = c->ea;
+  c->cur_cls = WAM_PROF_ACTION_TEMB;
+  RET(temb(c, false, &io->sched[j], s));
+  c->cur_cls = WAM_PROF_ACTION_IO;
+  {
+    Lin L{&c->m_w_in, &c->m_ain, matp(c, x.inw), c->a_state, d.da, d.bf16 ? d.Kin : d.Pa, 0, &c->p_a_in};
+    RET(linear(c, false, L, d.Ma, epi_base(kEpiStoreF32, vecp(c, x.inb), c->x_a, nullptr, d.da), nullptr, s));
+  }
+  for (int i = 0; i < d.N; ++i) {
+    const float* mod = c->mod_a + (size_t)i * 6 * d.da;
+    c->cur_cls = WAM_PROF_ACTION_NORM;
+    RET(norm(c, c->x_a, c->h_a, d.Ma, d.da, mod + d.da, mod, nullptr, s));
+    c->cur_cls = WAM_PROF_ACTION_QKV;
+    Lin Lq{&c->m_w_qkv_a, &c->m_ha, matp(c, blk(x, i, kQkvW)), c->h_a, 3 * d.A, d.da, i, &c->p_a_qkv};
+    RET(linear(c, false, Lq, d.Ma, epi_qkv(c, false, i), c->qkv_tmp_a, s));
+    if (ev_wait) CK(cudaStreamWaitEvent(s, ev_wait[i], 0));
+    c->cur_cls = WAM_PROF_ACTION_ATTN;
+    RET(attention(c, false, i, s));
+    if (record_used) CK(cudaEventRecord(c->ev_used[i], s));
+    c->cur_cls = WAM_PROF_ACTION_OPROJ;
+    EpiArgs eo = epi_base(kEpiGateRes, vecp(c, blk(x, i, kOB)), c->x_a, nullptr, d.da);
+    eo.gate = mod + 2 * d.da;
+    Lin Lo{&c->m_w_o_a, &c->m_oa, matp(c, blk(x, i, kOW)), c->o_a, d.da, d.A, i, &c->p_a_o};
+    RET(linear(c, false, Lo, d.Ma, eo, nullptr, s));
+    c->cur_cls = WAM_PROF_ACTION_NORM;
+    RET(norm(c, c->x_a, c->h_a, d.Ma, d.da, mod + 4 * d.da, mod + 3 * d.da, nullptr, s));
+    c->cur_cls = WAM_PROF_ACTION_FFN_UP;
+    Lin L1{&c->m_w_f1_a, &c->m_ha, matp(c, blk(x, i, kF1W)), c->h_a, d.Fa, d.da, i, &c->p_a_f1};
+    RET(linear(c, false, L1, d.Ma, epi_base(kEpiGelu, vecp(c, blk(x, i, kF1B)), nullptr, c->f_a, d.Fa), nullptr, s));
+    c->cur_cls = WAM_PROF_ACTION_FFN_DOWN;
+    EpiArgs e2 = epi_base(kEpiGateRes, vecp(c, blk(x, i, kF2B)), c->x_a, nullptr, d.da);
+    e2.gate = mod + 5 * d.da;
+    Lin L2{&c->m_w_f2_a, &c->m_fa, matp(c, blk(x, i, kF2W)), c->f_a, d.da, d.Fa, i, &c->p_a_f2};
+    RET(linear(c, false, L2, d.Ma, e2, nullptr, s));
+  }
+  c->cur_cls = WAM_PROF_ACTION_IO;
+  RET(norm(c, c->x_a, c->h_a, d.Ma, d.da, nullptr, nullptr, vecp(c, x.fng), s));
+  EpiArgs ee = epi_base(kEpiEuler, vecp(c, x.outb), c->a_state, nullptr, d.Pa);
+  ee.aio = io;
+  ee.step = j;
+  ee.a_next = d.bf16 ? c->a_in : nullptr;
+  ee.a_next_ld = d.Kin;
+  Lin Lout{&c->m_w_out, &c->m_ha, matp(c, x.outw), c->h_a, d.Pa, d.da, 0, &c->p_a_out};
+  RET(linear(c, false, Lout, d.Ma, ee, nullptr, s));
+  return WAM_OK;
+}
+
+// A whole chunk: video once, then `steps` Euler steps (or the joint one-step).
+wam_status enqueue_chunk(wam_ctx* c, int steps, int mode, bool joint, cudaStream_t sv, cudaStream_t sa,
+                         cudaEvent_t* ev_kv) {
+  const Dims& d = c->d;
+  const bool cewp = mode == WAM_SCHED_CEWP;
+  cudaStream_t s_act = cewp ? sa : sv;
+  if (cewp) {
+    CK(cudaEventRecord(c->ev_fork, sv));
+    CK(cudaStreamWaitEvent(sa, c->ev_fork, 0));
+  }
+  // action-side prologue (no dependence on the video expert)
+  c->launches++;
+  c->cur_cls = WAM_PROF_ACTION_IO;
+  {
+  ProfScope ps(c, s_act);
+  if (joint)
+    CK(launch_noise_action(c->aio_chunk, c->a_state, d.bf16 ? c->a_in : nullptr, d.bf16, d.Ma, d.Pa, d.Kin, s_act));
+  else
+    CK(launch_init_action(c->aio_chunk, c->a_state, d.bf16 ? c->a_in : nullptr, d.bf16, d.Ma, d.Pa, d.Kin, s_act));
+  }
+  if (cewp) {
+    // Enqueue the two experts interleaved block by block is not needed: the
+    // streams run concurrently; the per-block events order Attn^a_i after P^v_i.
+    RET(enqueue_video(c, sv, c->vio_chunk, joint, ev_kv, false));
+    for (int j = 0; j < steps; ++j) RET(enqueue_action_step(c, sa, c->aio_chunk, j, j == 0 ? ev_kv : nullptr, false));
+  } else {
+    RET(enqueue_video(c, sv, c->vio_chunk, joint, nullptr, false));
+    for (int j = 0; j < steps; ++j) RET(enqueue_action_step(c, sv, c->aio_chunk, j, nullptr, false));
+  }
+  c->launches++;
+  {
+    c->cur_cls = WAM_PROF_ACTION_IO;
+    ProfScope ps(c, s_act);
+    CK(launch_copy_out(c->aio_chunk, c->a_state, d.Ma * d.Pa, s_act));
+  }
+  if (cewp) {
+    CK(cudaEventRecord(c->ev_join, sa));
+    CK(cudaStreamWaitEvent(sv, c->ev_join, 0));
+  }
+  return WAM_OK;
+}
+
+wam_status set_chunk_io(wam_ctx* c, const VideoIo& v, const ActionIo& a, cudaStream_t sv) {
+  if (!c->vio_valid || memcmp(&v, &c->vio_shadow, sizeof v) != 0) {
+    CK(launch_set_video_io(c->vio_chunk, v, sv));
+    c->vio_shadow = v;
+    c->vio_valid = true;
+  }
+  if (!c->aio_valid || memcmp(&a, &c->aio_shadow, sizeof a) != 0) {
+    CK(launch_set_action_io(c->aio_chunk, a, sv));
+    c->aio_shadow = a;
+    c->aio_valid = true;
+  }
+  return WAM_OK;
+}
+
+wam_status run_chunk(wam_ctx* c, int steps, int mode, int use_graph, bool joint, cudaStream_t sv, cudaStream_t sa) {
+  const long long key = ((long long)steps << 8) | (mode << 1) | (joint ? 1 : 0);
+  if (!use_graph) {
+    c->launches = 0;
+    RET(enqueue_chunk(c, steps, mode, joint, sv, mode == WAM_SCHED_CEWP ? sa : sv, c->ev_kv.data()));
+    c->launch_counts[key] = c->launches;
+  } else {
+    auto it = c->graphs.find(key);
+    if (it == c->graphs.end()) {
+      cudaGraph_t graph = nullptr;
+      c->launches = 0;
+      CK(cudaStreamBeginCapture(c->cap_v, cudaStreamCaptureModeThreadLocal));
+      wam_status st = enqueue_chunk(c, steps, mode, joint, c->cap_v, c->cap_a, c->ev_kv_cap.data());
+      cudaError_t ce = cudaStreamEndCapture(c->cap_v, &graph);
+      if (st != WAM_OK) {
+        if (graph) cudaGraphDestroy(graph);
+        return st;
+      }
+      CK(ce);
+      cudaGraphExec_t exec = nullptr;
+      cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
+      cudaGraphDestroy(graph);
+      CK(ie);
+      it = c->graphs.emplace(key, exec).first;
+      c->launch_counts[key] = c->launches;
+    }
+    CK(cudaGraphLaunch(it->second, sv));
+  }
+  if (mode == WAM_SCHED_CEWP && sa != sv) {
+    CK(cudaEventRecord(c->ev_post, sv));
+    CK(cudaStreamWaitEvent(sa, c->ev_post, 0));
+  }
+  return WAM_OK;
+}
+
+bool valid_schedule(const float* t, int S) {
+  for (int j = 0; j <= S; ++j)
+    if (!(t[j] >= 0.f && t[j] <= 1.f)) return false;
+  for (int j = 0; j < S; ++j)
+    if (!(t[j] > t[j + 1])) return false;
+  return true;
+}
+
+template <typename T>
+wam_status dalloc(wam_ctx* c, T** p, size_t bytes) {
+  if (bytes == 0) bytes = 256;
+  cudaError_t e = cudaMalloc((void**)p, bytes);
+  if (e == cudaErrorMemoryAllocation) {
+    cudaGetLastError();
+    return fail(c, WAM_ERR_OOM, "cudaMalloc(%zu) failed: out of device memory", bytes);
+  }
+  CK(e);
+  CK(cudaMemset(*p, 0, bytes));
+  return WAM_OK;
+}
+
+bool check_cfg(const wam_config* g, std::string* why) {
+  auto bad = [&](const char* m) {
+    *why = m;
+    return false;
+  };
+  if (g->n_blocks < 1 || g->d_video < 8 || g->d_action < 8 || g->n_heads < 1 || g->head_dim < 2) return bad("sizes must be positive");
+  if (g->l_video < 1 || g->l_action < 1 || g->l_cond < 0 || g->batch < 1 || g->action_dim < 1) return bad("token counts");
+  if (g->head_dim % 2) return bad("head_dim must be even");
+  if (g->d_video % 8 || g->d_action % 8 || g->ffn_video % 8 || g->ffn_action % 8) return bad("widths must be multiples of 8");
+  if (g->video_has_output && g->video_patch_dim <= 0) return bad("a video output needs patch input");
+  if (g->video_patch_dim > 0 && g->l_cond != 0) return bad("patch input takes no conditioning tokens");
+  if (g->lora_rank < 0) return bad("lora_rank");
+  if (g->dtype == WAM_BF16) {
+    const int A = g->n_heads * g->head_dim;
+    if (g->head_dim != 64) return bad("bf16 path needs head_dim 64");
+    if (g->d_video % 64 || g->d_action % 64 || g->ffn_video % 128 || g->ffn_action % 64 || A % 128)
+      return bad("bf16 path needs widths in multiples of 64 (ffn_video, attention width: 128)");
+    if (g->video_patch_dim % 64) return bad("bf16 path needs video_patch_dim multiple of 64");
+    if (g->batch * g->l_action > 256) return bad("bf16 path supports at most 256 action tokens per chunk");
+    if (g->l_action > 64) return bad("bf16 path supports at most 64 action tokens per sample");
+    if (g->lora_rank > 0 && g->lora_rank % 64) return bad("lora_rank must be a multiple of 64");
+  } else if (g->dtype == WAM_FP32) {
+    if (g->head_dim > 64 || (g->head_dim != 16 && g->head_dim != 32 && g->head_dim != 64))
+      return bad("fp32 path supports head_dim 16, 32, 64");
+    if (g->d_video % 4 || g->d_action % 4) return bad("fp32 widths must be multiples of 4");
+  } else {
+    return bad("dtype");
+  }
+  return true;
+}
+
+}  // namespace
+
+// ===================================================================== ABI ==
+extern "C" {
+
+wam_status wam_preset(int k, wam_config* o) {
+  if (!o) return WAM_ERR_INVALID_ARG;
+  wam_config g{};
+  g.action_dim = 30;
+  g.batch = 1;
+  g.lora_scale = 1.0f;
+  switch (k) {
+    case 1:
+      g.n_blocks = 2; g.d_video = 64; g.d_action = 64; g.n_heads = 4; g.head_dim = 16;
+      g.ffn_video = 256; g.ffn_action = 256; g.l_cond = 0; g.l_video = 64; g.l_action = 16;
+      g.dtype = WAM_FP32;
+      break;
+    case 2:
+    case 3:
+    case 4:
+      g.n_blocks = 28; g.d_video = 1536; g.d_action = 768; g.n_heads = 24; g.head_dim = 64;
+      g.ffn_video = 6144; g.ffn_action = 3072; g.l_cond = 64; g.l_video = 1024; g.l_action = 32;
+      g.dtype = WAM_BF16;
+      if (k == 4) {
+        g.l_video = 2048;
+        g.batch = 8;
+      }
+      break;
+    case 5:
+      g.n_blocks = 30; g.d_video = 1536; g.d_action = 1536; g.n_heads = 24; g.head_dim = 64;
+      g.ffn_video = 6144; g.ffn_action = 6144; g.l_cond = 0; g.l_video = 1024; g.l_action = 16;
+      g.video_patch_dim = 192; g.lora_rank = 128; g.video_has_output = 1; g.dtype = WAM_BF16;
+      break;
+    default:
+      return WAM_ERR_INVALID_ARG;
+  }
+  *o = g;
+  return WAM_OK;
+}
+
+const char* wam_status_str(wam_status s) {
+  switch (s) {
+    case WAM_OK: return "ok";
+    case WAM_ERR_INVALID_ARG: return "invalid argument";
+    case WAM_ERR_UNSUPPORTED: return "unsupported";
+    case WAM_ERR_OOM: return "out of device memory";
+    case WAM_ERR_CUDA: return "CUDA error";
+    case WAM_ERR_TIMEOUT: return "device wait timed out";
+    case WAM_ERR_STATE: return "invalid call order";
+  }
+  return "unknown status";
+}
+
+const char* wam_last_error(wam_ctx* c) { return c ? c->last_error.c_str() : ""; }
+
+void wam_destroy(wam_ctx* c) {
+  if (!c) return;
+  cudaSetDevice(c->device);
+  cudaDeviceSynchronize();
+  for (auto& kv : c->graphs) cudaGraphExecDestroy(kv.second);
+  for (auto* v : {&c->ev_kv, &c->ev_kv_cap, &c->ev_used})
+    for (auto e : *v) cudaEventDestroy(e);
+  for (auto e : {c->ev_fork, c->ev_join, c->ev_pre, c->ev_post})
+    if (e) cudaEventDestroy(e);
+  for (auto e : c->prof_pool) cudaEventDestroy(e);
+  if (c->cap_v) cudaStreamDestroy(c->cap_v);
+  if (c->cap_a) cudaStreamDestroy(c->cap_a);
+  void* bufs[] = {c->wmat, c->wvec, c->x_v, c->x_a, c->a_state, c->x_sigma, c->h_v, c->q_v, c->o_v, c->f_v,
+                  c->x_vin, c->h_a, c->q_a, c->o_a, c->f_a, c->a_in, c->qkv_tmp_v, c->qkv_tmp_a, c->kv,
+                  c->mod_v, c->mod_a, c->temb_v, c->temb_a, c->rope_cos, c->rope_sin, c->ws_gemm, c->tk_gemm,
+                  c->ws_attn, c->tk_attn, c->status, c->vio_chunk, c->vio_eager, c->aio_chunk, c->aio_eager,
+                  c->h_video, c->h_cond, c->h_noise, c->h_out, c->j_vout, c->j_aout};
+  for (void* p : bufs)
+    if (p) cudaFree(p);
+  delete c;
+}
+
+wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
+  if (!cfg || !out) return WAM_ERR_INVALID_ARG;
+  std::string why;
+  if (!check_cfg(cfg, &why)) return WAM_ERR_INVALID_ARG;
+  if (cfg->lora_rank > 0 && cfg->dtype == WAM_BF16) return WAM_ERR_UNSUPPORTED;
+  std::unique_ptr<wam_ctx> holder(new wam_ctx());
+  wam_ctx* c = holder.get();
+  c->cfg = *cfg;
+  CK(cudaGetDevice(&c->device));
+  CK(prepare_tc_gemm());
+  Dims& d = c->d;
+  d.N = cfg->n_blocks; d.dv = cfg->d_video; d.da = cfg->d_action; d.H = cfg->n_heads; d.Dh = cfg->head_dim;
+  d.A = d.H * d.Dh; d.Fv = cfg->ffn_video; d.Fa = cfg->ffn_action; d.Lc = cfg->l_cond; d.Lvid = cfg->l_video;
+  d.Lv = d.Lc + d.Lvid; d.La = cfg->l_action; d.Pa = cfg->action_dim; d.Pv = cfg->video_patch_dim;
+  d.B = cfg->batch; d.r = cfg->lora_rank; d.Ltot = d.Lv + d.La; d.Mv = d.B * d.Lv; d.Ma = d.B * d.La;
+  d.bf16 = cfg->dtype == WAM_BF16;
+  d.Kin = d.bf16 ? (d.Pa + 63) / 64 * 64 : d.Pa;
+  c->esz = d.bf16 ? 2 : 4;
+
+  add_expert(c, true);
+  add_expert(c, false);
+  layout_params(c);
+
+  RET(dalloc(c, &c->wmat, c->wmat_elems * c->esz));
+  RET(dalloc(c, &c->wvec, c->wvec_elems * sizeof(float)));
+  for (size_t p = 0; p < c->params.size(); ++p) {
+    const PEntry& e = c->params[p];
+    void* dst = e.matrix ? matp(c, (int)p) : (void*)vecp(c, (int)p);
+    CK(launch_gen_param(seed, p, e.count(), 0.02, e.ones, d.bf16, dst, e.matrix && d.bf16, e.cols,
+                        e.matrix ? e.ld : e.cols, 0));
+  }
+
+  const size_t ae = c->esz;
+  RET(dalloc(c, &c->x_v, (size_t)d.Mv * d.dv * 4));
+  RET(dalloc(c, &c->h_v, (size_t)d.Mv * d.dv * ae));
+  RET(dalloc(c, &c->q_v, (size_t)d.Mv * d.A * ae));
+  RET(dalloc(c, &c->o_v, (size_t)d.Mv * d.A * ae));
+  RET(dalloc(c, &c->f_v, (size_t)d.Mv * d.Fv * ae));
+  RET(dalloc(c, &c->x_a, (size_t)d.Ma * d.da * 4));
+  RET(dalloc(c, &c->h_a, (size_t)d.Ma * d.da * ae));
+  RET(dalloc(c, &c->q_a, (size_t)d.Ma * d.A * ae));
+  RET(dalloc(c, &c->o_a, (size_t)d.Ma * d.A * ae));
+  RET(dalloc(c, &c->f_a, (size_t)d.Ma * d.Fa * ae));
+  RET(dalloc(c, &c->a_state, (size_t)d.Ma * d.Pa * 4));
+  RET(dalloc(c, &c->a_in, (size_t)d.Ma * d.Kin * ae));
+  if (d.Pv > 0) {
+    RET(dalloc(c, &c->x_sigma, (size_t)d.Mv * d.Pv * 4));
+    RET(dalloc(c, &c->x_vin, (size_t)d.Mv * d.Pv * ae));
+  }
+  if (!d.bf16) {
+    RET(dalloc(c, &c->qkv_tmp_v, (size_t)d.Mv * 3 * d.A * 4));
+    RET(dalloc(c, &c->qkv_tmp_a, (size_t)d.Ma * 3 * d.A * 4));
+  }
+  RET(dalloc(c, &c->kv, (size_t)2 * d.N * d.B * d.H * d.Ltot * d.Dh * ae));
+  RET(dalloc(c, &c->mod_v, (size_t)d.N * 6 * d.dv * 4));
+  RET(dalloc(c, &c->mod_a, (size_t)d.N * 6 * d.da * 4));
+  RET(dalloc(c, &c->temb_v, (size_t)(256 + 2 * d.dv) * 4));
+  RET(dalloc(c, &c->temb_a, (size_t)(256 + 2 * d.da) * 4));
+  RET(dalloc(c, &c->rope_cos, (size_t)d.Ltot * d.Dh / 2 * 4));
+  RET(dalloc(c, &c->rope_sin, (size_t)d.Ltot * d.Dh / 2 * 4));
+  RET(dalloc(c, &c->status, 256));
+  RET(dalloc(c, &c->vio_chunk, sizeof(VideoIo)));
+  RET(dalloc(c, &c->vio_eager, sizeof(VideoIo)));
+  RET(dalloc(c, &c->aio_chunk, sizeof(ActionIo)));
+  RET(dalloc(c, &c->aio_eager, sizeof(ActionIo)));
+  CK(launch_rope_table(c->rope_cos, c->rope_sin, d.Ltot, d.Dh, 0));
+
+  // GEMM plans (bf16 path) and workspaces
+  size_t ws = 0;
+  int tiles = 1;
+  if (d.bf16) {
+    c->p_v_qkv = {128, 1};
+    c->p_v_o = {128, 1};
+    c->p_v_f1 = {256, 1};
+    c->p_v_f2 = {128, 1};
+    c->p_v_in = {128, 1};
+    c->p_v_out = {64, 1};
+    const int bn_a = d.Ma <= 32 ? 32 : (d.Ma <= 64 ? 64 : (d.Ma <= 128 ? 128 : 256));
+    c->p_a_in = plan_swap(d.da, d.Ma, d.Kin, bn_a);
+    c->p_a_qkv = plan_swap(3 * d.A, d.Ma, d.da, bn_a);
+    c->p_a_o = plan_swap(d.da, d.Ma, d.A, bn_a);
+    c->p_a_f1 = plan_swap(d.Fa, d.Ma, d.da, bn_a);
+    c->p_a_f2 = plan_swap(d.da, d.Ma, d.Fa, bn_a);
+    c->p_a_out = plan_swap(d.Pa, d.Ma, d.da, bn_a);
+    struct {
+      GemmPlan* p;
+      int rows;
+    } aps[] = {{&c->p_a_in, d.da}, {&c->p_a_qkv, 3 * d.A}, {&c->p_a_o, d.da},
+               {&c->p_a_f1, d.Fa}, {&c->p_a_f2, d.da},     {&c->p_a_out, d.Pa}};
+    for (auto& a : aps) {
+      ws = std::max(ws, ws_floats(*a.p, a.rows, d.Ma));
+      tiles = std::max(tiles, tiles_of(*a.p, a.rows, d.Ma));
+    }
+    c->attn_splits = std::max(1, (d.Lv + d.La + 127) / 128);
+  }
+  RET(dalloc(c, &c->ws_gemm, ws * 4));
+  RET(dalloc(c, &c->tk_gemm, (size_t)tiles * 4));
+  RET(dalloc(c, &c->ws_attn, attention_ws_floats(d.B, d.H, d.Dh, d.La, c->attn_splits) * 4));
+  RET(dalloc(c, &c->tk_attn, (size_t)d.B * d.H * 4));
+
+  if (d.bf16) {
+    bool ok = true;
+    auto wmap = [&](CUtensorMap* m, const ExpertIdx& x, int local, int rows, int K, int box) {
+      ok = ok && make_tmap_3d(m, matp(c, blk(x, 0, local)), K, rows, d.N, blk_stride_bytes(c, x, local), box);
+    };
+    auto amap = [&](CUtensorMap* m, const void* p, int rows, int K, int box) {
+      ok = ok && make_tmap_3d(m, p, K, rows, 1, 0, box);
+    };
+    const int bnv_qkv = c->p_v_qkv.bn, bnv_o = c->p_v_o.bn, bnv_f1 = c->p_v_f1.bn, bnv_f2 = c->p_v_f2.bn;
+    const int bna = c->p_a_qkv.bn;
+    amap(&c->m_hv, c->h_v, d.Mv, d.dv, 128);
+    amap(&c->m_ov, c->o_v, d.Mv, d.A, 128);
+    amap(&c->m_fv, c->f_v, d.Mv, d.Fv, 128);
+    wmap(&c->m_w_qkv_v, c->ev, kQkvW, 3 * d.A, d.dv, bnv_qkv);
+    wmap(&c->m_w_o_v, c->ev, kOW, d.dv, d.A, bnv_o);
+    wmap(&c->m_w_f1_v, c->ev, kF1W, d.Fv, d.dv, bnv_f1);
+    wmap(&c->m_w_f2_v, c->ev, kF2W, d.dv, d.Fv, bnv_f2);
+    if (d.Pv > 0) {
+      amap(&c->m_xvin, c->x_vin, d.Mv, d.Pv, 128);
+      amap(&c->m_w_vin, matp(c, c->ev.inw), d.dv, d.Pv, c->p_v_in.bn);
+    }
+    if (cfg->video_has_output) amap(&c->m_w_vout, matp(c, c->ev.outw), d.Pv, d.dv, c->p_v_out.bn);
+    amap(&c->m_w_in, matp(c, c->ea.inw), d.da, d.Kin, 128);
+    wmap(&c->m_w_qkv_a, c->ea, kQkvW, 3 * d.A, d.da, 128);
+    wmap(&c->m_w_o_a, c->ea, kOW, d.da, d.A, 128);
+    wmap(&c->m_w_f1_a, c->ea, kF1W, d.Fa, d.da, 128);
+    wmap(&c->m_w_f2_a, c->ea, kF2W, d.da, d.Fa, 128);
+    amap(&c->m_w_out, matp(c, c->ea.outw), d.Pa, d.da, 128);
+    amap(&c->m_ain, c->a_in, d.Ma, d.Kin, bna);
+    amap(&c->m_ha, c->h_a, d.Ma, d.da, bna);
+    amap(&c->m_oa, c->o_a, d.Ma, d.A, bna);
+    amap(&c->m_fa, c->f_a, d.Ma, d.Fa, bna);
+    if (!ok) return fail(c, WAM_ERR_CUDA, "tensor map creation failed");
+  }
+
+  c->ev_kv.resize(d.N);
+  c->ev_kv_cap.resize(d.N);
+  c->ev_used.resize(d.N);
+  for (int i = 0; i < d.N; ++i) {
+    CK(cudaEventCreateWithFlags(&c->ev_kv[i], cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&c->ev_kv_cap[i], cudaEventDisableTiming));
+    CK(cudaEventCreateWithFlags(&c->ev_used[i], cudaEventDisableTiming));
+  }
+  for (auto* e : {&c->ev_fork, &c->ev_join, &c->ev_pre, &c->ev_post})
+    CK(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
+  CK(cudaStreamCreateWithFlags(&c->cap_v, cudaStreamNonBlocking));
+  CK(cudaStreamCreateWithFlags(&c->cap_a, cudaStreamNonBlocking));
+  CK(cudaDeviceSynchronize());
+  *out = holder.release();
+  return WAM_OK;
+}
+
+wam_status wam_video_forward(wam_ctx* c, const float* video, const float* cond, float t_video, void* stream) {
+  if (!c || !video || (c->d.Lc > 0 && !cond) || c->d.Pv > 0 || !(t_video >= 0.f && t_video <= 1.f))
+    return fail(c, WAM_ERR_INVALID_ARG, "wam_video_forward: bad arguments");
+  cudaStream_t s = (cudaStream_t)stream;
+  VideoIo v{};
+  v.video = video;
+  v.cond = cond;
+  v.t = t_video;
+  CK(launch_set_video_io(c->vio_eager, v, s));
+  RET(enqueue_video(c, s, c->vio_eager, false, c->ev_kv.data(), true));
+  c->video_done = true;
+  return WAM_OK;
+}
+
+wam_status wam_action_step(wam_ctx* c, float* actions, float t_from, float t_to, void* stream) {
+  if (!c || !actions) return fail(c, WAM_ERR_INVALID_ARG, "wam_action_step: null argument");
+  if (!(t_from > t_to && t_to >= 0.f && t_from <= 1.f))
+    return fail(c, WAM_ERR_INVALID_ARG, "wam_action_step: need 1 >= t_from > t_to >= 0");
+  if (!c->video_done) return fail(c, WAM_ERR_STATE, "wam_action_step before wam_video_forward");
+  cudaStream_t s = (cudaStream_t)stream;
+  const Dims& d = c->d;
+  ActionIo a{};
+  a.a_in = actions;
+  a.a_out = actions;
+  a.sched[0] = t_from;
+  a.sched[1] = t_to;
+  a.steps = 1;
+  CK(launch_set_action_io(c->aio_eager, a, s));
+  CK(launch_init_action(c->aio_eager, c->a_state, d.bf16 ? c->a_in : nullptr, d.bf16, d.Ma, d.Pa, d.Kin, s));
+  RET(enqueue_action_step(c, s, c->aio_eager, 0, c->ev_kv.data(), true));
+  CK(launch_copy_out(c->aio_eager, c->a_state, d.Ma * d.Pa, s));
+  return WAM_OK;
+}
+
+wam_status wam_infer_chunk(wam_ctx* c, const float* video, const float* cond, const float* noise, float* out, int S,
+                           const float* t_sched, int mode, int use_graph, void* stream_video, void* stream_action) {
+  if (!c) return WAM_ERR_INVALID_ARG;
+  if (!video || !noise || !out || (c->d.Lc > 0 && !cond) || c->d.Pv > 0)
+    return fail(c, WAM_ERR_INVALID_ARG, "wam_infer_chunk: null buffer or patch-input model");
+  if (S < 1 || S > kMaxSteps) return fail(c, WAM_ERR_INVALID_ARG, "wam_infer_chunk: S out of range");
+  if (mode != WAM_SCHED_SEQUENTIAL && mode != WAM_SCHED_CEWP)
+    return fail(c, WAM_ERR_INVALID_ARG, "wam_infer_chunk: bad mode");
+  ActionIo a{};
+  for (int j = 0; j <= S; ++j) a.sched[j] = t_sched ? t_sched[j] : (float)(S - j) / (float)S;
+  if (!valid_schedule(a.sched, S)) return fail(c, WAM_ERR_INVALID_ARG, "wam_infer_chunk: schedule not decreasing in [0,1]");
+  a.steps = S;
+  a.a_in = noise;
+  a.a_out = out;
+  VideoIo v{};
+  v.video = video;
+  v.cond = cond;
+  v.t = 0.f;
+  cudaStream_t sv = (cudaStream_t)stream_video, sa = (cudaStream_t)stream_action;
+  if (mode == WAM_SCHED_CEWP && sa == sv) return fail(c, WAM_ERR_INVALID_ARG, "CEWP needs two distinct streams");
+  CK(cudaEventRecord(c->ev_pre, sa));
+  CK(cudaStreamWaitEvent(sv, c->ev_pre, 0));
+  RET(set_chunk_io(c, v, a, sv));
+  return run_chunk(c, S, mode, use_graph, false, sv, sa);
+}
+
+wam_status wam_infer_chunk_host(wam_ctx* c, const float* hv, const float* hc, const float* hn, float* hout, int S,
+                                const float* t_sched, int mode, int use_graph, void* stream_video, void* stream_action) {
+  if (!c || !hv || !hn || !hout || (c->d.Lc > 0 && !hc)) return fail(c, WAM_ERR_INVALID_ARG, "null host buffer");
+  const Dims& d = c->d;
+  const size_t nv = (size_t)d.B * d.Lvid * d.dv, nc = (size_t)d.B * d.Lc * d.dv, nn = (size_t)d.Ma * d.Pa;
+  if (!c->h_video) {
+    RET(dalloc(c, &c->h_video, nv * 4));
+    RET(dalloc(c, &c->h_cond, nc * 4));
+    RET(dalloc(c, &c->h_noise, nn * 4));
+    RET(dalloc(c, &c->h_out, nn * 4));
+  }
+  cudaStream_t sv = (cudaStream_t)stream_video;
+  CK(cudaMemcpyAsync(c->h_video, hv, nv * 4, cudaMemcpyHostToDevice, sv));
+  if (nc) CK(cudaMemcpyAsync(c->h_cond, hc, nc * 4, cudaMemcpyHostToDevice, sv));
+  CK(cudaMemcpyAsync(c->h_noise, hn, nn * 4, cudaMemcpyHostToDevice, sv));
+  RET(wam_infer_chunk(c, c->h_video, nc ? c->h_cond : nullptr, c->h_noise, c->h_out, S, t_sched, mode, use_graph,
+                      stream_video, stream_action));
+  CK(cudaMemcpyAsync(hout, c->h_out, nn * 4, cudaMemcpyDeviceToHost, sv));
+  CK(cudaStreamSynchronize(sv));
+  return WAM_OK;
+}
+
+wam_status wam_joint_one_step(wam_ctx* c, const float* vclean, const float* veps, const float* aclean,
+                              const float* aeps, float u_v, float u_a, float s_v, float s_a, float* vout, float* aout,
+                              int mode, int use_graph, void* stream_video, void* stream_action) {
+  if (!c) return WAM_ERR_INVALID_ARG;
+  if (c->d.Pv <= 0 || !c->cfg.video_has_output)
+    return fail(c, WAM_ERR_UNSUPPORTED, "wam_joint_one_step needs a patch-input model with a video output");
+  if (!vclean || !veps || !aclean || !aeps || !vout || !aout || !(u_v >= 0.f && u_v <= 1.f) ||
+      !(u_a > 0.f && u_a <= 1.f) || !(s_v > 0.f) || !(s_a > 0.f))
+    return fail(c, WAM_ERR_INVALID_ARG, "wam_joint_one_step: bad arguments");
+  cudaStream_t sv = (cudaStream_t)stream_video, sa = (cudaStream_t)stream_action;
+  if (mode == WAM_SCHED_CEWP && sa == sv) return fail(c, WAM_ERR_INVALID_ARG, "CEWP needs two distinct streams");
+  VideoIo v{};
+  v.video = vclean;
+  v.eps = veps;
+  v.video_out = vout;
+  v.u = u_v;
+  v.shift = s_v;
+  ActionIo a{};
+  a.a_in = aeps;
+  a.a_clean = aclean;
+  a.a_out = aout;
+  a.u = u_a;
+  a.shift = s_a;
+  a.steps = 1;
+  CK(cudaEventRecord(c->ev_pre, sa));
+  CK(cudaStreamWaitEvent(sv, c->ev_pre, 0));
+  RET(set_chunk_io(c, v, a, sv));
+  return run_chunk(c, 1, mode, use_graph, true, sv, sa);
+}
+
+wam_status wam_profile_chunk(wam_ctx* c, const float* video, const float* cond, const float* noise, float* out, int S,
+                             void* stream, float* host_ms, int* host_counts) {
+  if (!c || !host_ms || !host_counts) return WAM_ERR_INVALID_ARG;
+  if (!video || !noise || !out || (c->d.Lc > 0 && !cond) || c->d.Pv > 0 || S < 1 || S > kMaxSteps)
+    return fail(c, WAM_ERR_INVALID_ARG, "wam_profile_chunk: bad arguments");
+  cudaStream_t s = (cudaStream_t)stream;
+  ActionIo a{};
+  for (int j = 0; j <= S; ++j) a.sched[j] = (float)(S - j) / (float)S;
+  a.steps = S;
+  a.a_in = noise;
+  a.a_out = out;
+  VideoIo v{};
+  v.video = video;
+  v.cond = cond;
+  RET(set_chunk_io(c, v, a, s));
+  c->prof.clear();
+  c->prof_next = 0;
+  c->prof_on = true;
+  c->launches = 0;
+  wam_status st = enqueue_chunk(c, S, WAM_SCHED_SEQUENTIAL, false, s, s, c->ev_kv.data());
+  c->prof_on = false;
+  RET(st);
+  CK(cudaStreamSynchronize(s));
+  for (int k = 0; k < WAM_PROF_CLASSES; ++k) {
+    host_ms[k] = 0.f;
+    host_counts[k] = 0;
+  }
+  for (auto& r : c->prof) {
+    float ms = 0.f;
+    CK(cudaEventElapsedTime(&ms, r.a, r.b));
+    host_ms[r.cls] += ms;
+    host_counts[r.cls] += 1;
+  }
+  return WAM_OK;
+}
+
+wam_status wam_export_params(wam_ctx* c, float* host, size_t* nbytes) {
+  if (!c || !nbytes) return WAM_ERR_INVALID_ARG;
+  size_t total = 0;
+  for (auto& e : c->params) total += e.count();
+  if (!host) {
+    *nbytes = total * 4;
+    return WAM_OK;
+  }
+  if (*nbytes < total * 4) return fail(c, WAM_ERR_INVALID_ARG, "export buffer too small");
+  float* tmp = nullptr;
+  size_t mx = 0;
+  for (auto& e : c->params) mx = std::max(mx, e.count());
+  RET(dalloc(c, &tmp, mx * 4));
+  size_t at = 0;
+  wam_status st = WAM_OK;
+  for (size_t p = 0; p < c->params.size() && st == WAM_OK; ++p) {
+    const PEntry& e = c->params[p];
+    const void* src = e.matrix ? matp(c, (int)p) : (const void*)vecp(c, (int)p);
+    cudaError_t ce = launch_to_f32(src, e.matrix && c->d.bf16, tmp, e.count(), e.cols, e.matrix ? e.ld : e.cols, 0);
+    if (ce == cudaSuccess) ce = cudaMemcpy(host + at, tmp, e.count() * 4, cudaMemcpyDeviceToHost);
+    if (ce != cudaSuccess) st = fail(c, WAM_ERR_CUDA, "export: %s", cudaGetErrorString(ce));
+    at += e.count();
+  }
+  cudaFree(tmp);
+  *nbytes = total * 4;
+  return st;
+}
+
+wam_status wam_import_params(wam_ctx* c, const float* host, size_t nbytes) {
+  if (!c || !host) return WAM_ERR_INVALID_ARG;
+  size_t total = 0;
+  for (auto& e : c->params) total += e.count();
+  if (nbytes != total * 4) return fail(c, WAM_ERR_INVALID_ARG, "import size mismatch");
+  CK(cudaDeviceSynchronize());
+  std::vector<uint16_t> hb;
+  size_t at = 0;
+  for (size_t p = 0; p < c->params.size(); ++p) {
+    const PEntry& e = c->params[p];
+    const float* src = host + at;
+    at += e.count();
+    if (!e.matrix) {
+      std::vector<float> v(src, src + e.count());
+      if (c->d.bf16)
+        for (auto& f : v) {
+          uint32_t b;
+          memcpy(&b, &f, 4);
+          b = (b + 0x7FFFu + ((b >> 16) & 1u)) & 0xFFFF0000u;
+          memcpy(&f, &b, 4);
+        }
+      CK(cudaMemcpy(vecp(c, (int)p), v.data(), e.count() * 4, cudaMemcpyHostToDevice));
+      continue;
+    }
+    if (c->d.bf16) {
+      hb.assign((size_t)e.rows * e.ld, 0);
+      for (int r = 0; r < e.rows; ++r)
+        for (int k = 0; k < e.cols; ++k) {
+          uint32_t b;
+          memcpy(&b, &src[(size_t)r * e.cols + k], 4);
+          hb[(size_t)r * e.ld + k] = (uint16_t)((b + 0x7FFFu + ((b >> 16) & 1u)) >> 16);
+        }
+      CK(cudaMemcpy(matp(c, (int)p), hb.data(), hb.size() * 2, cudaMemcpyHostToDevice));
+    } else {
+      CK(cudaMemcpy(matp(c, (int)p), src, e.count() * 4, cudaMemcpyHostToDevice));
+    }
+  }
+  return WAM_OK;
+}
+
+wam_status wam_read_kv(wam_ctx* c, int block, int which, float* host, size_t* nbytes) {
+  if (!c || !nbytes || block < 0 || block >= c->d.N || (which != 0 && which != 1)) return WAM_ERR_INVALID_ARG;
+  const Dims& d = c->d;
+  const size_t n = (size_t)d.B * d.H * d.Ltot * d.Dh;
+  if (!host) {
+    *nbytes = n * 4;
+    return WAM_OK;
+  }
+  if (*nbytes < n * 4) return fail(c, WAM_ERR_INVALID_ARG, "read_kv buffer too small");
+  CK(cudaDeviceSynchronize());
+  float* tmp = nullptr;
+  RET(dalloc(c, &tmp, n * 4));
+  cudaError_t ce = launch_to_f32(which ? vcache(c, block) : kcache(c, block), d.bf16, tmp, n, 1, 1, 0);
+  if (ce == cudaSuccess) ce = cudaMemcpy(host, tmp, n * 4, cudaMemcpyDeviceToHost);
+  cudaFree(tmp);
+  CK(ce);
+  return WAM_OK;
+}
+
+wam_status wam_check_device_status(wam_ctx* c) {
+  if (!c) return WAM_ERR_INVALID_ARG;
+  CK(cudaDeviceSynchronize());
+  unsigned st = 0;
+  CK(cudaMemcpy(&st, c->status, 4, cudaMemcpyDeviceToHost));
+  if (st) {
+    CK(cudaMemset(c->status, 0, 4));
+    return fail(c, WAM_ERR_TIMEOUT, "device bounded wait gave up (status bits 0x%x)", st);
+  }
+  return WAM_OK;
+}
+
+int wam_chunk_kernel_count(wam_ctx* c, int S) {
+  if (!c) return -1;
+  for (auto& kv : c->launch_counts)
+    if ((kv.first >> 8) == S) return kv.second;
+  return -1;
+}
+
+// ------------------------------------------------- single-op entry points --
+wam_status wam_op_linear(int dtype, const void* x, const void* w, const float* bias, float* out, int M, int N, int K,
+                         int swap, int splits, void* stream) {
+  if (!x || !w || !bias || !out || M < 1 || N < 1 || K < 1) return WAM_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  EpiArgs e;
+  e.kind = kEpiStoreF32;
+  e.bias = bias;
+  e.out_f32 = out;
+  e.ld_out = N;
+  if (dtype == WAM_FP32) return launch_f32_gemm((const float*)x, (const float*)w, M, N, K, e, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
+  if (dtype != WAM_BF16 || K % 64) return WAM_ERR_INVALID_ARG;
+  const int bn = swap ? (M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256) : 128;
+  if (swap && M > 256) return WAM_ERR_INVALID_ARG;
+  static thread_local float* ws = nullptr;
+  static thread_local int* tk = nullptr;
+  static thread_local size_t ws_cap = 0, tk_cap = 0;
+  const int rows_w = N, tiles = swap ? ((N + 127) / 128) : 1;
+  const int kb = K / 64;
+  int sp = swap ? std::max(1, std::min(splits, kb)) : 1;
+  const size_t need = swap && sp > 1 ? (size_t)tiles * sp * 128 * bn : 0;
+  if (need > ws_cap) {
+    if (ws) cudaFree(ws);
+    if (cudaMalloc(&ws, need * 4) != cudaSuccess) return WAM_ERR_OOM;
+    ws_cap = need;
+  }
+  if ((size_t)tiles > tk_cap) {
+    if (tk) cudaFree(tk);
+    if (cudaMalloc(&tk, tiles * 4) != cudaSuccess) return WAM_ERR_OOM;
+    if (cudaMemset(tk, 0, tiles * 4) != cudaSuccess) return WAM_ERR_CUDA;
+    tk_cap = tiles;
+  }
+  static thread_local unsigned* status = nullptr;
+  if (!status) {
+    if (prepare_tc_gemm() != cudaSuccess) return WAM_ERR_CUDA;
+    if (cudaMalloc(&status, 4) != cudaSuccess) return WAM_ERR_OOM;
+    cudaMemset(status, 0, 4);
+  }
+  CUtensorMap mx, mw;
+  if (!make_tmap_3d(&mx, x, K, M, 1, 0, swap ? bn : 128) || !make_tmap_3d(&mw, w, K, rows_w, 1, 0, swap ? 128 : bn))
+    return WAM_ERR_INVALID_ARG;
+  TcGemm g;
+  g.map_a = swap ? &mw : &mx;
+  g.map_b = swap ? &mx : &mw;
+  g.rows_a = swap ? N : M;
+  g.rows_b = swap ? M : N;
+  g.K = K;
+  g.z_a = g.z_b = 0;
+  g.bn = bn;
+  g.splits = sp;
+  g.swap = swap != 0;
+  g.ws = ws;
+  g.tickets = tk;
+  g.status = status;
+  return launch_tc_gemm(g, e, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
+}
+
+wam_status wam_op_attention(int dtype, const void* q, const void* k, const void* v, void* out, int B, int H, int Dh,
+                            int Lq, int Lk, int Lcache, int splits, void* stream) {
+  if (!q || !k || !v || !out || B < 1 || H < 1 || Lq < 1 || Lk < 1 || Lk > Lcache) return WAM_ERR_INVALID_ARG;
+  AttnArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.B = B;
+  a.H = H;
+  a.Dh = Dh;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.Lcache = Lcache;
+  a.splits = splits < 1 ? 1 : splits;
+  a.ws = nullptr;
+  a.tickets = nullptr;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (dtype == WAM_FP32) return launch_attention_f32(a, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
+  if (dtype != WAM_BF16 || Dh != 64) return WAM_ERR_INVALID_ARG;
+  if (a.splits > 1) {
+    if (Lq > 64) return WAM_ERR_INVALID_ARG;
+    static thread_local float* ws = nullptr;
+    static thread_local int* tk = nullptr;
+    static thread_local size_t cap = 0, tcap = 0;
+    const size_t need = attention_ws_floats(B, H, Dh, Lq, a.splits);
+    if (need > cap) {
+      if (ws) cudaFree(ws);
+      if (cudaMalloc(&ws, need * 4) != cudaSuccess) return WAM_ERR_OOM;
+      cap = need;
+    }
+    if ((size_t)B * H > tcap) {
+      if (tk) cudaFree(tk);
+      if (cudaMalloc(&tk, (size_t)B * H * 4) != cudaSuccess) return WAM_ERR_OOM;
+      if (cudaMemset(tk, 0, (size_t)B * H * 4) != cudaSuccess) return WAM_ERR_CUDA;
+      tcap = (size_t)B * H;
+    }
+    a.ws = ws;
+    a.tickets = tk;
+  }
+  return launch_attention_bf16(a, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
+}
+
+}  // extern "C"

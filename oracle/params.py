@@ -28,6 +28,9 @@ CUDA library implements the same rule independently):
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 from .config import WamConfig
@@ -36,7 +39,7 @@ G = np.uint64(0x9E3779B97F4A7C15)
 _C1 = np.uint64(0xBF58476D1CE4E5B9)
 _C2 = np.uint64(0x94D049BB133111EB)
 STD = 0.02
-_CHUNK = 1 << 22
+_CHUNK = 1 << 20
 
 
 def _expert_specs(cfg: WamConfig, expert: str):
@@ -112,15 +115,31 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
     return r.view(np.float32)
 
 
+def _pool():
+    global _POOL
+    if _POOL is None:
+        _POOL = ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1))
+    return _POOL
+
+
+_POOL = None
+
+
 def generate_param(cfg: WamConfig, seed: int, pid: int, shape, std) -> np.ndarray:
     n = int(np.prod(shape))
     if std is None:
         out = np.ones(n, np.float32)
     else:
         out = np.empty(n, np.float32)
-        for s in range(0, n, _CHUNK):
+
+        def fill(s):
             c = min(_CHUNK, n - s)
             out[s:s + c] = (std * normal_block(seed, pid, s, c)).astype(np.float32)
+        starts = range(0, n, _CHUNK)
+        if n > _CHUNK:   # chunks are independent (counter-based); numpy releases the GIL
+            list(_pool().map(fill, starts))
+        else:
+            fill(0)
     if cfg.dtype == "bf16":
         out = round_bf16(out)
     return out.reshape(shape)

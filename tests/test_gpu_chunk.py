@@ -1,0 +1,169 @@
+"""End-to-end parity of the chunk on the GPU, through the C ABI, against the
+oracle: seeded parameters, the fp32 debug path (rel. L2 <= 1e-4), the bf16
+path (rel. L2 <= 1e-2) on a_0 and v_eff = a_1 - a_0, CEWP == sequential
+bitwise, graph == eager bitwise, the per-block K/V publish, the closed-form
+constant-velocity case and the eager video/action API."""
+import numpy as np
+import pytest
+
+import mot_dit_b200 as W
+from oracle import model as M
+from oracle import params as PR
+from wam_testlib import MID_BF16, check_parity, f32_sched, inputs, ocfg, oracle_chunk, rel_l2, run_chunk
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def _mid():
+    return W.WamConfig(**MID_BF16)
+
+
+@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+def test_seeded_params_match_oracle_generator(cfg):
+    c = W.preset(1) if cfg == "tiny" else _mid()
+    wam = W.Wam(c, seed=1234)
+    flat = wam.export_params()
+    P = PR.generate_params(ocfg(c), 1234)
+    ref = np.concatenate([P[n].ravel() for n, _, _ in PR.param_specs(ocfg(c))])
+    assert flat.shape == ref.shape
+    diff = flat != ref
+    # device and host libm may differ by one ulp in log/cos: allow a rare
+    # one-ulp (fp32) difference, nothing else
+    if diff.any():
+        assert diff.mean() < 1e-5
+        ulp = np.abs(flat[diff].view(np.int32).astype(np.int64) - ref[diff].view(np.int32).astype(np.int64))
+        assert ulp.max() <= (1 << 16 if c.dtype == 1 else 1)
+    wam.close()
+
+
+@pytest.mark.parametrize("S,mode,graph", [(1, W.CEWP, True), (1, W.SEQUENTIAL, False), (3, W.CEWP, False),
+                                          (3, W.SEQUENTIAL, True)])
+def test_tiny_fp32_parity(S, mode, graph):
+    c = W.preset(1)
+    wam = W.Wam(c, seed=5)
+    inp = inputs(c, 5)
+    a0 = run_chunk(wam, inp, S=S, mode=mode, use_graph=graph)
+    ref_a0, ref_veff = oracle_chunk(c, 5, inp, S=S)
+    check_parity(a0, inp, ref_a0, ref_veff, c.dtype)
+
+
+def test_mid_bf16_parity_and_kv_publish():
+    c = _mid()
+    wam = W.Wam(c, seed=11)
+    inp = inputs(c, 11)
+    a0 = run_chunk(wam, inp, S=1)
+    oc = ocfg(c)
+    P = PR.generate_params(oc, 11)
+    ref_a0, ref_veff = M.infer_chunk(oc, P, inp, t_sched=f32_sched(1))
+    check_parity(a0, inp, ref_a0, ref_veff, c.dtype)
+    # the K/V every video block publishes (rows [0, L_v) of the cache) and the
+    # action expert's own K/V of the last step (rows [L_v, L_v + L_a))
+    kv, _, _ = M.video_expert(oc, P, inp["video"], inp["cond"], 0.0)
+    for i in range(c.n_blocks):
+        k = wam.read_kv(i, 0)
+        v = wam.read_kv(i, 1)
+        assert rel_l2(k[:, :, :oc.l_v], kv[i][0]) < 1e-2, i
+        assert rel_l2(v[:, :, :oc.l_v], kv[i][1]) < 1e-2, i
+        assert np.abs(k[:, :, oc.l_v:]).sum() > 0
+
+
+@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+def test_cewp_equals_sequential_bitwise(cfg):
+    c = W.preset(1) if cfg == "tiny" else _mid()
+    wam = W.Wam(c, seed=3)
+    for seed in (0, 1, 2):
+        inp = inputs(c, seed)
+        outs = [run_chunk(wam, inp, S=S, mode=m, use_graph=g)
+                for S in (1, 3) for m, g in ((W.CEWP, True), (W.SEQUENTIAL, True), (W.CEWP, False),
+                                              (W.SEQUENTIAL, False))]
+        for S_idx in (0, 1):
+            group = outs[4 * S_idx: 4 * S_idx + 4]
+            for o in group[1:]:
+                assert np.array_equal(o, group[0])
+    # repeated graph launches stay bitwise stable
+    inp = inputs(c, 9)
+    first = run_chunk(wam, inp, S=1)
+    for _ in range(20):
+        assert np.array_equal(run_chunk(wam, inp, S=1), first)
+
+
+@pytest.mark.parametrize("cfg,S", [("tiny", 1), ("tiny", 8), ("mid", 1), ("mid", 8)])
+def test_constant_velocity_closed_form(cfg, S):
+    """All parameters zero except the action output bias b = 0.5: v = b for any
+    input, so a_0 = a_1 - 0.5 exactly (dyadic grid)."""
+    c = W.preset(1) if cfg == "tiny" else _mid()
+    wam = W.Wam(c, seed=0)
+    names = [n for n, _, _ in PR.param_specs(ocfg(c))]
+    sizes = [int(np.prod(s)) for _, s, _ in PR.param_specs(ocfg(c))]
+    flat = np.zeros(sum(sizes), np.float32)
+    at = 0
+    for n, sz in zip(names, sizes):
+        if n == "action.out.b":
+            flat[at:at + sz] = 0.5
+        at += sz
+    wam.import_params(flat)
+    inp = inputs(c, 4)
+    a0 = run_chunk(wam, inp, S=S)
+    # the state is fp32: each Euler step subtracts 0.5/S = 2^-k and rounds once,
+    # which is exact except where a negative value crosses a power of two
+    want = inp["noise"].copy()
+    for _ in range(S):
+        want = want - np.float32(0.5 / S)
+    np.testing.assert_array_equal(a0, want)
+    assert np.abs(a0.astype(np.float64) - (inp["noise"].astype(np.float64) - 0.5)).max() <= S * 2.0 ** -22 * 4
+
+
+def test_eager_video_and_action_steps_match_chunk():
+    c = _mid()
+    wam = W.Wam(c, seed=21)
+    inp = inputs(c, 21)
+    ref = run_chunk(wam, inp, S=2, mode=W.CEWP, use_graph=True)
+    dev = torch.device("cuda", 0)
+    video = torch.from_numpy(inp["video"]).to(dev)
+    cond = torch.from_numpy(inp["cond"]).to(dev)
+    a = torch.from_numpy(inp["noise"]).to(dev)
+    sv, sa = torch.cuda.Stream(), torch.cuda.Stream()
+    wam.video_forward(video, cond, 0.0, stream=sv)
+    wam.action_step(a, 1.0, 0.5, stream=sa)
+    wam.action_step(a, 0.5, 0.0, stream=sa)
+    sa.synchronize()
+    sv.synchronize()
+    wam.check_device_status()
+    assert np.array_equal(a.cpu().numpy(), ref)
+
+
+def test_host_buffer_entry_point_matches_device_one():
+    c = _mid()
+    wam = W.Wam(c, seed=8)
+    inp = inputs(c, 8)
+    ref = run_chunk(wam, inp, S=1)
+    out = np.zeros_like(inp["noise"])
+    sv, sa = torch.cuda.Stream(), torch.cuda.Stream()
+    wam.infer_chunk_host(inp["video"], inp["cond"], inp["noise"], out, S=1, stream_video=sv, stream_action=sa)
+    assert np.array_equal(out, ref)
+
+
+def test_argument_errors_enqueue_nothing():
+    c = _mid()
+    wam = W.Wam(c, seed=0)
+    inp = inputs(c, 0)
+    dev = torch.device("cuda", 0)
+    video = torch.from_numpy(inp["video"]).to(dev)
+    noise = torch.from_numpy(inp["noise"]).to(dev)
+    out = torch.empty_like(noise)
+    with pytest.raises(W.WamError) as e:
+        wam.infer_chunk(video, None, noise, out, S=1)           # missing conditioning tokens
+    assert e.value.status == 1
+    cond = torch.from_numpy(inp["cond"]).to(dev)
+    for S, t in ((0, None), (65, None), (2, [1.0, 0.7, 0.8]), (1, [1.5, 0.0])):
+        with pytest.raises(W.WamError):
+            wam.infer_chunk(video, cond, noise, out, S=S, t_sched=t)
+    sv = torch.cuda.Stream()
+    with pytest.raises(W.WamError):   # CEWP with one stream
+        wam.infer_chunk(video, cond, noise, out, S=1, mode=W.CEWP, stream_video=sv, stream_action=sv)
+    fresh = W.Wam(c, seed=0)
+    with pytest.raises(W.WamError) as e:
+        fresh.action_step(out, 1.0, 0.0)
+    assert e.value.status == 6
+    wam.check_device_status()

@@ -1,0 +1,94 @@
+"""Single-kernel parity on the GPU, through the C ABI: the tcgen05 GEMM (both
+orientations, split-K), the fp32 SIMT GEMM, and the attention kernels (video
+single pass, action split-KV, fp32) against the oracle's definitions."""
+import numpy as np
+import pytest
+
+import mot_dit_b200 as W
+from oracle import model as M
+from oracle.params import round_bf16
+from wam_testlib import rel_l2
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _bf16(a):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(DEV).to(torch.bfloat16)
+
+
+def _f32(a):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(DEV)
+
+
+@pytest.mark.parametrize("M_,N,K,swap,splits", [
+    (200, 384, 256, False, 1),     # ragged M tail, 2 x 3 tiles
+    (1088, 256, 128, False, 1),    # 8.5 row tiles
+    (32, 300, 512, True, 1),       # few tokens, ragged feature tail
+    (32, 300, 512, True, 4),       # split-K, fixed-order reduction
+    (16, 30, 768, True, 3),        # action out-projection shape
+    (256, 128, 192, True, 1),      # 256-token column tile
+])
+def test_linear_bf16(M_, N, K, swap, splits):
+    rng = np.random.default_rng(M_ + N + K)
+    x = round_bf16(rng.standard_normal((M_, K)).astype(np.float32))
+    w = round_bf16((0.05 * rng.standard_normal((N, K))).astype(np.float32))
+    b = rng.standard_normal(N).astype(np.float32)
+    out = torch.full((M_, N), float("nan"), device=DEV)
+    W.op_linear(W.BF16, _bf16(x), _bf16(w), _f32(b), out, M_, N, K, swap=swap, splits=splits)
+    torch.cuda.synchronize()
+    ref = x.astype(np.float64) @ w.astype(np.float64).T + b
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    assert rel_l2(got, ref) < 2e-6
+
+
+def test_linear_f32():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((70, 48)).astype(np.float32)
+    w = rng.standard_normal((50, 48)).astype(np.float32)
+    b = rng.standard_normal(50).astype(np.float32)
+    out = torch.zeros(70, 50, device=DEV)
+    W.op_linear(W.FP32, _f32(x), _f32(w), _f32(b), out, 70, 50, 48)
+    torch.cuda.synchronize()
+    ref = x.astype(np.float64) @ w.astype(np.float64).T + b
+    assert rel_l2(out.cpu().numpy(), ref) < 1e-6
+
+
+def _attn_case(B, H, Dh, Lq, Lk, Lc, seed):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, H, Lq, Dh)).astype(np.float32)
+    k = rng.standard_normal((B, H, Lc, Dh)).astype(np.float32)
+    v = rng.standard_normal((B, H, Lc, Dh)).astype(np.float32)
+    return q, k, v
+
+
+@pytest.mark.parametrize("B,H,Lq,Lk,Lc,splits", [
+    (2, 3, 100, 100, 130, 1),      # video: ragged queries and keys
+    (1, 2, 1088, 1088, 1120, 1),   # full video length
+    (1, 4, 32, 1120, 1120, 9),     # action: joint keys, split-KV
+    (2, 2, 16, 300, 310, 3),       # action, 16 queries, ragged split
+])
+def test_attention_bf16(B, H, Lq, Lk, Lc, splits):
+    q, k, v = _attn_case(B, H, 64, Lq, Lk, Lc, Lq + Lk)
+    q, k, v = (round_bf16(a) for a in (q, k, v))
+    out = torch.full((B * Lq, H * 64), float("nan"), device=DEV, dtype=torch.bfloat16)
+    W.op_attention(W.BF16, _bf16(q), _bf16(k), _bf16(v), out, B, H, 64, Lq, Lk, Lc, splits=splits)
+    torch.cuda.synchronize()
+    ref = M.merge_heads(M.attention(q.astype(np.float64), k[:, :, :Lk].astype(np.float64),
+                                    v[:, :, :Lk].astype(np.float64))).reshape(B * Lq, H * 64)
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert rel_l2(got, ref) < 1e-2
+
+
+def test_attention_f32():
+    B, H, Dh, Lq, Lk, Lc = 1, 4, 16, 80, 80, 96
+    q, k, v = _attn_case(B, H, Dh, Lq, Lk, Lc, 7)
+    out = torch.zeros(B * Lq, H * Dh, device=DEV)
+    W.op_attention(W.FP32, _f32(q), _f32(k), _f32(v), out, B, H, Dh, Lq, Lk, Lc)
+    torch.cuda.synchronize()
+    ref = M.merge_heads(M.attention(q.astype(np.float64), k[:, :, :Lk].astype(np.float64),
+                                    v[:, :, :Lk].astype(np.float64))).reshape(B * Lq, H * Dh)
+    assert rel_l2(out.cpu().numpy(), ref) < 1e-5
