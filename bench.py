@@ -356,7 +356,7 @@ def run_ours(args, rank, world, local_rank):
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": None,
                      "peak_kind": f"{peaks['_kind']} bf16 sustained",
-                     "launches_timed": g_launch, "method": "CUDA events around each launch, eager sequential chunk"},
+                     "launches_timed": g_launch, "method": "CUDA event-record nodes around each launch in a captured sequential chunk"},
         "chunk_roofline": {"ms": round(chunk_roof, 4), "t_tensor_ms": round(t_tc, 4), "t_hbm_ms": round(t_hbm, 4),
                            "flops": flops, "bytes": bytes_, "frac": round(chunk_roof / ms_per_step, 4)},
         "breakdown": breakdown,

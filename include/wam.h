@@ -184,8 +184,9 @@ typedef enum {
   WAM_PROF_CLASSES
 } wam_prof_class;
 
-/* Measurement: run one chunk (S uniform steps) eagerly with the sequential
- * schedule on `stream`, with a CUDA event pair around every launch, and
+/* Measurement: run one chunk (S uniform steps) with the sequential schedule
+ * on `stream` -- captured once into a CUDA graph with an event-record node
+ * before and after every launch, then replayed -- and
  * return per class the summed launch durations host_ms[WAM_PROF_CLASSES] and
  * the launch counts host_counts[WAM_PROF_CLASSES].  Synchronises `stream`.
  * Arguments as in wam_infer_chunk.  (QKV and the action in / out projections

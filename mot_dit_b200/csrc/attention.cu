@@ -27,6 +27,7 @@ constexpr int kD = 64;      // head dim of the bf16 path
 constexpr int kTQ = 64;     // queries per CTA (4 warps x 16)
 constexpr int kTK = 64;     // keys per tile
 constexpr int kAttnThreads = 128;
+constexpr int kMaxSplits = 32;  // key splits of the action attention
 
 // Row-major [64][64] bf16 tile, 16-byte chunks XOR-swizzled by row.
 __device__ __forceinline__ uint32_t tile_off(int row, int chunk) {
@@ -220,20 +221,35 @@ __global__ void __launch_bounds__(kAttnThreads)
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // Combine in split order: per row r, M = max_s m_s, den = sum_s 2^((m_s - M) c) l_s,
+  // then O[r, :] = sum_s (2^((m_s - M) c) / den) O_s[r, :].
+  // the Q/K/V tiles are no longer needed: reuse them for the per-row factors
+  float (*s_f)[kTQ] = reinterpret_cast<float (*)[kTQ]>(smem);
   const float* cO = ws + bh * splits * (kTQ * kD);
   const float* cM = ws + (size_t)gridDim.z / splits * H * splits * kTQ * kD + bh * splits * kTQ * 2;
+  // every (m, l) of every split in flight at once, into shared memory
+  float* s_ml = reinterpret_cast<float*>(smem) + kMaxSplits * kTQ;  // [splits][kTQ][2]
+  for (int i = tid; i < splits * kTQ * 2; i += kAttnThreads) s_ml[i] = __ldcg(cM + i);
+  __syncthreads();
+  if (tid < kTQ) {
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < splits; ++s2) M = fmaxf(M, s_ml[(s2 * kTQ + tid) * 2]);
+    float den = 0.f;
+    for (int s2 = 0; s2 < splits; ++s2) {
+      const float f = exp2f((s_ml[(s2 * kTQ + tid) * 2] - M) * sl2e);
+      s_f[s2][tid] = f;
+      den += f * s_ml[(s2 * kTQ + tid) * 2 + 1];
+    }
+    const float inv = 1.0f / den;
+    for (int s2 = 0; s2 < splits; ++s2) s_f[s2][tid] *= inv;
+  }
+  __syncthreads();
   for (int idx = tid; idx < Lq * kD; idx += kAttnThreads) {
     const int row = idx / kD, d = idx - row * kD;
-    float M = -INFINITY;
-    for (int s2 = 0; s2 < splits; ++s2) M = fmaxf(M, __ldcg(cM + (s2 * kTQ + row) * 2));
-    float num = 0.f, den = 0.f;
-    for (int s2 = 0; s2 < splits; ++s2) {
-      const float ms = __ldcg(cM + (s2 * kTQ + row) * 2);
-      const float f = exp2f((ms - M) * sl2e);
-      num += f * __ldcg(cO + (size_t)s2 * kTQ * kD + row * kD + d);
-      den += f * __ldcg(cM + (s2 * kTQ + row) * 2 + 1);
-    }
-    out[(size_t)(b * Lq + row) * A + h * kD + d] = __float2bfloat16_rn(num / den);
+    float acc = 0.f;
+#pragma unroll 4
+    for (int s2 = 0; s2 < splits; ++s2) acc += s_f[s2][row] * __ldcg(cO + (size_t)s2 * kTQ * kD + row * kD + d);
+    out[(size_t)(b * Lq + row) * A + h * kD + d] = __float2bfloat16_rn(acc);
   }
   if (tid == 0) tickets[bh] = 0;
 }
@@ -305,6 +321,7 @@ cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s) {
   int kps = (a.Lk + splits - 1) / splits;
   kps = (kps + kTK - 1) / kTK * kTK;
   const int used = (a.Lk + kps - 1) / kps;  // non-empty splits only
+  if (used > kMaxSplits) return cudaErrorInvalidValue;
   dim3 grid((a.Lq + kTQ - 1) / kTQ, a.H, a.B * used);
   const auto* q = reinterpret_cast<const __nv_bfloat16*>(a.q);
   const auto* k = reinterpret_cast<const __nv_bfloat16*>(a.k);

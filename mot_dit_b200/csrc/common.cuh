@@ -208,15 +208,22 @@ __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g, bool v
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(g), "r"(n)
                : "memory");
 }
+// 16-byte async copy into shared memory, always valid source.
+__device__ __forceinline__ void cp_async16_ca(uint32_t saddr, const void* g) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// GELU, tanh form: 0.5 x (1 + tanh(z)), z = sqrt(2/pi) (x + 0.044715 x^3),
+// evaluated through the identity 0.5 (1 + tanh(z)) = 1 / (1 + exp(-2 z)).
 __device__ __forceinline__ float gelu_tanh(float x) {
-  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
-  return 0.5f * x * (1.0f + tanhf(k0 * (x + 0.044715f * x * x * x)));
+  const float k2 = 1.5957691216057308f;  // 2 sqrt(2/pi)
+  const float z2 = k2 * (x + 0.044715f * x * x * x);
+  return __fdividef(x, 1.0f + __expf(-z2));
 }
 
 }  // namespace wam

@@ -80,6 +80,7 @@ struct TcGemm {
   int bn;                    // N tile (32, 64, 128, 256)
   int splits;                // split-K factor (swap only)
   bool swap;
+  int max_ctas;              // persistent grid size (0: one CTA per SM)
   float* ws;                 // split-K partials, splits * tiles * 128 * bn floats
   int* tickets;              // one per output tile, zero on entry, left zero
   unsigned* status;

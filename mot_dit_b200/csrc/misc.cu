@@ -17,7 +17,11 @@ constexpr int kNormWarps = 8;
 
 // ------------------------------------------------- norm + modulation -------
 // h = rms(x) * (gain ? gain[n] : 1 + scale[n]) + (shift ? shift[n] : 0);
-// rms(x) = x / sqrt(mean(x^2) + 1e-6).  One warp per row.
+// rms(x) = x / sqrt(mean(x^2) + 1e-6).  One warp per row; a lane holds up to
+// kNormV float4 of the row in registers so every load of the row is in flight
+// at once (d <= 32 * 4 * kNormV).
+constexpr int kNormV = 12;
+
 template <bool BF16>
 __global__ void __launch_bounds__(32 * kNormWarps)
     norm_mod_kernel(const float* __restrict__ x, void* __restrict__ h, int M, int d, const float* __restrict__ scale,
@@ -27,24 +31,38 @@ __global__ void __launch_bounds__(32 * kNormWarps)
   if (row >= M) return;
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * d);
   const int n4 = d >> 2;
+  float4 v[kNormV];
   float ss = 0.f;
-  for (int i = lane; i < n4; i += 32) {
-    const float4 v = xr[i];
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+#pragma unroll
+  for (int k = 0; k < kNormV; ++k) {
+    const int i = lane + 32 * k;
+    v[k] = i < n4 ? xr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+#pragma unroll
+  for (int k = 0; k < kNormV; ++k) ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float r = 1.0f / sqrtf(ss / (float)d + 1e-6f);
-  for (int i = lane; i < n4; i += 32) {
-    const float4 v = xr[i];
-    float y[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = 4 * i + j;
-      const float mul = gain ? gain[n] : 1.0f + scale[n];
-      const float add = shift ? shift[n] : 0.f;
-      y[j] = y[j] * r * mul + add;
+  for (int k = 0; k < kNormV; ++k) {
+    const int i = lane + 32 * k;
+    if (i >= n4) break;
+    float y[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+    float4 mul4, add4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (gain) {
+      mul4 = __ldg(reinterpret_cast<const float4*>(gain) + i);
+    } else {
+      mul4 = __ldg(reinterpret_cast<const float4*>(scale) + i);
+      mul4.x += 1.f;
+      mul4.y += 1.f;
+      mul4.z += 1.f;
+      mul4.w += 1.f;
     }
+    if (shift) add4 = __ldg(reinterpret_cast<const float4*>(shift) + i);
+    y[0] = y[0] * r * mul4.x + add4.x;
+    y[1] = y[1] * r * mul4.y + add4.y;
+    y[2] = y[2] * r * mul4.z + add4.z;
+    y[3] = y[3] * r * mul4.w + add4.w;
     if (BF16) {
       uint2 p;
       p.x = pack_bf16(y[0], y[1]);
@@ -248,7 +266,7 @@ int grid_for(size_t n, int threads) {
 
 cudaError_t launch_norm_mod(const float* x, void* h, bool h_bf16, int M, int d, const float* scale,
                             const float* shift, const float* gain, cudaStream_t s) {
-  if (d % 4 != 0) return cudaErrorInvalidValue;
+  if (d % 4 != 0 || d > 32 * 4 * kNormV) return cudaErrorInvalidValue;
   dim3 grid((M + kNormWarps - 1) / kNormWarps);
   if (h_bf16)
     norm_mod_kernel<true><<<grid, 32 * kNormWarps, 0, s>>>(x, h, M, d, scale, shift, gain);

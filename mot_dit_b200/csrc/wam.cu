@@ -53,7 +53,7 @@ struct Dims {
 };
 
 struct GemmPlan {
-  int bn = 128, splits = 1;
+  int bn = 128, splits = 1, max_ctas = 0;
 };
 
 }  // namespace
@@ -157,11 +157,11 @@ struct ProfScope {
     }
     cudaEvent_t a = c->prof_pool[c->prof_next++];
     b = c->prof_pool[c->prof_next++];
-    cudaEventRecord(a, s);
+    cudaEventRecordWithFlags(a, s, cudaEventRecordExternal);
     c->prof.push_back({c->cur_cls, a, b});
   }
   ~ProfScope() {
-    if (b) cudaEventRecord(b, s);
+    if (b) cudaEventRecordWithFlags(b, s, cudaEventRecordExternal);
   }
 };
 
@@ -305,6 +305,7 @@ wam_status run_tc(wam_ctx* c, const CUtensorMap& A, const CUtensorMap& Bm, int r
   g.bn = p.bn;
   g.splits = p.splits;
   g.swap = swap;
+  g.max_ctas = p.max_ctas;
   g.ws = c->ws_gemm;
   g.tickets = c->tk_gemm;
   g.status = c->status;
@@ -838,12 +839,12 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   size_t ws = 0;
   int tiles = 1;
   if (d.bf16) {
-    c->p_v_qkv = {128, 1};
-    c->p_v_o = {128, 1};
-    c->p_v_f1 = {256, 1};
-    c->p_v_f2 = {128, 1};
-    c->p_v_in = {128, 1};
-    c->p_v_out = {64, 1};
+    c->p_v_qkv = {128, 1, 0};
+    c->p_v_o = {128, 1, 0};
+    c->p_v_f1 = {128, 1, 0};
+    c->p_v_f2 = {128, 1, 0};
+    c->p_v_in = {128, 1, 0};
+    c->p_v_out = {64, 1, 0};
     const int bn_a = d.Ma <= 32 ? 32 : (d.Ma <= 64 ? 64 : (d.Ma <= 128 ? 128 : 256));
     c->p_a_in = plan_swap(d.da, d.Ma, d.Kin, bn_a);
     c->p_a_qkv = plan_swap(3 * d.A, d.Ma, d.da, bn_a);
@@ -1046,14 +1047,32 @@ wam_status wam_profile_chunk(wam_ctx* c, const float* video, const float* cond, 
   v.video = video;
   v.cond = cond;
   RET(set_chunk_io(c, v, a, s));
+  // Capture the sequential chunk with an event-record node around every
+  // launch, then replay it: the kernels run back to back as in the timed
+  // graph, without host launch latency between them.
+  CK(cudaStreamSynchronize(s));
   c->prof.clear();
   c->prof_next = 0;
   c->prof_on = true;
   c->launches = 0;
-  wam_status st = enqueue_chunk(c, S, WAM_SCHED_SEQUENTIAL, false, s, s, c->ev_kv.data());
+  cudaGraph_t graph = nullptr;
+  CK(cudaStreamBeginCapture(c->cap_v, cudaStreamCaptureModeThreadLocal));
+  wam_status st = enqueue_chunk(c, S, WAM_SCHED_SEQUENTIAL, false, c->cap_v, c->cap_v, c->ev_kv_cap.data());
   c->prof_on = false;
-  RET(st);
-  CK(cudaStreamSynchronize(s));
+  cudaError_t ce = cudaStreamEndCapture(c->cap_v, &graph);
+  if (st != WAM_OK) {
+    if (graph) cudaGraphDestroy(graph);
+    return st;
+  }
+  CK(ce);
+  cudaGraphExec_t exec = nullptr;
+  ce = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  CK(ce);
+  ce = cudaGraphLaunch(exec, s);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
+  cudaGraphExecDestroy(exec);
+  CK(ce);
   for (int k = 0; k < WAM_PROF_CLASSES; ++k) {
     host_ms[k] = 0.f;
     host_counts[k] = 0;
@@ -1224,6 +1243,7 @@ wam_status wam_op_linear(int dtype, const void* x, const void* w, const float* b
   g.bn = bn;
   g.splits = sp;
   g.swap = swap != 0;
+  g.max_ctas = 0;
   g.ws = ws;
   g.tickets = tk;
   g.status = status;
