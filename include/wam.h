@@ -213,6 +213,31 @@ wam_status wam_op_linear(int dtype, const void* dev_x, const void* dev_w, const 
 wam_status wam_op_attention(int dtype, const void* dev_q, const void* dev_k, const void* dev_v, void* dev_out,
                             int B, int H, int Dh, int Lq, int Lk, int Lcache, int splits, void* stream);
 
+/* Allocation-free split-KV attention.  (An addition for deployment; the
+ * paper has no counterpart.)  Same computation, kernel and arguments as
+ * wam_op_attention with dtype WAM_BF16, Dh = 64 and splits >= 2, for callers
+ * that cannot let a library allocate device memory while they run -- a
+ * control loop that must not call cudaMalloc after start-up (the call can
+ * synchronise the device and has unbounded latency), or a process whose
+ * device memory budget belongs to another allocator.  Its scratch (per-split
+ * partial outputs, row maxima and sums, and the tickets that pick the
+ * combining CTA) is a fixed 8 MiB + 4 KiB array compiled into the library,
+ * held by every GPU that loads the library until the process exits; the call
+ * makes no allocation.
+ *   - Limits: B * H * s * (64*64 + 128) floats <= 2^21 and B * H <= 1024,
+ *     where s is the number of non-empty key splits (at most 32);
+ *     1 <= Lq <= 64.  A call beyond them returns WAM_ERR_UNSUPPORTED and
+ *     enqueues nothing.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before
+ *     any stream capture.
+ *   - Every call shares the array: calls that overlap on the GPU (other
+ *     streams, other threads) race.  Each call clears the tickets it uses
+ *     before its kernel runs.
+ *   - Enqueued on `stream`; returns WAM_ERR_INVALID_ARG for bad arguments. */
+wam_status wam_op_attention_noalloc(const void* dev_q, const void* dev_k, const void* dev_v, void* dev_out, int B,
+                                    int H, int Lq, int Lk, int Lcache, int splits, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,6 +19,7 @@ from ._binding import (  # noqa: F401
     lib,
     library_path,
     op_attention,
+    op_attention_noalloc,
     op_linear,
     preset,
 )

@@ -77,6 +77,7 @@ def lib():
         "wam_last_error": (C.c_char_p, [_P]),
         "wam_op_linear": (C.c_int, [C.c_int, _P, _P, _P, _P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _P]),
         "wam_op_attention": (C.c_int, [C.c_int, _P, _P, _P, _P] + [C.c_int] * 7 + [_P]),
+        "wam_op_attention_noalloc": (C.c_int, [_P, _P, _P, _P] + [C.c_int] * 6 + [_P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -223,3 +224,11 @@ def op_attention(dtype, q, k, v, out, B, H, Dh, Lq, Lk, Lcache, splits=1, stream
                                 _stream(stream))
     if st:
         raise WamError(st, "wam_op_attention")
+
+
+def op_attention_noalloc(q, k, v, out, B, H, Lq, Lk, Lcache, splits, stream=None):
+    """Split-KV bf16 attention with library-owned static scratch (no allocation)."""
+    st = lib().wam_op_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Lq, Lk, Lcache, splits,
+                                        _stream(stream))
+    if st:
+        raise WamError(st, "wam_op_attention_noalloc")
