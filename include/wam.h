@@ -213,6 +213,15 @@ wam_status wam_op_linear(int dtype, const void* dev_x, const void* dev_w, const 
 wam_status wam_op_attention(int dtype, const void* dev_q, const void* dev_k, const void* dev_v, void* dev_out,
                             int B, int H, int Dh, int Lq, int Lk, int Lcache, int splits, void* stream);
 
+/* h[M, d] = rms(x) * (dev_gain ? gain : 1 + scale) + (dev_shift ? shift : 0)
+ * per row, rms(x) = x / sqrt(mean(x^2) + 1e-6): the RMSNorm / AdaLN
+ * modulation prologue of every block (and, with a gain, the final norm).
+ * x fp32 [M, d]; h bf16 (dtype WAM_BF16) or fp32 (WAM_FP32); d a multiple
+ * of 4 and <= 1536; scale / shift / gain fp32 [d] (dev_scale required when
+ * dev_gain is NULL).  Enqueued on `stream`. */
+wam_status wam_op_norm_mod(int dtype, const float* dev_x, void* dev_h, int M, int d, const float* dev_scale,
+                           const float* dev_shift, const float* dev_gain, void* stream);
+
 /* Allocation-free split-KV attention.  (An addition for deployment; the
  * paper has no counterpart.)  Same computation, kernel and arguments as
  * wam_op_attention with dtype WAM_BF16, Dh = 64 and splits >= 2, for callers

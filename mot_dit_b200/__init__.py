@@ -21,5 +21,6 @@ from ._binding import (  # noqa: F401
     op_attention,
     op_attention_noalloc,
     op_linear,
+    op_norm_mod,
     preset,
 )

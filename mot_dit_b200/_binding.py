@@ -78,6 +78,7 @@ def lib():
         "wam_op_linear": (C.c_int, [C.c_int, _P, _P, _P, _P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _P]),
         "wam_op_attention": (C.c_int, [C.c_int, _P, _P, _P, _P] + [C.c_int] * 7 + [_P]),
         "wam_op_attention_noalloc": (C.c_int, [_P, _P, _P, _P] + [C.c_int] * 6 + [_P]),
+        "wam_op_norm_mod": (C.c_int, [C.c_int, _P, _P, C.c_int, C.c_int, _P, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -217,6 +218,12 @@ def op_linear(dtype, x, w, bias, out, M, N, K, swap=False, splits=1, stream=None
                              _stream(stream))
     if st:
         raise WamError(st, "wam_op_linear")
+
+
+def op_norm_mod(dtype, x, h, M, d, scale=None, shift=None, gain=None, stream=None):
+    st = lib().wam_op_norm_mod(dtype, _ptr(x), _ptr(h), M, d, _ptr(scale), _ptr(shift), _ptr(gain), _stream(stream))
+    if st:
+        raise WamError(st, "wam_op_norm_mod")
 
 
 def op_attention(dtype, q, k, v, out, B, H, Dh, Lq, Lk, Lcache, splits=1, stream=None):

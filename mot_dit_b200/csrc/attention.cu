@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(kAttnThreads)
   const int k_end = min(Lk, k_begin + keys_per_split);
   const int ntiles = (k_end - k_begin + kTK - 1) / kTK;
 
+  pdl_trigger();
+  pdl_wait();
   const __nv_bfloat16* qb = q + (size_t)(b * H + h) * Lq * kD;
   const __nv_bfloat16* kb = kc + (size_t)(b * H + h) * Lcache * kD;
   const __nv_bfloat16* vb = vc + (size_t)(b * H + h) * Lcache * kD;
@@ -328,12 +330,10 @@ cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s) {
   const auto* v = reinterpret_cast<const __nv_bfloat16*>(a.v);
   auto* o = reinterpret_cast<__nv_bfloat16*>(a.out);
   if (used > 1)
-    attn_bf16_kernel<true><<<grid, kAttnThreads, 0, s>>>(q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache, used, kps, a.ws,
-                                                         a.tickets);
-  else
-    attn_bf16_kernel<false><<<grid, kAttnThreads, 0, s>>>(q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache, 1, kps, nullptr,
-                                                          nullptr);
-  return cudaGetLastError();
+    return launch_k(attn_bf16_kernel<true>, grid, dim3(kAttnThreads), 0, s, q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache,
+                    used, kps, a.ws, a.tickets);
+  return launch_k(attn_bf16_kernel<false>, grid, dim3(kAttnThreads), 0, s, q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache, 1,
+                  kps, (float*)nullptr, (int*)nullptr);
 }
 
 cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t s) {

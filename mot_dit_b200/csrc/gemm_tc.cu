@@ -48,7 +48,7 @@ struct TileCfg {
   static constexpr int kABytes = BM * BK * 2;
   static constexpr int kBBytes = BN * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
+  static constexpr int kTmemCols = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
   // Normal orientation, BN <= 128: each epilogue warp prefetches its 32 x BN
   // residual rows (gate-residual) or 32 RoPE rows (QKV) while the MMA runs.
   static constexpr bool kPrefetch = !SWAP && BN <= 128;
@@ -62,7 +62,6 @@ struct TileCfg {
   static constexpr int kSmem = kStages * kStageBytes + kEpiBytes + kResBytes + kBarBytes + 1024;
   static_assert(kStages >= 3, "shared memory ring too shallow");
 };
-constexpr int kRopeStride = 36;  // floats per prefetched RoPE row (32 + pad, 16-byte aligned)
 
 struct GemmK {
   int rows_a, rows_b, K;
@@ -130,9 +129,11 @@ __device__ __forceinline__ EpiRegs hoist(const EpiArgs& e) {
 
 // Per-head QK-RMSNorm (gain), RoPE, and scatter of one 64-channel head vector
 // of token m.  section: 0 = q, 1 = k, 2 = v.  cs_row / sn_row: the token's
-// cos / sin row (prefetched in shared memory, or null to read the table).
+// cos / sin row, prefetched in shared memory with its 16-byte chunks permuted
+// by XOR with swz (or null to read the table).
 __device__ __forceinline__ void qkv_emit(const EpiRegs& R, int section, int head, int m, float (&x)[64],
-                                         const float* cs_row = nullptr, const float* sn_row = nullptr) {
+                                         const float* cs_row = nullptr, const float* sn_row = nullptr,
+                                         int swz = 0) {
   const int b = m / R.seq_len, l = m - b * R.seq_len;
   if (section < 2) {
     const float4* g4 = reinterpret_cast<const float4*>((section == 0 ? R.gq : R.gk) + head * 64);
@@ -153,7 +154,7 @@ __device__ __forceinline__ void qkv_emit(const EpiRegs& R, int section, int head
     const float4* sn = reinterpret_cast<const float4*>(sn_row ? sn_row : R.rope_sin + pos * 32);
 #pragma unroll
     for (int j4 = 0; j4 < 8; ++j4) {
-      const float4 c4 = cs[j4], s4 = sn[j4];
+      const float4 c4 = cs[cs_row ? (j4 ^ swz) : j4], s4 = sn[sn_row ? (j4 ^ swz) : j4];
       const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss4[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -262,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();  // the next kernel may start its own set-up now
 
   // unit u -> (tile_a, tile_b, split); split fastest, then tile_a, then tile_b
   auto decode = [&](int u, int& ta, int& tb, int& sp) {
@@ -275,11 +277,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int it = 0, issued = 0;
       bool ok = true;
+      // The weights never change during a chunk: the first unit's weight tiles
+      // are requested before waiting for the previous kernel (dependent launch).
+      int pre = 0;
+      if (blockIdx.x < g.units) {
+        int ta, tb, sp;
+        decode(blockIdx.x, ta, tb, sp);
+        const int kb0 = sp * g.kb_per_split, kb1 = min(kb_total, kb0 + g.kb_per_split);
+        pre = min(C::kStages, kb1 - kb0);
+        for (int i = 0; i < pre; ++i) {
+          mbar_arrive_expect_tx(&full[i], C::kStageBytes);
+          if (SWAP)
+            tma_load_3d(sA + i * C::kABytes, &map_a, &full[i], (kb0 + i) * BK, ta * BM, g.z_a);
+          else
+            tma_load_3d(sB + i * C::kBBytes, &map_b, &full[i], (kb0 + i) * BK, tb * BN, g.z_b);
+        }
+        pdl_wait();
+        for (int i = 0; i < pre; ++i) {
+          if (SWAP)
+            tma_load_3d(sB + i * C::kBBytes, &map_b, &full[i], (kb0 + i) * BK, tb * BN, g.z_b);
+          else
+            tma_load_3d(sA + i * C::kABytes, &map_a, &full[i], (kb0 + i) * BK, ta * BM, g.z_a);
+        }
+        issued = pre;
+      } else {
+        pdl_wait();
+      }
       for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x) {
         int ta, tb, sp;
         decode(u, ta, tb, sp);
         const int kb0 = sp * g.kb_per_split, kb1 = min(kb_total, kb0 + g.kb_per_split);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          if (it < pre) continue;  // issued above
           const int s = it % C::kStages;
           if (it >= C::kStages &&
               !mbar_wait(&empty[s], ((it / C::kStages) - 1) & 1, g.status, kStatusTimeoutTmaEmpty, abort_flag)) {
@@ -333,11 +362,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    pdl_wait();  // outputs / residual rows belong to the previous kernel until it is done
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const EpiRegs R = hoist(e);
     float* res = sRes + quad * (32 * BN);  // this warp's prefetched residual rows / RoPE rows
-    constexpr bool kRopeFits = C::kPrefetch && 32 * BN >= 2 * 32 * kRopeStride;
+    constexpr bool kRopeFits = C::kPrefetch && BN >= 64;  // 32 cos + 32 sin rows of 32 floats
     int lt = 0;
     for (int u = blockIdx.x; u < g.units; u += gridDim.x, ++lt) {
       int ta, tb, sp;
@@ -365,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int m = min(m0 + r, g.rows_a - 1);
             const int pos = R.cache_off + (m % R.seq_len);
             const float* src = (which ? R.rope_sin : R.rope_cos) + pos * 32 + 4 * c4;
-            cp_async16(smem_u32(res + which * (32 * kRopeStride) + r * kRopeStride + 4 * c4), src, true);
+            cp_async16(smem_u32(res + which * (32 * 32) + r * 32 + 4 * (c4 ^ (r & 7))), src, true);
           }
           cp_async_commit();
           prefetched = true;
@@ -414,8 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 x[4 * j + 3] += bb.w;
               }
               if constexpr (kRopeFits)
-                qkv_emit(R, n / R.attn_dim, (n % R.attn_dim) / 64, m, x, res + lane * kRopeStride,
-                         res + 32 * kRopeStride + lane * kRopeStride);
+                qkv_emit(R, n / R.attn_dim, (n % R.attn_dim) / 64, m, x, res + lane * 32, res + 32 * 32 + lane * 32,
+                         lane & 7);
               else
                 qkv_emit(R, n / R.attn_dim, (n % R.attn_dim) / 64, m, x);
             }
@@ -655,8 +685,7 @@ cudaError_t launch_bn(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
   int ctas = t.max_ctas > 0 ? t.max_ctas : g_num_sms;
   if (ctas > g.units) ctas = g.units;
   if (ctas < 1) ctas = 1;
-  tc_gemm_kernel<BN, SWAP><<<ctas, kThreads, C::kSmem, s>>>(*t.map_a, *t.map_b, g, e);
-  return cudaGetLastError();
+  return launch_k(tc_gemm_kernel<BN, SWAP>, dim3(ctas), dim3(kThreads), C::kSmem, s, *t.map_a, *t.map_b, g, e);
 }
 
 }  // namespace
@@ -671,6 +700,7 @@ cudaError_t prepare_tc_gemm() {
   if ((e = prepare_bn<128, true>()) != cudaSuccess) return e;
   if ((e = prepare_bn<256, true>()) != cudaSuccess) return e;
   if ((e = prepare_bn<64, false>()) != cudaSuccess) return e;
+  if ((e = prepare_bn<96, false>()) != cudaSuccess) return e;
   if ((e = prepare_bn<128, false>()) != cudaSuccess) return e;
   return prepare_bn<256, false>();
 }
@@ -689,6 +719,7 @@ cudaError_t launch_tc_gemm(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
   } else {
     switch (t.bn) {
       case 64: return launch_bn<64, false>(t, e, s);
+      case 96: return launch_bn<96, false>(t, e, s);
       case 128: return launch_bn<128, false>(t, e, s);
       case 256: return launch_bn<256, false>(t, e, s);
     }

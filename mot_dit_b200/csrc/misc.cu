@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -26,6 +27,8 @@ template <bool BF16>
 __global__ void __launch_bounds__(32 * kNormWarps)
     norm_mod_kernel(const float* __restrict__ x, void* __restrict__ h, int M, int d, const float* __restrict__ scale,
                     const float* __restrict__ shift, const float* __restrict__ gain) {
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.x * kNormWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
@@ -88,6 +91,8 @@ __global__ void __launch_bounds__(32 * kGemvWarps)
                 const float* __restrict__ bias, float* __restrict__ y, int N, int K, const float* __restrict__ T0,
                 size_t T_stride, int n_blocks, float* __restrict__ mod) {
   extern __shared__ float xs[];
+  pdl_trigger();
+  pdl_wait();
   if (mode == 2) {
     const double tt = (double)t[0];
     for (int k = threadIdx.x; k < 128; k += blockDim.x) {
@@ -155,6 +160,8 @@ __global__ void set_action_io_kernel(ActionIo* dst, ActionIo v) {
 
 __global__ void init_video_kernel(const VideoIo* __restrict__ io, float* __restrict__ x, int B, int Lc, int Lvid,
                                   int d) {
+  pdl_trigger();
+  pdl_wait();
   const size_t n = (size_t)B * (Lc + Lvid) * d;
   const float* video = io->video;
   const float* cond = io->cond;
@@ -174,6 +181,8 @@ __device__ __forceinline__ void write_in(void* a_in, bool bf16, size_t idx, floa
 
 __global__ void init_action_kernel(const ActionIo* __restrict__ io, float* __restrict__ a_state, void* a_in,
                                    int bf16, int M, int P, int ld_in) {
+  pdl_trigger();
+  pdl_wait();
   const float* src = io->a_in;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < M * P; i += gridDim.x * blockDim.x) {
     const float v = src[i];
@@ -184,6 +193,8 @@ __global__ void init_action_kernel(const ActionIo* __restrict__ io, float* __res
 
 __global__ void noise_action_kernel(const ActionIo* __restrict__ io, float* __restrict__ a_state, void* a_in,
                                     int bf16, int M, int P, int ld_in) {
+  pdl_trigger();
+  pdl_wait();
   const float sigma = io->sched[0];
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < M * P; i += gridDim.x * blockDim.x) {
     const float v = (1.0f - sigma) * io->a_clean[i] + sigma * io->a_in[i];
@@ -194,6 +205,8 @@ __global__ void noise_action_kernel(const ActionIo* __restrict__ io, float* __re
 
 __global__ void noise_video_kernel(const VideoIo* __restrict__ io, float* __restrict__ xs, void* x_act, int bf16,
                                    int n_rows, int P, int ld_act) {
+  pdl_trigger();
+  pdl_wait();
   const float sigma = io->t;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_rows * P; i += gridDim.x * blockDim.x) {
     const float v = (1.0f - sigma) * io->video[i] + sigma * io->eps[i];
@@ -203,6 +216,8 @@ __global__ void noise_video_kernel(const VideoIo* __restrict__ io, float* __rest
 }
 
 __global__ void copy_out_kernel(const ActionIo* __restrict__ io, const float* __restrict__ a, int n) {
+  pdl_trigger();
+  pdl_wait();
   float* out = io->a_out;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) out[i] = a[i];
 }
@@ -268,11 +283,8 @@ cudaError_t launch_norm_mod(const float* x, void* h, bool h_bf16, int M, int d, 
                             const float* shift, const float* gain, cudaStream_t s) {
   if (d % 4 != 0 || d > 32 * 4 * kNormV) return cudaErrorInvalidValue;
   dim3 grid((M + kNormWarps - 1) / kNormWarps);
-  if (h_bf16)
-    norm_mod_kernel<true><<<grid, 32 * kNormWarps, 0, s>>>(x, h, M, d, scale, shift, gain);
-  else
-    norm_mod_kernel<false><<<grid, 32 * kNormWarps, 0, s>>>(x, h, M, d, scale, shift, gain);
-  return cudaGetLastError();
+  if (h_bf16) return launch_k(norm_mod_kernel<true>, grid, dim3(32 * kNormWarps), 0, s, x, h, M, d, scale, shift, gain);
+  return launch_k(norm_mod_kernel<false>, grid, dim3(32 * kNormWarps), 0, s, x, h, M, d, scale, shift, gain);
 }
 
 cudaError_t launch_temb(const TembArgs& a, cudaStream_t s) {
@@ -283,13 +295,12 @@ cudaError_t launch_temb(const TembArgs& a, cudaStream_t s) {
   auto gemv = [&](const void* W, const float* x, int mode, const float* b, float* y, int N, int K, bool mod) {
     dim3 grid((N + kGemvWarps - 1) / kGemvWarps);
     const size_t sm = (size_t)(mode == 2 ? 256 : K) * sizeof(float);
+    float* modp = mod ? a.mod : nullptr;
     if (a.bf16)
-      gemv_kernel<true><<<grid, 32 * kGemvWarps, sm, s>>>(W, x, a.t, mode, b, y, N, K, a.T0, a.T_stride, a.n_blocks,
-                                                           mod ? a.mod : nullptr);
-    else
-      gemv_kernel<false><<<grid, 32 * kGemvWarps, sm, s>>>(W, x, a.t, mode, b, y, N, K, a.T0, a.T_stride,
-                                                            a.n_blocks, mod ? a.mod : nullptr);
-    return cudaGetLastError();
+      return launch_k(gemv_kernel<true>, grid, dim3(32 * kGemvWarps), sm, s, W, x, a.t, mode, b, y, N, K, a.T0,
+                      a.T_stride, a.n_blocks, modp);
+    return launch_k(gemv_kernel<false>, grid, dim3(32 * kGemvWarps), sm, s, W, x, a.t, mode, b, y, N, K, a.T0,
+                    a.T_stride, a.n_blocks, modp);
   };
   cudaError_t e;
   if ((e = gemv(a.w1, nullptr, 2, a.b1, c1, d, 256, false)) != cudaSuccess) return e;
@@ -299,32 +310,29 @@ cudaError_t launch_temb(const TembArgs& a, cudaStream_t s) {
 
 cudaError_t launch_init_video(const VideoIo* io, float* x, int B, int Lc, int Lvid, int d, cudaStream_t s) {
   const size_t n = (size_t)B * (Lc + Lvid) * d;
-  init_video_kernel<<<grid_for(n, 256), 256, 0, s>>>(io, x, B, Lc, Lvid, d);
-  return cudaGetLastError();
+  return launch_k(init_video_kernel, dim3(grid_for(n, 256)), dim3(256), 0, s, io, x, B, Lc, Lvid, d);
 }
 
 cudaError_t launch_init_action(const ActionIo* io, float* a_state, void* a_in, bool a_in_bf16, int M, int P,
                                int ld_in, cudaStream_t s) {
-  init_action_kernel<<<grid_for((size_t)M * P, 256), 256, 0, s>>>(io, a_state, a_in, a_in_bf16, M, P, ld_in);
-  return cudaGetLastError();
+  return launch_k(init_action_kernel, dim3(grid_for((size_t)M * P, 256)), dim3(256), 0, s, io, a_state, a_in,
+                  (int)a_in_bf16, M, P, ld_in);
 }
 
 cudaError_t launch_noise_action(const ActionIo* io, float* a_state, void* a_in, bool a_in_bf16, int M, int P,
                                 int ld_in, cudaStream_t s) {
-  noise_action_kernel<<<grid_for((size_t)M * P, 256), 256, 0, s>>>(io, a_state, a_in, a_in_bf16, M, P, ld_in);
-  return cudaGetLastError();
+  return launch_k(noise_action_kernel, dim3(grid_for((size_t)M * P, 256)), dim3(256), 0, s, io, a_state, a_in,
+                  (int)a_in_bf16, M, P, ld_in);
 }
 
 cudaError_t launch_noise_video(const VideoIo* io, float* x_sigma, void* x_act, bool act_bf16, int n_rows, int P,
                                int ld_act, cudaStream_t s) {
-  noise_video_kernel<<<grid_for((size_t)n_rows * P, 256), 256, 0, s>>>(io, x_sigma, x_act, act_bf16, n_rows, P,
-                                                                       ld_act);
-  return cudaGetLastError();
+  return launch_k(noise_video_kernel, dim3(grid_for((size_t)n_rows * P, 256)), dim3(256), 0, s, io, x_sigma, x_act,
+                  (int)act_bf16, n_rows, P, ld_act);
 }
 
 cudaError_t launch_copy_out(const ActionIo* io, const float* a_state, int n, cudaStream_t s) {
-  copy_out_kernel<<<grid_for(n, 256), 256, 0, s>>>(io, a_state, n);
-  return cudaGetLastError();
+  return launch_k(copy_out_kernel, dim3(grid_for(n, 256)), dim3(256), 0, s, io, a_state, n);
 }
 
 cudaError_t launch_set_video_io(VideoIo* dst, const VideoIo& v, cudaStream_t s) {
@@ -352,6 +360,14 @@ cudaError_t launch_rope_table(float* cos_t, float* sin_t, int L, int Dh, cudaStr
 cudaError_t launch_to_f32(const void* src, bool src_bf16, float* dst, size_t n, int cols, int ld, cudaStream_t s) {
   to_f32_kernel<<<grid_for(n, 256), 256, 0, s>>>(src, src_bf16, dst, n, cols, ld);
   return cudaGetLastError();
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("WAM_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
 }
 
 // ------------------------------------------------------- tensor maps -------

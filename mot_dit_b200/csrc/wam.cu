@@ -839,7 +839,14 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   size_t ws = 0;
   int tiles = 1;
   if (d.bf16) {
-    c->p_v_qkv = {128, 1, 0};
+    // Tiles and persistent grid sizes for the video GEMMs (config 2: 9 row
+    // tiles of 128): out-proj / FFN-down 1536/128 -> 108 units, one round on
+    // 108 SMs; QKV 4608/128 -> 324 units, three rounds -- on 108 CTAs, the same
+    // makespan as on all 148; FFN-up 6144/128 -> 432 units on all SMs.  The
+    // SMs the video GEMMs leave free run the action stream under CEWP.
+    const int v_rows = (d.Mv + 127) / 128;
+    const int ctas_third = std::min(std::max(1, (v_rows * (3 * d.A / 128) + 2) / 3), 148);
+    c->p_v_qkv = {128, 1, ctas_third};
     c->p_v_o = {128, 1, 0};
     c->p_v_f1 = {128, 1, 0};
     c->p_v_f2 = {128, 1, 0};
@@ -1248,6 +1255,16 @@ wam_status wam_op_linear(int dtype, const void* x, const void* w, const float* b
   g.tickets = tk;
   g.status = status;
   return launch_tc_gemm(g, e, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
+}
+
+wam_status wam_op_norm_mod(int dtype, const float* x, void* h, int M, int d, const float* scale, const float* shift,
+                           const float* gain, void* stream) {
+  if (!x || !h || M < 1 || d < 4 || d % 4 || d > 1536 || (!gain && !scale) ||
+      (dtype != WAM_BF16 && dtype != WAM_FP32))
+    return WAM_ERR_INVALID_ARG;
+  return launch_norm_mod(x, h, dtype == WAM_BF16, M, d, scale, shift, gain, (cudaStream_t)stream) == cudaSuccess
+             ? WAM_OK
+             : WAM_ERR_CUDA;
 }
 
 wam_status wam_op_attention(int dtype, const void* q, const void* k, const void* v, void* out, int B, int H, int Dh,

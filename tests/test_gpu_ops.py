@@ -92,3 +92,23 @@ def test_attention_f32():
     ref = M.merge_heads(M.attention(q.astype(np.float64), k[:, :, :Lk].astype(np.float64),
                                     v[:, :, :Lk].astype(np.float64))).reshape(B * Lq, H * Dh)
     assert rel_l2(out.cpu().numpy(), ref) < 1e-5
+
+
+@pytest.mark.parametrize("dtype,rows,d,mode", [(W.BF16, 1088, 1536, "mod"), (W.BF16, 32, 768, "mod"),
+                                             (W.BF16, 37, 768, "gain"), (W.FP32, 80, 64, "mod")])
+def test_norm_modulation(dtype, rows, d, mode):
+    """rms(x)(1 + scale) + shift (block prologue) and rms(x) * gain (final norm)."""
+    rng = np.random.default_rng(rows + d)
+    x = (3.0 * rng.standard_normal((rows, d))).astype(np.float32)
+    sc, sh, g = (rng.standard_normal(d).astype(np.float32) * 0.1 for _ in range(3))
+    tdt = torch.bfloat16 if dtype == W.BF16 else torch.float32
+    h = torch.full((rows, d), float("nan"), device=DEV, dtype=tdt)
+    if mode == "mod":
+        W.op_norm_mod(dtype, _f32(x), h, rows, d, scale=_f32(sc), shift=_f32(sh))
+        ref = M.modulate(x.astype(np.float64), sh.astype(np.float64), sc.astype(np.float64))
+    else:
+        W.op_norm_mod(dtype, _f32(x), h, rows, d, gain=_f32(g))
+        ref = M.rms_norm(x.astype(np.float64)) * g
+    torch.cuda.synchronize()
+    got = h.float().cpu().numpy()
+    assert rel_l2(got, ref) < (4e-3 if dtype == W.BF16 else 1e-6)
