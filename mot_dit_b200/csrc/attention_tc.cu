@@ -1,0 +1,355 @@
+// Video-query attention on the 5th-generation tensor cores (tcgen05).
+//
+// softmax(Q K^T / sqrt(64)) V for one (sample, head) and 128 queries per CTA,
+// over keys [0, Lk) of the per-block cache (the video expert's own keys;
+// RealtimeWAM summary page, 前置知识 "Mixture-of-Transformers": video queries
+// see video keys only).
+//
+// Per 128-key tile j:
+//   S_j  = Q K_j^T       tcgen05.mma M=128 N=128 K=64, fp32 in TMEM (128 cols)
+//   P_j  = exp2((S_j - m_j) log2e / 8)      softmax warps, thread = query row,
+//          rounded to bf16 into shared memory in the 128B-swizzled K-major
+//          layout the next MMA reads (fence.proxy.async before the hand-off)
+//   PV_j = P_j V_j       tcgen05.mma M=128 N=64 K=128, V as the MN-major B
+//          operand (the cache rows are [key][64 channels]), fp32 in TMEM
+//   O    = O alpha_j + PV_j in registers (online-softmax rescale)
+// The MMA warp issues S_{j+1} before PV_j, so the next scores are ready when
+// the softmax warps finish tile j; K/V tiles are double-buffered by TMA.
+//
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer, warps 2..5 softmax / output (warp w owns TMEM lanes 32*(w%4)..+31).
+// Every wait is bounded (see common.cuh).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace wam {
+namespace {
+
+constexpr int kQ = 128;       // queries per CTA
+constexpr int kKT = 128;      // keys per tile
+constexpr int kDh = 64;
+constexpr int kStagesKV = 2;
+constexpr int kTileBytes = kKT * kDh * 2;  // 16 KB (one K or V tile, also the Q tile)
+constexpr int kPBytes = kQ * kKT * 2;      // 32 KB
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 256;             // S: cols [0,128), PV: cols [128,192)
+constexpr int kBarBytes = 128;
+// No alignment slack: two CTAs per SM need every byte (2 x (112 KB + 1 KB reserved) <= 228 KB).
+constexpr int kSmem = kTileBytes + kStagesKV * 2 * kTileBytes + kPBytes + kBarBytes;
+
+// Shared-memory descriptor of an MN-major bf16 operand stored as rows of 128
+// bytes (64 elements along N) with the 128-byte swizzle, consecutive K rows
+// 128 B apart, 8-row groups 1024 B apart (a TMA SWIZZLE_128B tile of [K][64]).
+__device__ __forceinline__ uint64_t smem_desc_mn128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);  // start address
+  d |= static_cast<uint64_t>(1) << 16;                // leading byte offset (one 64-wide atom: unused)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;        // stride byte offset: 8 K-rows x 128 B
+  d |= static_cast<uint64_t>(1) << 46;                // descriptor version (sm_100)
+  d |= static_cast<uint64_t>(2) << 61;                // layout: 128-byte swizzle
+  return d;
+}
+
+__device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 32 lanes x 64 consecutive 32-bit columns, one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 2^x on the special-function unit (the hardware approximation, flushing
+// denormal results to zero; its relative error is far below bf16 rounding).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+struct AttnTcK {
+  int H, Lq, Lk, B;
+  int zq0, zk0, zv0;  // z (matrix) index of (b=0, h=0) in the Q / K / V maps
+  __nv_bfloat16* out;  // [B*Lq, H*64]
+  unsigned* status;
+};
+
+__global__ void __launch_bounds__(kThreads, 2)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                   const __grid_constant__ CUtensorMap map_v, const AttnTcK a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The 128-byte swizzle pattern is a function of the address bits: every tile
+  // must start on a 1024-byte boundary.
+  if (smem_u32(smem_raw) & 1023) {
+    if (threadIdx.x == 0) atomicOr(a.status, kStatusTimeoutDrain);
+    return;
+  }
+  uint8_t* smem = smem_raw;
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + kTileBytes;                       // [stage] K tiles
+  uint8_t* sV = sK + kStagesKV * kTileBytes;           // [stage] V tiles
+  uint8_t* sP = sV + kStagesKV * kTileBytes;           // two 64-key blocks of [128][128 B]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sP + kPBytes);
+  uint64_t* q_full = bar + 0;
+  uint64_t* kv_full = bar + 1;   // [2]
+  uint64_t* kv_empty = bar + 3;  // [2]
+  uint64_t* s_full = bar + 5;
+  uint64_t* p_full = bar + 6;
+  uint64_t* pv_full = bar + 7;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q0 = blockIdx.x * kQ, h = blockIdx.y, b = blockIdx.z;
+  const int bh = b * a.H + h;
+  const int ntiles = (a.Lk + kKT - 1) / kKT;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kStagesKV; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(pv_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&map_q);
+    prefetch_tensormap(&map_k);
+    prefetch_tensormap(&map_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_trigger();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      pdl_wait();
+      mbar_arrive_expect_tx(q_full, kTileBytes);
+      tma_load_3d(sQ, &map_q, q_full, 0, q0, a.zq0 + bh);
+      int issued = 0;
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j % kStagesKV;
+        if (j >= kStagesKV &&
+            !mbar_wait(&kv_empty[s], ((j / kStagesKV) - 1) & 1, a.status, kStatusTimeoutTmaEmpty, abort_flag))
+          break;
+        mbar_arrive_expect_tx(&kv_full[s], 2 * kTileBytes);
+        tma_load_3d(sK + s * kTileBytes, &map_k, &kv_full[s], 0, j * kKT, a.zk0 + bh);
+        tma_load_3d(sV + s * kTileBytes, &map_v, &kv_full[s], 0, j * kKT, a.zv0 + bh);
+        issued = j + 1;
+      }
+      mbar_wait(q_full, 0, a.status, kStatusTimeoutDrain, nullptr);
+      for (int j = max(0, issued - kStagesKV); j < issued; ++j)
+        mbar_wait(&kv_full[j % kStagesKV], (j / kStagesKV) & 1, a.status, kStatusTimeoutDrain, nullptr);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kQ, kKT);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kQ, kDh) | (1u << 16);  // B (V) is MN-major
+      const uint32_t t_s = tmem, t_pv = tmem + 128;
+      const uint32_t aq = smem_u32(sQ);
+      auto issue_s = [&](int j) {
+        const int s = j % kStagesKV;
+        if (!mbar_wait(&kv_full[s], (j / kStagesKV) & 1, a.status, kStatusTimeoutTmaFull, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t ak = smem_u32(sK + s * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kDh / 16; ++kk)
+          tc_mma_bf16(t_s, smem_desc_k128(aq + kk * 32), smem_desc_k128(ak + kk * 32), idesc_s, kk > 0 ? 1u : 0u);
+        tc_commit(s_full);
+        return true;
+      };
+      bool ok = mbar_wait(q_full, 0, a.status, kStatusTimeoutTmaFull, abort_flag) && issue_s(0);
+      for (int j = 0; j < ntiles && ok; ++j) {
+        // P_j written (and S_j, PV_{j-1} read) by the softmax warps
+        if (!mbar_wait(p_full, j & 1, a.status, kStatusTimeoutAccum, abort_flag)) break;
+        tc_fence_after();
+        if (j + 1 < ntiles && !issue_s(j + 1)) break;
+        const int s = j % kStagesKV;
+        const uint32_t ap = smem_u32(sP), av = smem_u32(sV + s * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kKT / 16; ++kk)
+          tc_mma_bf16(t_pv, smem_desc_k128(ap + (kk >> 2) * (kQ * 128) + (kk & 3) * 32),
+                      smem_desc_mn128(av + kk * 16 * 128), idesc_pv, kk > 0 ? 1u : 0u);
+        tc_commit(pv_full);
+        tc_commit(&kv_empty[s]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------ softmax warps
+    pdl_wait();
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // query row within the tile
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float sl2e = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
+    float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
+    float o[kDh];
+#pragma unroll
+    for (int i = 0; i < kDh; ++i) o[i] = 0.f;
+    uint8_t* prow = sP + r * 128;
+    const int swz = r & 7;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      if (!mbar_wait(s_full, j & 1, a.status, kStatusTimeoutAccum, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int kbase = j * kKT;
+      const int nvalid = min(kKT, a.Lk - kbase);  // keys of this tile inside [0, Lk)
+      // pass 1: row maximum of the valid keys
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kKT; c += 64) {
+        float v[64];
+        tmem_ld64(t_row + c, v);
+        if (nvalid == kKT) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) mx = fmaxf(mx, v[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (c + i < nvalid) mx = fmaxf(mx, v[i]);
+        }
+      }
+      const float m_new = fmaxf(m, mx);
+      const float alpha = ex2((m - m_new) * sl2e);  // m = -inf on the first tile: alpha = 0
+      const float mb = m_new * sl2e;
+      // O += PV_{j-1} (relative to the previous maximum); frees P and the PV columns
+      if (j > 0) {
+        if (!mbar_wait(pv_full, (j - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float pv[64];
+        tmem_ld64(t_row + 128, pv);
+#pragma unroll
+        for (int i = 0; i < kDh; ++i) o[i] = o[i] * alpha_prev + pv[i];
+      }
+      // pass 2: P = 2^(s log2e/8 - m log2e/8) as bf16 into the swizzled P tile
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < kKT; c += 64) {
+        float v[64];
+        tmem_ld64(t_row + c, v);
+        if (nvalid == kKT) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            v[i] = ex2(fmaf(v[i], sl2e, -mb));
+            rs += v[i];
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            v[i] = (c + i < nvalid) ? ex2(fmaf(v[i], sl2e, -mb)) : 0.f;
+            rs += v[i];
+          }
+        }
+        uint8_t* blk = prow + (c >> 6) * (kQ * 128);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint4 w;
+          w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+          w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+          w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+          w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+          *reinterpret_cast<uint4*>(blk + ((q ^ swz) << 4)) = w;
+        }
+      }
+      l = l * alpha + rs;
+      m = m_new;
+      alpha_prev = alpha;
+      tc_fence_before();
+      fence_proxy_async_smem();  // P (generic-proxy stores) -> tensor-core reads
+      mbar_arrive_cta(p_full);
+    }
+    if (ok && ntiles > 0 &&
+        mbar_wait(pv_full, (ntiles - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag)) {
+      tc_fence_after();
+      float pv[64];
+      tmem_ld64(t_row + 128, pv);
+#pragma unroll
+      for (int i = 0; i < kDh; ++i) o[i] = o[i] * alpha_prev + pv[i];
+      const int qi = q0 + r;
+      if (qi < a.Lq) {
+        const float inv = 1.0f / l;
+        uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)b * a.Lq + qi) * (a.H * kDh) + h * kDh);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint4 w;
+          w.x = pack_bf16(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
+          w.y = pack_bf16(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
+          w.z = pack_bf16(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
+          w.w = pack_bf16(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
+          dst[j] = w;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0 && ntiles > 0) mbar_wait(pv_full, (ntiles - 1) & 1, a.status, kStatusTimeoutDrain, nullptr);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t prepare_attention_tc() {
+  return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+}
+
+cudaError_t launch_attention_tc(const AttnTc& t, cudaStream_t s) {
+  if (t.Lq < 1 || t.Lk < 1) return cudaErrorInvalidValue;
+  AttnTcK k;
+  k.H = t.H;
+  k.Lq = t.Lq;
+  k.Lk = t.Lk;
+  k.B = t.B;
+  k.zq0 = t.zq0;
+  k.zk0 = t.zk0;
+  k.zv0 = t.zv0;
+  k.out = reinterpret_cast<__nv_bfloat16*>(t.out);
+  k.status = t.status;
+  dim3 grid((t.Lq + kQ - 1) / kQ, t.H, t.B);
+  return launch_k(attn_tc_kernel, grid, dim3(kThreads), kSmem, s, *t.map_q, *t.map_k, *t.map_v, k);
+}
+
+}  // namespace wam

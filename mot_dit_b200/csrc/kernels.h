@@ -147,6 +147,21 @@ struct AttnArgs {
   int* tickets;      // B*H counters, zero on entry, left zero
 };
 cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s);
+
+// Tensor-core (tcgen05) attention for video queries: one pass over keys
+// [0, Lk) for 128-query tiles.  Q / K / V are 3-D TMA maps over [z][rows][64]
+// bf16 (box 64 x 128); (b, h) reads matrix z0 + b*H + h of each map.
+struct AttnTc {
+  const CUtensorMap* map_q;
+  const CUtensorMap* map_k;
+  const CUtensorMap* map_v;
+  int zq0, zk0, zv0;
+  int B, H, Lq, Lk;
+  void* out;  // bf16 [B*Lq, H*64]
+  unsigned* status;
+};
+cudaError_t launch_attention_tc(const AttnTc& a, cudaStream_t s);
+cudaError_t prepare_attention_tc();
 cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t s);
 size_t attention_ws_floats(int B, int H, int Dh, int Lq, int splits);
 

@@ -98,6 +98,7 @@ struct wam_ctx {
   // TMA maps
   CUtensorMap m_hv, m_ov, m_fv, m_xvin, m_w_qkv_v, m_w_o_v, m_w_f1_v, m_w_f2_v, m_w_vin, m_w_vout;
   CUtensorMap m_w_in, m_w_qkv_a, m_w_o_a, m_w_f1_a, m_w_f2_a, m_w_out, m_ain, m_ha, m_oa, m_fa;
+  CUtensorMap m_qv, m_cache;  // video-attention operands
 
   // events and streams
   std::vector<cudaEvent_t> ev_kv, ev_kv_cap, ev_used;
@@ -426,6 +427,23 @@ wam_status attention(wam_ctx* c, bool video, int i, cudaStream_t s) {
   a.tickets = c->tk_attn;
   c->launches++;
   ProfScope ps(c, s);
+  if (d.bf16 && video) {
+    AttnTc t;
+    t.map_q = &c->m_qv;
+    t.map_k = &c->m_cache;
+    t.map_v = &c->m_cache;
+    t.zq0 = 0;
+    t.zk0 = (2 * i) * d.B * d.H;
+    t.zv0 = (2 * i + 1) * d.B * d.H;
+    t.B = d.B;
+    t.H = d.H;
+    t.Lq = d.Lv;
+    t.Lk = d.Lv;
+    t.out = c->o_v;
+    t.status = c->status;
+    CK(launch_attention_tc(t, s));
+    return WAM_OK;
+  }
   CK(d.bf16 ? launch_attention_bf16(a, s) : launch_attention_f32(a, s));
   return WAM_OK;
 }
@@ -778,6 +796,7 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   c->cfg = *cfg;
   CK(cudaGetDevice(&c->device));
   CK(prepare_tc_gemm());
+  CK(prepare_attention_tc());
   Dims& d = c->d;
   d.N = cfg->n_blocks; d.dv = cfg->d_video; d.da = cfg->d_action; d.H = cfg->n_heads; d.Dh = cfg->head_dim;
   d.A = d.H * d.Dh; d.Fv = cfg->ffn_video; d.Fa = cfg->ffn_action; d.Lc = cfg->l_cond; d.Lvid = cfg->l_video;
@@ -907,6 +926,8 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     amap(&c->m_ha, c->h_a, d.Ma, d.da, bna);
     amap(&c->m_oa, c->o_a, d.Ma, d.A, bna);
     amap(&c->m_fa, c->f_a, d.Ma, d.Fa, bna);
+    ok = ok && make_tmap_3d(&c->m_qv, c->q_v, d.Dh, d.Lv, d.B * d.H, (size_t)d.Lv * d.Dh * 2, 128);
+    ok = ok && make_tmap_3d(&c->m_cache, c->kv, d.Dh, d.Ltot, 2 * d.N * d.B * d.H, (size_t)d.Ltot * d.Dh * 2, 128);
     if (!ok) return fail(c, WAM_ERR_CUDA, "tensor map creation failed");
   }
 
@@ -1287,6 +1308,31 @@ wam_status wam_op_attention(int dtype, const void* q, const void* k, const void*
   cudaStream_t s = (cudaStream_t)stream;
   if (dtype == WAM_FP32) return launch_attention_f32(a, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
   if (dtype != WAM_BF16 || Dh != 64) return WAM_ERR_INVALID_ARG;
+  if (a.splits == 1) {  // single pass: the tcgen05 kernel
+    static thread_local unsigned* st = nullptr;
+    if (!st) {
+      if (prepare_attention_tc() != cudaSuccess) return WAM_ERR_CUDA;
+      if (cudaMalloc(&st, 4) != cudaSuccess) return WAM_ERR_OOM;
+      if (cudaMemset(st, 0, 4) != cudaSuccess) return WAM_ERR_CUDA;
+    }
+    CUtensorMap mq, mk, mv;
+    if (!make_tmap_3d(&mq, q, 64, Lq, B * H, (size_t)Lq * 128, 128) ||
+        !make_tmap_3d(&mk, k, 64, Lcache, B * H, (size_t)Lcache * 128, 128) ||
+        !make_tmap_3d(&mv, v, 64, Lcache, B * H, (size_t)Lcache * 128, 128))
+      return WAM_ERR_INVALID_ARG;
+    AttnTc t;
+    t.map_q = &mq;
+    t.map_k = &mk;
+    t.map_v = &mv;
+    t.zq0 = t.zk0 = t.zv0 = 0;
+    t.B = B;
+    t.H = H;
+    t.Lq = Lq;
+    t.Lk = Lk;
+    t.out = out;
+    t.status = st;
+    return launch_attention_tc(t, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
+  }
   if (a.splits > 1) {
     if (Lq > 64) return WAM_ERR_INVALID_ARG;
     static thread_local float* ws = nullptr;
