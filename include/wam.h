@@ -201,9 +201,13 @@ const char* wam_last_error(wam_ctx* ctx);
 
 /* C[M, N] = X[M, K] W[N, K]^T + bias (fp32 out), X / W bf16 (dtype WAM_BF16)
  * on the tcgen05 path or fp32 (WAM_FP32) on the SIMT path.  swap selects
- * the few-token orientation (weight on the 128-row MMA operand), splits its
- * split-K factor.  K must be a multiple of 64 and ld of X / W equal K on the
- * bf16 path.  Uses a private workspace; enqueued on `stream`. */
+ * the few-token orientation (weight on the 128-row MMA operand, M <= 256).
+ * The bf16 path splits the k-blocks of all output tiles evenly over its
+ * persistent CTAs (stream-K; partial tiles summed in k order): `splits` is
+ * the number of CTAs per output tile when swapped, else the number of CTAs
+ * (0: one per SM).  K must be a multiple of 64, ld of X / W equal K, and N a
+ * multiple of 32 unless swapped, on the bf16 path.  Uses a private workspace
+ * (allocated on first use or growth); enqueued on `stream`. */
 wam_status wam_op_linear(int dtype, const void* dev_x, const void* dev_w, const float* dev_bias, float* dev_out,
                          int M, int N, int K, int swap, int splits, void* stream);
 

@@ -20,6 +20,7 @@ enum : unsigned {
   kStatusTimeoutTmaEmpty = 1u << 1,  // producer waited too long for a free stage
   kStatusTimeoutAccum = 1u << 2,     // epilogue waited too long for the accumulator
   kStatusTimeoutDrain = 1u << 3,     // teardown waited too long for copies in flight
+  kStatusTimeoutPeer = 1u << 4,      // waited too long for another CTA's partial tile
 };
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s

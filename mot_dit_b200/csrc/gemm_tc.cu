@@ -8,26 +8,34 @@
 // the fused epilogue (bias, gate-residual, GELU, QK-norm + RoPE + K/V publish,
 // Euler update, video endpoint).
 //
-// Persistent: each CTA walks a static, strided list of work units (tile x
-// split), so the schedule -- and every reduction order -- is a function of the
-// launch configuration only.  The accumulator is double-buffered in TMEM
-// (2 x BN columns): the MMA warp fills buffer b of unit j+1 while the epilogue
-// warps drain buffer b^1 of unit j.
+// Schedule (stream-K): the k-blocks of all output tiles, tile after tile, form
+// one range of W = tiles x KB blocks, and persistent CTA c of G owns blocks
+// [W c / G, W (c+1) / G).  Every CTA gets the same amount of MMA work however
+// the tile count falls on the SMs.  A tile whose k-range is shared by several
+// CTAs is finished by the last of its pieces to arrive (integer ticket), which
+// sums the fp32 partials in piece (= k) order: the result does not depend on
+// timing.  The accumulator is double-buffered in TMEM (2 x BN columns): the
+// MMA warp fills one while the epilogue warps drain the other.
+//
+// Split tiles.  Each piece takes an arrival ticket when its accumulator is
+// ready.  Every piece but the last to arrive publishes its fp32 partial to the
+// workspace and counts itself published; the last one waits (bounded) for
+// those counts -- of pieces that have already arrived, so the wait never
+// depends on a CTA that is not running -- and adds the partials, in piece
+// order, to its own accumulator read from TMEM.  The last arrival is almost
+// always piece 0, the final segment of its CTA: the shared-memory ring is
+// idle by then, and the partials come in with bulk copies.
 //
 // Orientation.  Normal: A = X (128 tokens on TMEM lanes), B = W (BN features).
 // Swapped (few tokens, e.g. the action expert's 32): A = W (128 features on
 // TMEM lanes), B = X (BN tokens) -- the weight stream fills the 128-row MMA
 // operand instead of padding the token dimension.
 //
-// Split-K (swapped only): each unit reduces a K range into TMEM and writes an
-// fp32 partial tile; the last unit of a tile (integer ticket) sums the
-// partials in split order 0..S-1 -- a fixed order, so the result does not
-// depend on which CTA finishes last.
-//
-// Epilogue stores are coalesced: a 32 x 32 sub-tile held one-row-per-thread
-// after tcgen05.ld goes through padded shared memory and is written one row
-// per warp instruction (32 consecutive columns), except the QK-norm + RoPE
-// epilogue, which keeps a head's 64 channels in one thread.
+// Epilogue stores of the normal orientation go through shared memory: each
+// epilogue warp writes its 32-row output box in the 128-byte-swizzled layout
+// and one lane issues a TMA bulk-tensor store.  The gate-residual rows are
+// prefetched into that staging with cp.async while the MMA runs and updated in
+// place; the QKV epilogue prefetches its tokens' RoPE rows the same way.
 //
 // Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
 // issuer, warps 2..5 epilogue (warp w reads TMEM lanes 32*(w%4) .. +31).
@@ -42,46 +50,124 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int kThreads = 192;
+constexpr int kBox = 4096;  // one output box: 32 rows x 128 bytes
 
-template <int BN, bool SWAP>
+// Epilogue class of a kernel instance: which shared-memory staging it carries.
+enum : int {
+  kClassScalar = 0,  // per-element stores (Euler update, video endpoint; every swapped epilogue)
+  kClassStore = 1,   // fp32 store / GELU: two output boxes per warp
+  kClassRes = 2,     // gate-residual: the warp's 32 x BN residual rows (BN <= 128)
+  kClassQkv = 3,     // QK-norm + RoPE: 32 cos + 32 sin rows and two output boxes per warp
+};
+
+template <int BN, bool SWAP, int EPI>
 struct TileCfg {
   static constexpr int kABytes = BM * BK * 2;
   static constexpr int kBBytes = BN * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
-  // Normal orientation, BN <= 128: each epilogue warp prefetches its 32 x BN
-  // residual rows (gate-residual) or 32 RoPE rows (QKV) while the MMA runs.
-  static constexpr bool kPrefetch = !SWAP && BN <= 128;
-  static constexpr int kResBytes = kPrefetch ? 4 * 32 * BN * 4 : 0;
-  // Swapped orientation: [32 tokens][128 features + 1] fp32 staging of the QKV epilogue.
-  static constexpr int kEpiBytes = SWAP ? 32 * (BM + 1) * 4 : 0;
+  static constexpr int kWarpStg = SWAP ? 0
+                                       : (EPI == kClassStore ? 2 * kBox
+                                                             : (EPI == kClassRes ? 32 * BN * 4
+                                                                                 : (EPI == kClassQkv ? 4 * kBox : 0)));
+  static constexpr int kSwapStg = SWAP ? 32 * (BM + 1) * 4 : 0;  // swapped QKV staging [32 tokens][129]
+  // the tile's bias slice (and gate or QK gains) in shared memory, normal orientation
+  static constexpr int kVecBytes = (SWAP || EPI == kClassScalar) ? 0 : (EPI == kClassStore ? 1 : 2) * BN * 4;
+  static constexpr int kExtra = 4 * kWarpStg + kSwapStg + kVecBytes;
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemMax = 232448;  // 227 KB per CTA
-  static constexpr int kFit = (kSmemMax - 1024 - kBarBytes - kResBytes - kEpiBytes) / kStageBytes;
-  static constexpr int kStages = kFit > 8 ? 8 : kFit;  // deep ring: TMA latency > a few MMA k-blocks
-  static constexpr int kSmem = kStages * kStageBytes + kEpiBytes + kResBytes + kBarBytes + 1024;
+  static constexpr int kFit = (kSmemMax - 1024 - kBarBytes - kExtra) / kStageBytes;
+  static constexpr int kStages = kFit > 8 ? 8 : kFit;
+  static constexpr int kSmem = kStages * kStageBytes + kExtra + kBarBytes + 1024;
   static_assert(kStages >= 3, "shared memory ring too shallow");
+  static_assert(EPI != kClassRes || BN <= 128, "residual staging holds at most 128 columns");
 };
 
 struct GemmK {
   int rows_a, rows_b, K;
   int z_a, z_b;
-  int tiles_a, tiles_b;
-  int kb_per_split, splits;
-  int units;
-  float* ws;
-  int* tickets;
+  int tiles_a;
+  int KB;        // k-blocks per tile
+  long long W;   // k-blocks of all tiles
+  int G;         // CTAs sharing them
+  float* ws;     // [G][2][BM * BN] partial tiles
+  int* tickets;  // [tiles][2]: pieces arrived, pieces published
   unsigned* status;
 };
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// First k-block of CTA c, and the CTA owning k-block x (the largest c with
+// W c / G <= x).
+__device__ __forceinline__ long long kbound(const GemmK& g, int c) { return g.W * c / g.G; }
+__device__ __forceinline__ int kowner(const GemmK& g, long long x) { return (int)(((x + 1) * g.G - 1) / g.W); }
 
-__device__ __forceinline__ void store_act(void* base, size_t idx, float v) {
-  reinterpret_cast<__nv_bfloat16*>(base)[idx] = __float2bfloat16_rn(v);
-}
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Generic-proxy writes to shared memory become visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// 3-D tiled store shared -> global; out-of-range rows / columns are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Contiguous bulk copy global -> shared completing `bytes` on `bar` (no multicast).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+// Later async-proxy reads of global memory see what this thread has observed.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Bounded wait until *count >= target (a counter other CTAs increment).
+__device__ __forceinline__ bool wait_count(const int* count, int target, unsigned* status, volatile int* abort) {
+  const volatile int* vc = count;
+  const unsigned long long t0 = globaltimer();
+  while (*vc < target) {
+    if (abort && *abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      atomicOr(status, kStatusTimeoutPeer);
+      return false;
+    }
+    __nanosleep(32);
+  }
+  return true;
+}
+
+// 16-byte chunk q of row r (0..31) of a 32 x 128-byte box: the layout a TMA
+// box with the 128-byte swizzle has in shared memory (chunk q at q ^ (r & 7)).
+__device__ __forceinline__ uint4* box_chunk(uint8_t* box, int r, int q) {
+  return reinterpret_cast<uint4*>(box + r * 128 + ((q ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void box_row_f32(uint8_t* box, int r, const float* v) {  // 32 values
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *box_chunk(box, r, q) = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                       __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+}
+__device__ __forceinline__ void box_row_bf16(uint8_t* box, int r, const float* v) {  // 64 values
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    uint4 w;
+    w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+    *box_chunk(box, r, q) = w;
+  }
 }
 
 // Epilogue arguments copied into registers once: the store loops never
@@ -102,6 +188,7 @@ struct EpiRegs {
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
   int seq_len, cache_len, cache_off, n_heads, attn_dim;
+  int zq0, zk0, zv0;
 };
 
 __device__ __forceinline__ EpiRegs hoist(const EpiArgs& e) {
@@ -124,52 +211,59 @@ __device__ __forceinline__ EpiRegs hoist(const EpiArgs& e) {
   r.cache_off = e.cache_off;
   r.n_heads = e.n_heads;
   r.attn_dim = e.attn_dim;
+  r.zq0 = e.zq0;
+  r.zk0 = e.zk0;
+  r.zv0 = e.zv0;
   return r;
 }
 
-// Per-head QK-RMSNorm (gain), RoPE, and scatter of one 64-channel head vector
-// of token m.  section: 0 = q, 1 = k, 2 = v.  cs_row / sn_row: the token's
-// cos / sin row, prefetched in shared memory with its 16-byte chunks permuted
-// by XOR with swz (or null to read the table).
-__device__ __forceinline__ void qkv_emit(const EpiRegs& R, int section, int head, int m, float (&x)[64],
-                                         const float* cs_row = nullptr, const float* sn_row = nullptr,
-                                         int swz = 0) {
-  const int b = m / R.seq_len, l = m - b * R.seq_len;
-  if (section < 2) {
-    const float4* g4 = reinterpret_cast<const float4*>((section == 0 ? R.gq : R.gk) + head * 64);
-    float ss = 0.f;
+// Per-head QK-RMSNorm (gain) and RoPE of the 64-channel head vector x of
+// token m (section 0 = q, 1 = k; 2 = v is left as is).  cs_row / sn_row: the
+// token's cos / sin row in shared memory with 16-byte chunk q at q ^ swz, or
+// null to read the tables.
+__device__ __forceinline__ void qk_norm_rope(const EpiRegs& R, int section, int head, int m, float (&x)[64],
+                                             const float* cs_row, const float* sn_row, int swz,
+                                             const float* gain = nullptr) {
+  if (section >= 2) return;
+  const int l = m % R.seq_len;
+  const float4* g4 = reinterpret_cast<const float4*>(gain ? gain : (section == 0 ? R.gq : R.gk) + head * 64);
+  float ss = 0.f;
 #pragma unroll
-    for (int j = 0; j < 64; ++j) ss += x[j] * x[j];
-    const float r = rsqrtf(ss * (1.0f / 64.0f) + 1e-6f);
+  for (int j = 0; j < 64; ++j) ss += x[j] * x[j];
+  const float r = rsqrtf(ss * (1.0f / 64.0f) + 1e-6f);
 #pragma unroll
-    for (int j4 = 0; j4 < 16; ++j4) {
-      const float4 gg = __ldg(g4 + j4);
-      x[4 * j4] *= r * gg.x;
-      x[4 * j4 + 1] *= r * gg.y;
-      x[4 * j4 + 2] *= r * gg.z;
-      x[4 * j4 + 3] *= r * gg.w;
-    }
-    const int pos = R.cache_off + l;
-    const float4* cs = reinterpret_cast<const float4*>(cs_row ? cs_row : R.rope_cos + pos * 32);
-    const float4* sn = reinterpret_cast<const float4*>(sn_row ? sn_row : R.rope_sin + pos * 32);
+  for (int j4 = 0; j4 < 16; ++j4) {
+    const float4 gg = gain ? g4[j4] : __ldg(g4 + j4);
+    x[4 * j4] *= r * gg.x;
+    x[4 * j4 + 1] *= r * gg.y;
+    x[4 * j4 + 2] *= r * gg.z;
+    x[4 * j4 + 3] *= r * gg.w;
+  }
+  const int pos = R.cache_off + l;
+  const float4* cs = reinterpret_cast<const float4*>(cs_row ? cs_row : R.rope_cos + pos * 32);
+  const float4* sn = reinterpret_cast<const float4*>(sn_row ? sn_row : R.rope_sin + pos * 32);
 #pragma unroll
-    for (int j4 = 0; j4 < 8; ++j4) {
-      const float4 c4 = cs[cs_row ? (j4 ^ swz) : j4], s4 = sn[sn_row ? (j4 ^ swz) : j4];
-      const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss4[4] = {s4.x, s4.y, s4.z, s4.w};
+  for (int j4 = 0; j4 < 8; ++j4) {
+    const float4 c4 = cs[cs_row ? (j4 ^ swz) : j4], s4 = sn[sn_row ? (j4 ^ swz) : j4];
+    const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ss4[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int j = 4 * j4 + q;
-        const float x1 = x[j], x2 = x[j + 32];
-        x[j] = x1 * cc[q] - x2 * ss4[q];
-        x[j + 32] = x1 * ss4[q] + x2 * cc[q];
-      }
+    for (int q = 0; q < 4; ++q) {
+      const int j = 4 * j4 + q;
+      const float x1 = x[j], x2 = x[j + 32];
+      x[j] = x1 * cc[q] - x2 * ss4[q];
+      x[j + 32] = x1 * ss4[q] + x2 * cc[q];
     }
   }
-  __nv_bfloat16* dst;
-  if (section == 0)
-    dst = R.q_out + ((size_t)(b * R.n_heads + head) * R.seq_len + l) * 64;
-  else
-    dst = (section == 1 ? R.k_cache : R.v_cache) + ((size_t)(b * R.n_heads + head) * R.cache_len + R.cache_off + l) * 64;
+}
+
+// Global row of token m, head `head` in Q (section 0) or the K / V cache.
+__device__ __forceinline__ __nv_bfloat16* qkv_dst(const EpiRegs& R, int section, int head, int m) {
+  const int b = m / R.seq_len, l = m - b * R.seq_len;
+  if (section == 0) return R.q_out + ((size_t)(b * R.n_heads + head) * R.seq_len + l) * 64;
+  return (section == 1 ? R.k_cache : R.v_cache) + ((size_t)(b * R.n_heads + head) * R.cache_len + R.cache_off + l) * 64;
+}
+
+__device__ __forceinline__ void store_head(__nv_bfloat16* dst, const float (&x)[64]) {
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -193,13 +287,13 @@ __device__ __forceinline__ void epi_elem(const EpiArgs& e, int m, int n, float y
       e.out_f32[idx] += gate * y;
       break;
     case kEpiGelu:
-      store_act(e.out_act, idx, gelu_tanh(y));
+      reinterpret_cast<__nv_bfloat16*>(e.out_act)[idx] = __float2bfloat16_rn(gelu_tanh(y));
       break;
     case kEpiEuler: {
       const float dt = e.aio->sched[e.step] - e.aio->sched[e.step + 1];
       const float a = e.out_f32[idx] - dt * y;
       e.out_f32[idx] = a;
-      if (e.a_next) store_act(e.a_next, (size_t)m * e.a_next_ld + n, a);
+      if (e.a_next) reinterpret_cast<__nv_bfloat16*>(e.a_next)[(size_t)m * e.a_next_ld + n] = __float2bfloat16_rn(a);
       break;
     }
     case kEpiVideoOut: {
@@ -215,28 +309,43 @@ __device__ __forceinline__ void epi_elem(const EpiArgs& e, int m, int n, float y
   }
 }
 
-template <int BN, bool SWAP>
+// The next segment of a CTA's k-block range starting at x: tile t, k-blocks
+// [kb0, kb1) of it.
+struct Seg {
+  int t, kb0, kb1;
+};
+__device__ __forceinline__ Seg seg_at(const GemmK& g, long long x, long long x_end) {
+  Seg s;
+  s.t = (int)(x / g.KB);
+  s.kb0 = (int)(x - (long long)s.t * g.KB);
+  const long long lim = s.kb0 + (x_end - x);
+  s.kb1 = lim < g.KB ? (int)lim : g.KB;
+  return s;
+}
+
+template <int BN, bool SWAP, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                   const __grid_constant__ CUtensorMap map_o, const __grid_constant__ CUtensorMap map_o2,
                    const GemmK g, const EpiArgs e) {
-  using C = TileCfg<BN, SWAP>;
+  using C = TileCfg<BN, SWAP, EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kStages * C::kABytes;
-  float* sEpi = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);  // swapped QKV staging
-  float* sRes = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + C::kEpiBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes + C::kEpiBytes + C::kResBytes);
+  uint8_t* sStg = smem + C::kStages * C::kStageBytes;  // epilogue staging (1024-byte aligned)
+  float* sVec = reinterpret_cast<float*>(sStg + 4 * C::kWarpStg + C::kSwapStg);  // [BN] bias, [BN] gate / gains
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + C::kExtra);
   uint64_t* empty = full + C::kStages;
   uint64_t* accf = empty + C::kStages;  // [2] accumulator ready (MMA -> epilogue)
   uint64_t* acce = accf + 2;            // [2] accumulator drained (epilogue -> MMA)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+  uint64_t* redb = acce + 2;            // partial tiles copied into the ring
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redb + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb_total = (g.K + BK - 1) / BK;
-  const int per_tile_units = g.splits;
+  const long long x_begin = kbound(g, blockIdx.x), x_end = kbound(g, blockIdx.x + 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -247,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&accf[b], 1);
       mbar_init(&acce[b], 4);
     }
+    mbar_init(redb, 1);
     *abort_flag = 0;
     *last_flag = 0;
     fence_barrier_init();
@@ -254,6 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&map_a);
     prefetch_tensormap(&map_b);
+    if (!SWAP && EPI != kClassScalar) prefetch_tensormap(&map_o);
+    if (!SWAP && EPI == kClassQkv) prefetch_tensormap(&map_o2);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -265,49 +377,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   pdl_trigger();  // the next kernel may start its own set-up now
 
-  // unit u -> (tile_a, tile_b, split); split fastest, then tile_a, then tile_b
-  auto decode = [&](int u, int& ta, int& tb, int& sp) {
-    sp = u % per_tile_units;
-    const int t = u / per_tile_units;
-    ta = t % g.tiles_a;
-    tb = t / g.tiles_a;
-  };
-
   if (warp == 0) {
     if (lane == 0) {
       int it = 0, issued = 0;
       bool ok = true;
-      // The weights never change during a chunk: the first unit's weight tiles
-      // are requested before waiting for the previous kernel (dependent launch).
+      // The weights never change during a chunk: the first segment's weight
+      // tiles are requested before waiting for the previous kernel.
       int pre = 0;
-      if (blockIdx.x < g.units) {
-        int ta, tb, sp;
-        decode(blockIdx.x, ta, tb, sp);
-        const int kb0 = sp * g.kb_per_split, kb1 = min(kb_total, kb0 + g.kb_per_split);
-        pre = min(C::kStages, kb1 - kb0);
+      if (x_begin < x_end) {
+        const Seg sg = seg_at(g, x_begin, x_end);
+        const int ta = sg.t % g.tiles_a, tb = sg.t / g.tiles_a;
+        pre = min(C::kStages, sg.kb1 - sg.kb0);
         for (int i = 0; i < pre; ++i) {
           mbar_arrive_expect_tx(&full[i], C::kStageBytes);
           if (SWAP)
-            tma_load_3d(sA + i * C::kABytes, &map_a, &full[i], (kb0 + i) * BK, ta * BM, g.z_a);
+            tma_load_3d(sA + i * C::kABytes, &map_a, &full[i], (sg.kb0 + i) * BK, ta * BM, g.z_a);
           else
-            tma_load_3d(sB + i * C::kBBytes, &map_b, &full[i], (kb0 + i) * BK, tb * BN, g.z_b);
+            tma_load_3d(sB + i * C::kBBytes, &map_b, &full[i], (sg.kb0 + i) * BK, tb * BN, g.z_b);
         }
         pdl_wait();
         for (int i = 0; i < pre; ++i) {
           if (SWAP)
-            tma_load_3d(sB + i * C::kBBytes, &map_b, &full[i], (kb0 + i) * BK, tb * BN, g.z_b);
+            tma_load_3d(sB + i * C::kBBytes, &map_b, &full[i], (sg.kb0 + i) * BK, tb * BN, g.z_b);
           else
-            tma_load_3d(sA + i * C::kABytes, &map_a, &full[i], (kb0 + i) * BK, ta * BM, g.z_a);
+            tma_load_3d(sA + i * C::kABytes, &map_a, &full[i], (sg.kb0 + i) * BK, ta * BM, g.z_a);
         }
         issued = pre;
       } else {
         pdl_wait();
       }
-      for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x) {
-        int ta, tb, sp;
-        decode(u, ta, tb, sp);
-        const int kb0 = sp * g.kb_per_split, kb1 = min(kb_total, kb0 + g.kb_per_split);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+      for (long long x = x_begin; x < x_end && ok;) {
+        const Seg sg = seg_at(g, x, x_end);
+        x += sg.kb1 - sg.kb0;
+        const int ta = sg.t % g.tiles_a, tb = sg.t / g.tiles_a;
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
           if (it < pre) continue;  // issued above
           const int s = it % C::kStages;
           if (it >= C::kStages &&
@@ -330,10 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
       int it = 0, lt = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < g.units && ok; u += gridDim.x, ++lt) {
-        int ta, tb, sp;
-        decode(u, ta, tb, sp);
-        const int kb0 = sp * g.kb_per_split, kb1 = min(kb_total, kb0 + g.kb_per_split);
+      for (long long x = x_begin; x < x_end && ok; ++lt) {
+        const Seg sg = seg_at(g, x, x_end);
+        x += sg.kb1 - sg.kb0;
         const int buf = lt & 1;
         if (lt >= 2 && !mbar_wait(&acce[buf], ((lt >> 1) - 1) & 1, g.status, kStatusTimeoutAccum, abort_flag)) {
           ok = false;
@@ -341,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + buf * BN;
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
           const int s = it % C::kStages;
           if (!mbar_wait(&full[s], (it / C::kStages) & 1, g.status, kStatusTimeoutTmaFull, abort_flag)) {
             ok = false;
@@ -353,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             tc_mma_bf16(d_tmem, smem_desc_k128(a0 + k * 32), smem_desc_k128(b0 + k * 32), idesc,
-                        (kb > kb0 || k > 0) ? 1u : 0u);
+                        (kb > sg.kb0 || k > 0) ? 1u : 0u);
           tc_commit(&empty[s]);
         }
         tc_commit(&accf[buf]);
@@ -364,43 +466,75 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     pdl_wait();  // outputs / residual rows belong to the previous kernel until it is done
     const int quad = warp & 3;
-    const int row = quad * 32 + lane;
+    const int row = quad * 32 + lane;  // TMEM lane = tile row
     const EpiRegs R = hoist(e);
-    float* res = sRes + quad * (32 * BN);  // this warp's prefetched residual rows / RoPE rows
-    constexpr bool kRopeFits = C::kPrefetch && BN >= 64;  // 32 cos + 32 sin rows of 32 floats
+    uint8_t* stg = sStg + quad * C::kWarpStg;  // this warp's staging (normal orientation)
+    int nbox = 0;                              // output boxes this warp stored (double-buffer index)
     int lt = 0;
-    for (int u = blockIdx.x; u < g.units; u += gridDim.x, ++lt) {
-      int ta, tb, sp;
-      decode(u, ta, tb, sp);
+    for (long long x = x_begin; x < x_end; ++lt) {
+      const bool first_seg = (x == x_begin);
+      const Seg sg = seg_at(g, x, x_end);
+      x += sg.kb1 - sg.kb0;
+      const int t = sg.t;
+      const int ta = t % g.tiles_a, tb = t / g.tiles_a;
+      const long long t0 = (long long)t * g.KB;
+      const int c_first = kowner(g, t0);
+      const int npieces = kowner(g, t0 + g.KB - 1) - c_first + 1;
       const int buf = lt & 1;
+      const int m0w = ta * BM + quad * 32;  // normal orientation: this warp's first row
+      const int nb = tb * BN;
+
+      // ---- prefetch while the MMA of this segment runs
       bool prefetched = false;
-      if constexpr (C::kPrefetch) {
-        // While the MMA of this unit runs: bring this warp's residual rows
-        // (16-byte chunk q of row r at chunk q ^ (r & 7): thread-per-row
-        // reads are then conflict-free) or its tokens' RoPE rows into smem.
-        const int m0 = ta * BM + quad * 32, nb = tb * BN;
-        if (R.kind == kEpiGateRes) {
-          for (int k = lane; k < 32 * (BN / 4); k += 32) {
-            const int r = k / (BN / 4), q = k % (BN / 4);
-            const int m = m0 + r, n = nb + 4 * q;
-            const bool v = m < g.rows_a && n < g.rows_b;
-            cp_async16(smem_u32(res + r * BN + 4 * (q ^ (r & 7))),
-                       v ? (const void*)(R.out_f32 + (size_t)m * R.ld + n) : (const void*)R.out_f32, v);
-          }
-          cp_async_commit();
-          prefetched = true;
-        } else if (kRopeFits && R.kind == kEpiQkv) {
-          for (int k = lane; k < 32 * 16; k += 32) {
-            const int r = k >> 4, which = (k >> 3) & 1, c4 = k & 7;
-            const int m = min(m0 + r, g.rows_a - 1);
-            const int pos = R.cache_off + (m % R.seq_len);
-            const float* src = (which ? R.rope_sin : R.rope_cos) + pos * 32 + 4 * c4;
-            cp_async16(smem_u32(res + which * (32 * 32) + r * 32 + 4 * (c4 ^ (r & 7))), src, true);
+      if constexpr (C::kVecBytes > 0) {
+        // every warp is done with the previous segment's vectors
+        epi_bar();
+        if (quad == 0) {
+          for (int q4 = lane; q4 < BN / 4; q4 += 32) {
+            const int n = nb + 4 * q4;
+            const bool v = n < g.rows_b;
+            cp_async16(smem_u32(sVec + 4 * q4), v ? (const void*)(R.bias + n) : (const void*)R.bias, v);
+            if constexpr (EPI == kClassRes) {
+              cp_async16(smem_u32(sVec + BN + 4 * q4), v ? (const void*)(R.gate + n) : (const void*)R.gate, v);
+            } else if constexpr (EPI == kClassQkv) {
+              // gain of column n: q or k RMSNorm gain of its head channel; v columns take none
+              const int section = n / R.attn_dim;
+              const float* gsrc = section == 0 ? R.gq : R.gk;
+              const bool gv = v && section < 2;
+              cp_async16(smem_u32(sVec + BN + 4 * q4), gv ? (const void*)(gsrc + n % R.attn_dim) : (const void*)R.gq,
+                         gv);
+            }
           }
           cp_async_commit();
           prefetched = true;
         }
       }
+      if constexpr (!SWAP && (EPI == kClassRes || EPI == kClassQkv)) {
+        if (lane == 0) bulk_wait_read<0>();  // earlier stores have left the staging
+        __syncwarp();
+        if constexpr (EPI == kClassRes) {
+          // residual rows; box b holds columns [32 b, 32 b + 32) in the store layout
+          for (int k = lane; k < 32 * (BN / 4); k += 32) {
+            const int r = k / (BN / 4), q4 = k % (BN / 4);
+            const int m = m0w + r, n = nb + 4 * q4;
+            const bool v = m < g.rows_a && n < g.rows_b;
+            cp_async16(smem_u32(box_chunk(stg + (q4 >> 3) * kBox, r, q4 & 7)),
+                       v ? (const void*)(R.out_f32 + (size_t)m * R.ld + n) : (const void*)R.out_f32, v);
+          }
+        } else {
+          // cos rows of the warp's 32 tokens at [0, 4 KB), sin rows at [4 KB, 8 KB)
+          for (int k = lane; k < 32 * 16; k += 32) {
+            const int r = k >> 4, which = (k >> 3) & 1, c4 = k & 7;
+            const int m = min(m0w + r, g.rows_a - 1);
+            const int pos = R.cache_off + (m % R.seq_len);
+            const float* src = (which ? R.rope_sin : R.rope_cos) + pos * 32 + 4 * c4;
+            cp_async16(smem_u32(box_chunk(stg + which * kBox, r, c4)), src, true);
+          }
+        }
+        cp_async_commit();
+        prefetched = true;
+      }
+
       const bool ok = mbar_wait(&accf[buf], (lt >> 1) & 1, g.status, kStatusTimeoutAccum, abort_flag);
       if (prefetched) {
         cp_async_wait<0>();
@@ -419,44 +553,237 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&acce[buf]);
       };
 
-      if (!SWAP) {
-        // thread = output row m, 32 consecutive features per TMEM load
-        const int m = ta * BM + quad * 32 + lane;
-        const int nb = tb * BN;
-        const bool m_ok = m < g.rows_a;
-        if (R.kind == kEpiQkv) {
-          for (int c = 0; c < BN; c += 64) {
-            float x[64];
-            float (&lo)[32] = *reinterpret_cast<float(*)[32]>(&x[0]);
-            float (&hi)[32] = *reinterpret_cast<float(*)[32]>(&x[32]);
-            tmem_ld32(t_row + c, lo);
-            tmem_ld32(t_row + c + 32, hi);
-            if (c + 64 >= BN) release();
-            const int n = nb + c;
-            if (m_ok && n < g.rows_b) {
-              const float4* b4 = reinterpret_cast<const float4*>(R.bias + n);
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const float4 bb = __ldg(b4 + j);
-                x[4 * j] += bb.x;
-                x[4 * j + 1] += bb.y;
-                x[4 * j + 2] += bb.z;
-                x[4 * j + 3] += bb.w;
-              }
-              if constexpr (kRopeFits)
-                qkv_emit(R, n / R.attn_dim, (n % R.attn_dim) / 64, m, x, res + lane * 32, res + 32 * 32 + lane * 32,
-                         lane & 7);
-              else
-                qkv_emit(R, n / R.attn_dim, (n % R.attn_dim) / 64, m, x);
-            }
-          }
-        } else {
+      // ---- a tile shared with other CTAs (see "Split tiles" above)
+      const int mine = (int)blockIdx.x - c_first;  // this CTA's piece of tile t
+      bool from_smem = false;
+      if (npieces > 1) {
+        if (threadIdx.x == 64) {
+          const int prev = atomicAdd(g.tickets + 2 * t, 1);
+          *last_flag = (prev == npieces - 1) ? 1 : 0;
+        }
+        epi_bar();
+        if (*last_flag == 0) {
+          // publish: [32-column chunk][j][row][4], a warp's stores contiguous
+          float* my = g.ws + ((size_t)blockIdx.x * 2 + (first_seg ? 0 : 1)) * (BM * BN);
           for (int c = 0; c < BN; c += 32) {
             float v[32];
             tmem_ld32(t_row + c, v);
             if (c + 32 >= BN) release();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              __stcg(reinterpret_cast<float4*>(my + ((size_t)((c >> 5) * 8 + j) * BM + row) * 4),
+                     make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+          }
+          __threadfence();
+          epi_bar();
+          if (threadIdx.x == 64) atomicAdd(g.tickets + 2 * t + 1, 1);
+          continue;
+        }
+        // the last arrival reduces: the others have arrived; wait until they have published
+        if (threadIdx.x == 64) {
+          if (!wait_count(g.tickets + 2 * t + 1, npieces - 1, g.status, abort_flag)) {
+            *abort_flag = 1;
+          } else {
+            g.tickets[2 * t] = 0;  // every piece is done with the tickets
+            g.tickets[2 * t + 1] = 0;
+            __threadfence();
+            constexpr uint32_t kPart = BM * BN * 4;
+            if (x == x_end && (uint32_t)(npieces - 1) * kPart <= (uint32_t)(C::kStages * C::kStageBytes)) {
+              // the CTA's last segment: its MMAs are done and the ring is free
+              fence_proxy_async_global();
+              mbar_arrive_expect_tx(redb, (npieces - 1) * kPart);
+              int k = 0;
+              for (int p = 0; p < npieces; ++p) {
+                if (p == mine) continue;
+                const int cp = c_first + p;
+                const int slot = (p == 0 && t0 != kbound(g, cp)) ? 1 : 0;
+                const uint8_t* src = reinterpret_cast<const uint8_t*>(g.ws + ((size_t)cp * 2 + slot) * (BM * BN));
+                for (uint32_t o = 0; o < kPart; o += 32768)
+                  bulk_load(smem + k * kPart + o, src + o, min(32768u, kPart - o), redb);
+                ++k;
+              }
+              *last_flag = 2;
+            }
+          }
+        }
+        epi_bar();
+        if (*abort_flag) break;
+        from_smem = *last_flag == 2;
+        if (from_smem) {
+          // at most one bulk reduction per CTA (its last segment): phase 0
+          // (no early exit: the copies must land before the CTA may end)
+          if (!mbar_wait(redb, 0, g.status, kStatusTimeoutPeer, nullptr)) *abort_flag = 1;
+          epi_bar();
+          if (*abort_flag) break;
+        }
+        __threadfence();
+      }
+      // columns [c, c + 32) of this thread's row: the accumulator, or the sum of
+      // all pieces in k order with this CTA's own piece read from TMEM
+      auto get = [&](int c, float* v) {
+        if (npieces == 1) {
+          tmem_ld32(t_row + c, *reinterpret_cast<float(*)[32]>(v));
+          if (c + 32 >= BN) release();
+          return;
+        }
+        float own[32];
+        tmem_ld32(t_row + c, own);
+        if (c + 32 >= BN) release();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        int k = 0;
+        for (int p = 0; p < npieces; ++p) {
+          if (p == mine) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] += own[i];
+            continue;
+          }
+          float4 t4[8];
+          const size_t off = ((size_t)((c >> 5) * 8) * BM + row) * 4;
+          if (from_smem) {
+            const float* src = reinterpret_cast<const float*>(smem) + (size_t)k * (BM * BN) + off;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) t4[j] = *reinterpret_cast<const float4*>(src + (size_t)j * BM * 4);
+          } else {
+            const int cp = c_first + p;
+            const int slot = (p == 0 && t0 != kbound(g, cp)) ? 1 : 0;
+            const float* src = g.ws + ((size_t)cp * 2 + slot) * (BM * BN) + off;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) t4[j] = __ldcg(reinterpret_cast<const float4*>(src + (size_t)j * BM * 4));
+          }
+          ++k;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            v[4 * j] += t4[j].x;
+            v[4 * j + 1] += t4[j].y;
+            v[4 * j + 2] += t4[j].z;
+            v[4 * j + 3] += t4[j].w;
+          }
+        }
+      };
+
+      if constexpr (!SWAP) {
+        const int m = m0w + lane;
+        const bool warp_rows = m0w < g.rows_a;  // the warp has a valid row
+        if constexpr (EPI == kClassStore) {
+          const bool gelu = R.kind == kEpiGelu;
+          const int cols = gelu ? 64 : 32;  // one 128-byte box row
+          for (int c = 0; c < BN; c += cols) {
+            float v[64];
+            get(c, v);
+            if (gelu) get(c + 32, v + 32);
+            if (!warp_rows || nb + c >= g.rows_b) continue;
+            const float4* b4 = reinterpret_cast<const float4*>(sVec + c);
+            uint8_t* box = stg + (nbox & 1) * kBox;
+            if (nbox >= 2) {  // this buffer's previous store has been read out
+              if (lane == 0) bulk_wait_read<1>();
+              __syncwarp();
+            }
+            if (gelu) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const float4 bb = b4[j];
+                v[4 * j] = gelu_tanh(v[4 * j] + bb.x);
+                v[4 * j + 1] = gelu_tanh(v[4 * j + 1] + bb.y);
+                v[4 * j + 2] = gelu_tanh(v[4 * j + 2] + bb.z);
+                v[4 * j + 3] = gelu_tanh(v[4 * j + 3] + bb.w);
+              }
+              box_row_bf16(box, lane, v);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float4 bb = b4[j];
+                v[4 * j] += bb.x;
+                v[4 * j + 1] += bb.y;
+                v[4 * j + 2] += bb.z;
+                v[4 * j + 3] += bb.w;
+              }
+              box_row_f32(box, lane, v);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&map_o, box, nb + c, m0w, 0);
+              bulk_commit();
+            }
+            ++nbox;
+          }
+        } else if constexpr (EPI == kClassRes) {
+          for (int c = 0; c < BN; c += 32) {
+            float v[32];
+            get(c, v);
+            if (!warp_rows || nb + c >= g.rows_b) continue;
+            uint8_t* box = stg + (c >> 5) * kBox;  // the prefetched residual of these columns
+            const float4* b4 = reinterpret_cast<const float4*>(sVec + c);
+            const float4* g4 = reinterpret_cast<const float4*>(sVec + BN + c);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              uint4* p = box_chunk(box, lane, q);
+              const uint4 xo = *p;
+              const float4 bb = b4[q], gg = g4[q];
+              *p = make_uint4(__float_as_uint(__uint_as_float(xo.x) + gg.x * (v[4 * q] + bb.x)),
+                              __float_as_uint(__uint_as_float(xo.y) + gg.y * (v[4 * q + 1] + bb.y)),
+                              __float_as_uint(__uint_as_float(xo.z) + gg.z * (v[4 * q + 2] + bb.z)),
+                              __float_as_uint(__uint_as_float(xo.w) + gg.w * (v[4 * q + 3] + bb.w)));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&map_o, box, nb + c, m0w, 0);
+              bulk_commit();
+            }
+          }
+        } else if constexpr (EPI == kClassQkv) {
+          // all 32 tokens valid and in one sample: one TMA store per head
+          const bool whole = m0w + 32 <= g.rows_a && (m0w % R.seq_len) + 32 <= R.seq_len;
+          for (int c = 0; c < BN; c += 64) {
+            float x[64];
+            get(c, x);
+            get(c + 32, x + 32);
+            const int n = nb + c;
+            if (!warp_rows || n >= g.rows_b) continue;
+            const float4* b4 = reinterpret_cast<const float4*>(sVec + c);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float4 bb = b4[j];
+              x[4 * j] += bb.x;
+              x[4 * j + 1] += bb.y;
+              x[4 * j + 2] += bb.z;
+              x[4 * j + 3] += bb.w;
+            }
+            const int section = n / R.attn_dim, head = (n % R.attn_dim) / 64;
+            qk_norm_rope(R, section, head, min(m, g.rows_a - 1), x, reinterpret_cast<const float*>(stg + lane * 128),
+                         reinterpret_cast<const float*>(stg + kBox + lane * 128), lane & 7, sVec + BN + c);
+            if (whole) {
+              uint8_t* box = stg + (2 + (nbox & 1)) * kBox;
+              if (nbox >= 2) {
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+              }
+              box_row_bf16(box, lane, x);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                const int b = m0w / R.seq_len, l0 = m0w - b * R.seq_len;
+                const int bh = b * R.n_heads + head;
+                if (section == 0)
+                  tma_store_3d(&map_o, box, 0, l0, R.zq0 + bh);
+                else
+                  tma_store_3d(&map_o2, box, 0, R.cache_off + l0, (section == 1 ? R.zk0 : R.zv0) + bh);
+                bulk_commit();
+              }
+              ++nbox;
+            } else if (m < g.rows_a) {
+              store_head(qkv_dst(R, section, head, m), x);
+            }
+          }
+        } else {
+          // per-element epilogue (Euler update, video endpoint)
+          for (int c = 0; c < BN; c += 32) {
+            float v[32];
+            get(c, v);
             const int n0 = nb + c;
-            if (!m_ok || n0 >= g.rows_b) continue;
+            if (m >= g.rows_a || n0 >= g.rows_b) continue;
             const float4* b4 = reinterpret_cast<const float4*>(R.bias + n0);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -466,174 +793,78 @@ __global__ void __launch_bounds__(kThreads, 1)
               v[4 * j + 2] += bb.z;
               v[4 * j + 3] += bb.w;
             }
-            if (R.kind == kEpiStoreF32) {
-              float4* o = reinterpret_cast<float4*>(R.out_f32 + (size_t)m * R.ld + n0);
 #pragma unroll
-              for (int j = 0; j < 8; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            } else if (R.kind == kEpiGelu) {
-              uint4* o = reinterpret_cast<uint4*>(R.out_act + (size_t)m * R.ld + n0);
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                uint4 w;
-                w.x = pack_bf16(gelu_tanh(v[8 * j + 0]), gelu_tanh(v[8 * j + 1]));
-                w.y = pack_bf16(gelu_tanh(v[8 * j + 2]), gelu_tanh(v[8 * j + 3]));
-                w.z = pack_bf16(gelu_tanh(v[8 * j + 4]), gelu_tanh(v[8 * j + 5]));
-                w.w = pack_bf16(gelu_tanh(v[8 * j + 6]), gelu_tanh(v[8 * j + 7]));
-                o[j] = w;
-              }
-            } else if (R.kind == kEpiGateRes) {
-              float4 xo[8];
-              float4* o = reinterpret_cast<float4*>(R.out_f32 + (size_t)m * R.ld + n0);
-              if (C::kPrefetch) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                  xo[j] = *reinterpret_cast<const float4*>(res + lane * BN + 4 * (((c >> 2) + j) ^ (lane & 7)));
-              } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) xo[j] = o[j];
-              }
-              const float4* g4 = reinterpret_cast<const float4*>(R.gate + n0);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const float4 gg = __ldg(g4 + j);
-                o[j] = make_float4(xo[j].x + gg.x * v[4 * j], xo[j].y + gg.y * v[4 * j + 1],
-                                   xo[j].z + gg.z * v[4 * j + 2], xo[j].w + gg.w * v[4 * j + 3]);
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) epi_elem(e, m, n0 + j, v[j], 0.f);
-            }
+            for (int j = 0; j < 32; ++j) epi_elem(e, m, n0 + j, v[j], 0.f);
           }
         }
       } else {
         // swapped: TMEM lane = feature n, column = token
         const int n = ta * BM + row;
         const int mb = tb * BN;
-        const int tile_lin = ta + g.tiles_a * tb;
         const bool n_ok = n < g.rows_a;
         const float bias = n_ok ? __ldg(R.bias + n) : 0.f;
         const float gate = (n_ok && R.gate) ? __ldg(R.gate + n) : 0.f;
-        bool last = true;
-        if (g.splits > 1) {
-          float* my = g.ws + ((size_t)(tile_lin * g.splits + sp) * BM + row) * BN;
-          for (int c = 0; c < BN; c += 32) {
-            float v[32];
-            tmem_ld32(t_row + c, v);
-            if (c + 32 >= BN) release();
+        for (int c = 0; c < BN; c += 32) {
+          float v[32];
+          get(c, v);
+          if (R.kind == kEpiQkv) {
+            // stage [32 tokens][128 features + 1] and emit (token, head) items
+            float* stage = reinterpret_cast<float*>(sStg);
+            epi_bar();  // the previous chunk's readers are done with the stage
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              __stcg(reinterpret_cast<float4*>(my + c + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
-          }
-          __threadfence();
-          epi_bar();
-          if (threadIdx.x == 64) {
-            const int prev = atomicAdd(g.tickets + tile_lin, 1);
-            *last_flag = (prev == g.splits - 1) ? 1 : 0;
-          }
-          epi_bar();
-          last = *last_flag != 0;
-          __threadfence();
-        }
-        if (last) {
-          for (int c = 0; c < BN; c += 32) {
-            float v[32];
-            if (g.splits > 1) {
+            for (int j = 0; j < 32; ++j) stage[j * (BM + 1) + row] = v[j] + bias;
+            epi_bar();
+            const int tt = threadIdx.x - 64;
+            if (tt < 64) {
+              const int j = tt & 31, hh = tt >> 5;
+              const int m = mb + c + j;
+              const int n0 = ta * BM + hh * 64;
+              if (m < g.rows_b && n0 < g.rows_a) {
+                float xv[64];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = 0.f;
-              const float* p = g.ws + ((size_t)(tile_lin * g.splits) * BM + row) * BN + c;
-              const size_t sstride = (size_t)BM * BN;
-              int s = 0;
-              for (; s + 2 <= g.splits; s += 2) {  // two splits in flight, summed in split order
-                float4 t0[8], t1[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  t0[j] = __ldcg(reinterpret_cast<const float4*>(p + s * sstride) + j);
-                  t1[j] = __ldcg(reinterpret_cast<const float4*>(p + (s + 1) * sstride) + j);
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  v[4 * j] += t0[j].x;
-                  v[4 * j + 1] += t0[j].y;
-                  v[4 * j + 2] += t0[j].z;
-                  v[4 * j + 3] += t0[j].w;
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  v[4 * j] += t1[j].x;
-                  v[4 * j + 1] += t1[j].y;
-                  v[4 * j + 2] += t1[j].z;
-                  v[4 * j + 3] += t1[j].w;
-                }
-              }
-              for (; s < g.splits; ++s) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  const float4 t4 = __ldcg(reinterpret_cast<const float4*>(p + s * sstride) + j);
-                  v[4 * j] += t4.x;
-                  v[4 * j + 1] += t4.y;
-                  v[4 * j + 2] += t4.z;
-                  v[4 * j + 3] += t4.w;
-                }
-              }
-            } else {
-              tmem_ld32(t_row + c, v);
-              if (c + 32 >= BN) release();
-            }
-            if (R.kind == kEpiQkv) {
-              // stage [32 tokens][128 features + 1] and emit (token, head) items
-              float* stage = sEpi;
-              epi_bar();  // previous chunk's readers are done with the stage
-#pragma unroll
-              for (int j = 0; j < 32; ++j) stage[j * (BM + 1) + row] = v[j] + bias;
-              epi_bar();
-              const int t = threadIdx.x - 64;
-              if (t < 64) {
-                const int j = t & 31, hh = t >> 5;
-                const int m = mb + c + j;
-                const int n0 = ta * BM + hh * 64;
-                if (m < g.rows_b && n0 < g.rows_a) {
-                  float x[64];
-#pragma unroll
-                  for (int k = 0; k < 64; ++k) x[k] = stage[j * (BM + 1) + hh * 64 + k];
-                  qkv_emit(R, n0 / R.attn_dim, (n0 % R.attn_dim) / 64, m, x);
-                }
-              }
-            } else if (n_ok && R.kind == kEpiGateRes) {
-              float xo[32];
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int m = mb + c + j;
-                xo[j] = m < g.rows_b ? R.out_f32[(size_t)m * R.ld + n] : 0.f;
-              }
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int m = mb + c + j;
-                if (m < g.rows_b) R.out_f32[(size_t)m * R.ld + n] = xo[j] + gate * (v[j] + bias);
-              }
-            } else if (n_ok && R.kind == kEpiStoreF32) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int m = mb + c + j;
-                if (m < g.rows_b) R.out_f32[(size_t)m * R.ld + n] = v[j] + bias;
-              }
-            } else if (n_ok && R.kind == kEpiGelu) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int m = mb + c + j;
-                if (m < g.rows_b) R.out_act[(size_t)m * R.ld + n] = __float2bfloat16_rn(gelu_tanh(v[j] + bias));
-              }
-            } else if (n_ok) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int m = mb + c + j;
-                if (m < g.rows_b) epi_elem(e, m, n, v[j] + bias, gate);
+                for (int k = 0; k < 64; ++k) xv[k] = stage[j * (BM + 1) + hh * 64 + k];
+                const int section = n0 / R.attn_dim, head = (n0 % R.attn_dim) / 64;
+                qk_norm_rope(R, section, head, m, xv, nullptr, nullptr, 0);
+                store_head(qkv_dst(R, section, head, m), xv);
               }
             }
+          } else if (n_ok && R.kind == kEpiGateRes) {
+            float xo[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int m = mb + c + j;
+              xo[j] = m < g.rows_b ? R.out_f32[(size_t)m * R.ld + n] : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int m = mb + c + j;
+              if (m < g.rows_b) R.out_f32[(size_t)m * R.ld + n] = xo[j] + gate * (v[j] + bias);
+            }
+          } else if (n_ok && R.kind == kEpiStoreF32) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int m = mb + c + j;
+              if (m < g.rows_b) R.out_f32[(size_t)m * R.ld + n] = v[j] + bias;
+            }
+          } else if (n_ok && R.kind == kEpiGelu) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int m = mb + c + j;
+              if (m < g.rows_b) R.out_act[(size_t)m * R.ld + n] = __float2bfloat16_rn(gelu_tanh(v[j] + bias));
+            }
+          } else if (n_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int m = mb + c + j;
+              if (m < g.rows_b) epi_elem(e, m, n, v[j] + bias, gate);
+            }
           }
-          if (g.splits > 1 && threadIdx.x == 64) g.tickets[tile_lin] = 0;
         }
       }
     }
+    // the warp's bulk stores are complete before the CTA's shared memory goes away
+    if (!SWAP && EPI != kClassScalar && lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   // ------------------------------------------------------------- teardown
@@ -642,9 +873,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     // wait for the last commits of this CTA's MMAs before freeing TMEM
     if (lane == 0) {
-      int nloc = 0;
-      for (int u = blockIdx.x; u < g.units; u += gridDim.x) ++nloc;
-      for (int l = max(0, nloc - 2); l < nloc; ++l)
+      int nseg = 0;
+      for (long long x = x_begin; x < x_end; ++nseg) {
+        const Seg sg = seg_at(g, x, x_end);
+        x += sg.kb1 - sg.kb0;
+      }
+      for (int l = max(0, nseg - 2); l < nseg; ++l)
         mbar_wait(&accf[l & 1], (l >> 1) & 1, g.status, kStatusTimeoutDrain, nullptr);
     }
     __syncwarp();
@@ -653,75 +887,125 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BN, bool SWAP>
-cudaError_t prepare_bn() {
-  return cudaFuncSetAttribute(tc_gemm_kernel<BN, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TileCfg<BN, SWAP>::kSmem);
+template <int BN, bool SWAP, int EPI>
+cudaError_t prepare_one() {
+  return cudaFuncSetAttribute(tc_gemm_kernel<BN, SWAP, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TileCfg<BN, SWAP, EPI>::kSmem);
 }
 
 int g_num_sms = 0;
 
-template <int BN, bool SWAP>
-cudaError_t launch_bn(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
-  using C = TileCfg<BN, SWAP>;
+// Persistent grid size: swapped -- tiles x splits; normal -- max_ctas or one
+// per SM; never more CTAs than k-blocks.
+int ctas_of(const TcGemm& t) {
+  const int kb = (t.K + BK - 1) / BK;
+  const long long tiles = (long long)((t.rows_a + BM - 1) / BM) * ((t.rows_b + t.bn - 1) / t.bn);
+  long long want;
+  if (t.swap) {
+    int splits = t.splits < 1 ? 1 : t.splits;
+    if (splits > kb) splits = kb;
+    want = tiles * splits;
+  } else {
+    want = t.max_ctas > 0 ? t.max_ctas : g_num_sms;
+  }
+  const long long W = tiles * kb;
+  if (want > W) want = W;
+  if (want < 1) want = 1;
+  return (int)want;
+}
+
+template <int BN, bool SWAP, int EPI>
+cudaError_t launch_one(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
+  using C = TileCfg<BN, SWAP, EPI>;
   GemmK g;
   g.rows_a = t.rows_a;
   g.rows_b = t.rows_b;
   g.K = t.K;
   g.z_a = t.z_a;
   g.z_b = t.z_b;
-  const int kb_total = (t.K + BK - 1) / BK;
-  int splits = t.swap ? (t.splits < 1 ? 1 : t.splits) : 1;
-  if (splits > kb_total) splits = kb_total;
-  g.kb_per_split = (kb_total + splits - 1) / splits;
-  splits = (kb_total + g.kb_per_split - 1) / g.kb_per_split;  // no empty split
-  g.splits = splits;
   g.tiles_a = (t.rows_a + BM - 1) / BM;
-  g.tiles_b = (t.rows_b + BN - 1) / BN;
-  g.units = g.tiles_a * g.tiles_b * splits;
+  g.KB = (t.K + BK - 1) / BK;
+  g.W = (long long)g.tiles_a * ((t.rows_b + BN - 1) / BN) * g.KB;
+  g.G = ctas_of(t);
   g.ws = t.ws;
   g.tickets = t.tickets;
   g.status = t.status;
-  int ctas = t.max_ctas > 0 ? t.max_ctas : g_num_sms;
-  if (ctas > g.units) ctas = g.units;
-  if (ctas < 1) ctas = 1;
-  return launch_k(tc_gemm_kernel<BN, SWAP>, dim3(ctas), dim3(kThreads), C::kSmem, s, *t.map_a, *t.map_b, g, e);
+  // unused output maps are passed as copies of the A map
+  const CUtensorMap& mo = e.map_o ? *e.map_o : *t.map_a;
+  const CUtensorMap& mo2 = e.map_o2 ? *e.map_o2 : *t.map_a;
+  return launch_k(tc_gemm_kernel<BN, SWAP, EPI>, dim3(g.G), dim3(kThreads), C::kSmem, s, *t.map_a, *t.map_b, mo, mo2,
+                  g, e);
+}
+
+template <int BN>
+cudaError_t launch_normal(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
+  switch (e.kind) {
+    case kEpiStoreF32:
+    case kEpiGelu:
+      if (!e.map_o) return cudaErrorInvalidValue;
+      return launch_one<BN, false, kClassStore>(t, e, s);
+    case kEpiGateRes:
+      if constexpr (BN <= 128) {
+        if (!e.map_o) return cudaErrorInvalidValue;
+        return launch_one<BN, false, kClassRes>(t, e, s);
+      } else {
+        return cudaErrorInvalidValue;
+      }
+    case kEpiQkv:
+      if (!e.map_o || !e.map_o2) return cudaErrorInvalidValue;
+      return launch_one<BN, false, kClassQkv>(t, e, s);
+    default:
+      return launch_one<BN, false, kClassScalar>(t, e, s);
+  }
 }
 
 }  // namespace
+
+size_t tc_gemm_ws_floats(const TcGemm& t) { return (size_t)ctas_of(t) * 2 * BM * t.bn; }
 
 cudaError_t prepare_tc_gemm() {
   cudaError_t e;
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  if ((e = prepare_bn<32, true>()) != cudaSuccess) return e;
-  if ((e = prepare_bn<64, true>()) != cudaSuccess) return e;
-  if ((e = prepare_bn<128, true>()) != cudaSuccess) return e;
-  if ((e = prepare_bn<256, true>()) != cudaSuccess) return e;
-  if ((e = prepare_bn<64, false>()) != cudaSuccess) return e;
-  if ((e = prepare_bn<96, false>()) != cudaSuccess) return e;
-  if ((e = prepare_bn<128, false>()) != cudaSuccess) return e;
-  return prepare_bn<256, false>();
+#define WAM_PREP(BN, SW, EP) \
+  if ((e = prepare_one<BN, SW, EP>()) != cudaSuccess) return e;
+  WAM_PREP(32, true, kClassScalar)
+  WAM_PREP(64, true, kClassScalar)
+  WAM_PREP(128, true, kClassScalar)
+  WAM_PREP(256, true, kClassScalar)
+  WAM_PREP(64, false, kClassScalar)
+  WAM_PREP(64, false, kClassStore)
+  WAM_PREP(64, false, kClassRes)
+  WAM_PREP(64, false, kClassQkv)
+  WAM_PREP(128, false, kClassScalar)
+  WAM_PREP(128, false, kClassStore)
+  WAM_PREP(128, false, kClassRes)
+  WAM_PREP(128, false, kClassQkv)
+  WAM_PREP(256, false, kClassScalar)
+  WAM_PREP(256, false, kClassStore)
+  WAM_PREP(256, false, kClassQkv)
+#undef WAM_PREP
+  return cudaSuccess;
 }
 
 cudaError_t launch_tc_gemm(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
   if (g_num_sms == 0) return cudaErrorNotReady;
-  // the normal orientation's epilogue writes whole 32-feature groups
-  if (!t.swap && t.rows_b % 32 != 0) return cudaErrorInvalidValue;
+  if (!t.ws || !t.tickets) return cudaErrorInvalidValue;
   if (t.swap) {
     switch (t.bn) {
-      case 32: return launch_bn<32, true>(t, e, s);
-      case 64: return launch_bn<64, true>(t, e, s);
-      case 128: return launch_bn<128, true>(t, e, s);
-      case 256: return launch_bn<256, true>(t, e, s);
+      case 32: return launch_one<32, true, kClassScalar>(t, e, s);
+      case 64: return launch_one<64, true, kClassScalar>(t, e, s);
+      case 128: return launch_one<128, true, kClassScalar>(t, e, s);
+      case 256: return launch_one<256, true, kClassScalar>(t, e, s);
     }
   } else {
+    // the normal orientation's epilogue writes whole 32-feature groups
+    if (t.rows_b % 32 != 0) return cudaErrorInvalidValue;
     switch (t.bn) {
-      case 64: return launch_bn<64, false>(t, e, s);
-      case 96: return launch_bn<96, false>(t, e, s);
-      case 128: return launch_bn<128, false>(t, e, s);
-      case 256: return launch_bn<256, false>(t, e, s);
+      case 64: return launch_normal<64>(t, e, s);
+      case 128: return launch_normal<128>(t, e, s);
+      case 256: return launch_normal<256>(t, e, s);
     }
   }
   return cudaErrorInvalidValue;

@@ -86,6 +86,13 @@ struct EpiArgs {
   void* a_next = nullptr;           // next in-proj input (act dtype), ld = a_next_ld
   int a_next_ld = 0;
   const float* x_sigma = nullptr;   // joint variant: noised video patches
+  // Output tensor maps of the normal orientation's TMA-store epilogues
+  // (box 32 rows): map_o = the output matrix (fp32 [M, N], box 32 cols; bf16
+  // [M, N], box 64 cols) or Q ([B*H][L][64]); map_o2 = the K/V cache
+  // ([2*N*B*H][L_v + L_a][64]).  zq0 / zk0 / zv0: matrix index of (b=0, h=0).
+  const CUtensorMap* map_o = nullptr;
+  const CUtensorMap* map_o2 = nullptr;
+  int zq0 = 0, zk0 = 0, zv0 = 0;
 };
 
 // C[m, n] = sum_k X[m, k] W[n, k] (+ epilogue), bf16 operands via TMA into
@@ -97,13 +104,16 @@ struct TcGemm {
   int rows_a, rows_b, K;
   int z_a, z_b;              // matrix index (block) of each operand
   int bn;                    // N tile (32, 64, 128, 256)
-  int splits;                // split-K factor (swap only)
+  int splits;                // swapped: CTAs = tiles * splits (each tile's K split evenly)
   bool swap;
-  int max_ctas;              // persistent grid size (0: one CTA per SM)
-  float* ws;                 // split-K partials, splits * tiles * 128 * bn floats
-  int* tickets;              // one per output tile, zero on entry, left zero
+  int max_ctas;              // normal: persistent grid size (0: one CTA per SM)
+  float* ws;                 // partial tiles: 2 * CTAs * 128 * bn floats (tc_gemm_ws_floats)
+  int* tickets;              // two per output tile, zero on entry, left zero
   unsigned* status;
 };
+
+// Workspace floats the launch needs for K-split partial tiles.
+size_t tc_gemm_ws_floats(const TcGemm& g);
 
 cudaError_t launch_tc_gemm(const TcGemm& g, const EpiArgs& e, cudaStream_t s);
 // Sets the kernels' shared-memory attributes; call once per device before any
@@ -192,5 +202,9 @@ cudaError_t launch_to_f32(const void* src, bool src_bf16, float* dst, size_t n, 
 // TMA tensor-map creation (driver entry point resolved at run time).
 bool make_tmap_3d(CUtensorMap* map, const void* base, int K, int rows, int nmat, size_t mat_stride_bytes,
                   int box_rows);
+// General 3-D map with the 128-byte swizzle: elem_bytes 2 (bf16) or 4 (fp32),
+// dims (inner, rows, nmat), box (box_inner, box_rows, 1).
+bool make_tmap_sw128(CUtensorMap* map, const void* base, int elem_bytes, int inner, int rows, int nmat,
+                     size_t mat_stride_bytes, int box_inner, int box_rows);
 
 }  // namespace wam

@@ -376,8 +376,26 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 }  // namespace
 
-bool make_tmap_3d(CUtensorMap* map, const void* base, int K, int rows, int nmat, size_t mat_stride_bytes,
-                  int box_rows) {
+static bool encoder_ready();
+
+bool make_tmap_sw128(CUtensorMap* map, const void* base, int elem_bytes, int inner, int rows, int nmat,
+                     size_t mat_stride_bytes, int box_inner, int box_rows) {
+  if (!encoder_ready()) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((size_t)inner * elem_bytes) % 16 || mat_stride_bytes % 16 ||
+      box_inner * elem_bytes != 128)
+    return false;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)nmat};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * elem_bytes,
+                           (cuuint64_t)(nmat > 1 ? mat_stride_bytes : (size_t)inner * elem_bytes * rows)};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, elem_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static bool encoder_ready() {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -385,7 +403,12 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, int K, int rows, int nmat,
         q == cudaDriverEntryPointSuccess)
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   });
-  if (!g_encode) return false;
+  return g_encode != nullptr;
+}
+
+bool make_tmap_3d(CUtensorMap* map, const void* base, int K, int rows, int nmat, size_t mat_stride_bytes,
+                  int box_rows) {
+  if (!encoder_ready()) return false;
   if ((reinterpret_cast<uintptr_t>(base) & 15) || ((size_t)K * 2) % 16 || mat_stride_bytes % 16) return false;
   cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)rows, (cuuint64_t)nmat};
   cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)(nmat > 1 ? mat_stride_bytes : (size_t)K * 2 * rows)};

@@ -77,8 +77,10 @@ struct wam_ctx {
   void* kv = nullptr;                                 // [N][2][B][H][Ltot][Dh]
   float *mod_v = nullptr, *mod_a = nullptr, *temb_v = nullptr, *temb_a = nullptr;
   float *rope_cos = nullptr, *rope_sin = nullptr;
-  float* ws_gemm = nullptr;
+  float* ws_gemm = nullptr;  // action-stream GEMM partial tiles / tickets
   int* tk_gemm = nullptr;
+  float* ws_gemm_v = nullptr;  // video-stream GEMM partial tiles / tickets (the streams overlap)
+  int* tk_gemm_v = nullptr;
   float* ws_attn = nullptr;
   int* tk_attn = nullptr;
   unsigned* status = nullptr;
@@ -94,11 +96,17 @@ struct wam_ctx {
   GemmPlan p_v_qkv, p_v_o, p_v_f1, p_v_f2, p_v_in, p_v_out;
   GemmPlan p_a_in, p_a_qkv, p_a_o, p_a_f1, p_a_f2, p_a_out;
   int attn_splits = 1;
+  // Persistent grid of the video GEMMs while the action stream runs beside
+  // them (CEWP); otherwise they take every SM.
+  int video_ctas_overlap = 0;
+  bool video_overlap = false;
 
   // TMA maps
   CUtensorMap m_hv, m_ov, m_fv, m_xvin, m_w_qkv_v, m_w_o_v, m_w_f1_v, m_w_f2_v, m_w_vin, m_w_vout;
   CUtensorMap m_w_in, m_w_qkv_a, m_w_o_a, m_w_f1_a, m_w_f2_a, m_w_out, m_ain, m_ha, m_oa, m_fa;
   CUtensorMap m_qv, m_cache;  // video-attention operands
+  // video GEMM outputs (TMA stores, 32-row boxes): x_v fp32, f_v bf16, Q, the K/V cache
+  CUtensorMap m_xv_out, m_fv_out, m_qv_out, m_cache_out;
 
   // events and streams
   std::vector<cudaEvent_t> ev_kv, ev_kv_cap, ev_used;
@@ -282,19 +290,9 @@ GemmPlan plan_swap(int rows_w, int tokens, int K, int bn) {
   return p;
 }
 
-size_t ws_floats(const GemmPlan& p, int rows_w, int tokens) {
-  if (p.splits <= 1) return 0;
-  const int tiles = ((rows_w + 127) / 128) * ((tokens + p.bn - 1) / p.bn);
-  return (size_t)tiles * p.splits * 128 * p.bn;
-}
-
-int tiles_of(const GemmPlan& p, int rows_w, int tokens) {
-  return ((rows_w + 127) / 128) * ((tokens + p.bn - 1) / p.bn);
-}
-
 // --------------------------------------------------------- GEMM wrappers --
 wam_status run_tc(wam_ctx* c, const CUtensorMap& A, const CUtensorMap& Bm, int rows_a, int rows_b, int K, int z_a,
-                  int z_b, const GemmPlan& p, bool swap, const EpiArgs& e, cudaStream_t s) {
+                  int z_b, const GemmPlan& p, bool swap, const EpiArgs& e, cudaStream_t s, bool video) {
   TcGemm g;
   g.map_a = &A;
   g.map_b = &Bm;
@@ -306,9 +304,9 @@ wam_status run_tc(wam_ctx* c, const CUtensorMap& A, const CUtensorMap& Bm, int r
   g.bn = p.bn;
   g.splits = p.splits;
   g.swap = swap;
-  g.max_ctas = p.max_ctas;
-  g.ws = c->ws_gemm;
-  g.tickets = c->tk_gemm;
+  g.max_ctas = (video && c->video_overlap && p.max_ctas == 0) ? c->video_ctas_overlap : p.max_ctas;
+  g.ws = video ? c->ws_gemm_v : c->ws_gemm;
+  g.tickets = video ? c->tk_gemm_v : c->tk_gemm;
   g.status = c->status;
   c->launches++;
   CK(launch_tc_gemm(g, e, s));
@@ -361,9 +359,22 @@ wam_status linear(wam_ctx* c, bool video, const Lin& L, int M, const EpiArgs& e_
   const Dims& d = c->d;
   ProfScope ps(c, s);
   if (d.bf16) {
-    if (video)  // tokens on TMEM lanes
-      return run_tc(c, *L.map_x, *L.map_w, M, L.n_out, L.K, 0, L.z, *L.plan, false, e_in, s);
-    return run_tc(c, *L.map_w, *L.map_x, L.n_out, M, L.K, L.z, 0, *L.plan, true, e_in, s);
+    if (video) {  // tokens on TMEM lanes; outputs leave through TMA stores
+      EpiArgs e = e_in;
+      if (e.kind == kEpiQkv) {
+        e.map_o = &c->m_qv_out;
+        e.map_o2 = &c->m_cache_out;
+        e.zq0 = 0;
+        e.zk0 = 2 * L.z * d.B * d.H;
+        e.zv0 = (2 * L.z + 1) * d.B * d.H;
+      } else if (e.kind == kEpiGelu) {
+        e.map_o = &c->m_fv_out;
+      } else if (e.kind == kEpiStoreF32 || e.kind == kEpiGateRes) {
+        e.map_o = &c->m_xv_out;
+      }
+      return run_tc(c, *L.map_x, *L.map_w, M, L.n_out, L.K, 0, L.z, *L.plan, false, e, s, true);
+    }
+    return run_tc(c, *L.map_w, *L.map_x, L.n_out, M, L.K, L.z, 0, *L.plan, true, e_in, s, false);
   }
   if (e_in.kind == kEpiQkv) {
     EpiArgs st = epi_base(kEpiStoreF32, e_in.bias, qkv_tmp, nullptr, 3 * d.A);
@@ -589,7 +600,10 @@ wam_status enqueue_chunk(wam_ctx* c, int steps, int mode, bool joint, cudaStream
   if (cewp) {
     // Enqueue the two experts interleaved block by block is not needed: the
     // streams run concurrently; the per-block events order Attn^a_i after P^v_i.
-    RET(enqueue_video(c, sv, c->vio_chunk, joint, ev_kv, false));
+    c->video_overlap = true;
+    const wam_status st = enqueue_video(c, sv, c->vio_chunk, joint, ev_kv, false);
+    c->video_overlap = false;
+    RET(st);
     for (int j = 0; j < steps; ++j) RET(enqueue_action_step(c, sa, c->aio_chunk, j, j == 0 ? ev_kv : nullptr, false));
   } else {
     RET(enqueue_video(c, sv, c->vio_chunk, joint, nullptr, false));
@@ -778,7 +792,7 @@ void wam_destroy(wam_ctx* c) {
   if (c->cap_a) cudaStreamDestroy(c->cap_a);
   void* bufs[] = {c->wmat, c->wvec, c->x_v, c->x_a, c->a_state, c->x_sigma, c->h_v, c->q_v, c->o_v, c->f_v,
                   c->x_vin, c->h_a, c->q_a, c->o_a, c->f_a, c->a_in, c->qkv_tmp_v, c->qkv_tmp_a, c->kv,
-                  c->mod_v, c->mod_a, c->temb_v, c->temb_a, c->rope_cos, c->rope_sin, c->ws_gemm, c->tk_gemm,
+                  c->mod_v, c->mod_a, c->temb_v, c->temb_a, c->rope_cos, c->rope_sin, c->ws_gemm, c->tk_gemm, c->ws_gemm_v, c->tk_gemm_v,
                   c->ws_attn, c->tk_attn, c->status, c->vio_chunk, c->vio_eager, c->aio_chunk, c->aio_eager,
                   c->h_video, c->h_cond, c->h_noise, c->h_out, c->j_vout, c->j_aout};
   for (void* p : bufs)
@@ -855,19 +869,26 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   CK(launch_rope_table(c->rope_cos, c->rope_sin, d.Ltot, d.Dh, 0));
 
   // GEMM plans (bf16 path) and workspaces
-  size_t ws = 0;
-  int tiles = 1;
+  size_t ws = 0, ws_v = 0;
+  int tiles = 1, tiles_v = 1;
   if (d.bf16) {
-    // Tiles and persistent grid sizes for the video GEMMs (config 2: 9 row
-    // tiles of 128): out-proj / FFN-down 1536/128 -> 108 units, one round on
-    // 108 SMs; QKV 4608/128 -> 324 units, three rounds -- on 108 CTAs, the same
-    // makespan as on all 148; FFN-up 6144/128 -> 432 units on all SMs.  The
-    // SMs the video GEMMs leave free run the action stream under CEWP.
-    const int v_rows = (d.Mv + 127) / 128;
-    const int ctas_third = std::min(std::max(1, (v_rows * (3 * d.A / 128) + 2) / 3), 148);
-    c->p_v_qkv = {128, 1, ctas_third};
+    // Video GEMMs (tokens on TMEM lanes): stream-K over a persistent grid, so
+    // every CTA gets the same share of k-blocks whatever the tile count.  The
+    // wide projections (QKV, FFN-up) take 256-feature tiles (half the operand
+    // traffic per flop of 128); out-proj / FFN-down keep 128 (their residual
+    // staging holds 128 columns).  Under CEWP the video GEMMs leave about a
+    // quarter of the SMs to the action stream (108 of 148 measured best on
+    // the config-2 chunk); WAM_VIDEO_GEMM_CTAS overrides the count.
+    int nsm = 148;
+    CK(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, c->device));
+    c->video_ctas_overlap = std::max(1, nsm * 73 / 100);
+    if (const char* v = getenv("WAM_VIDEO_GEMM_CTAS")) {
+      const int n = atoi(v);
+      if (n > 0) c->video_ctas_overlap = std::min(n, nsm);
+    }
+    c->p_v_qkv = {256, 1, 0};
     c->p_v_o = {128, 1, 0};
-    c->p_v_f1 = {128, 1, 0};
+    c->p_v_f1 = {256, 1, 0};
     c->p_v_f2 = {128, 1, 0};
     c->p_v_in = {128, 1, 0};
     c->p_v_out = {64, 1, 0};
@@ -878,19 +899,37 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     c->p_a_f1 = plan_swap(d.Fa, d.Ma, d.da, bn_a);
     c->p_a_f2 = plan_swap(d.da, d.Ma, d.Fa, bn_a);
     c->p_a_out = plan_swap(d.Pa, d.Ma, d.da, bn_a);
-    struct {
-      GemmPlan* p;
-      int rows;
-    } aps[] = {{&c->p_a_in, d.da}, {&c->p_a_qkv, 3 * d.A}, {&c->p_a_o, d.da},
-               {&c->p_a_f1, d.Fa}, {&c->p_a_f2, d.da},     {&c->p_a_out, d.Pa}};
-    for (auto& a : aps) {
-      ws = std::max(ws, ws_floats(*a.p, a.rows, d.Ma));
-      tiles = std::max(tiles, tiles_of(*a.p, a.rows, d.Ma));
-    }
+    // workspace and tickets of one launch: rows_a x rows_b output, reduction K
+    auto need = [](const GemmPlan& p, int rows_a, int rows_b, int K, bool swap, size_t* w, int* t) {
+      TcGemm g{};
+      g.rows_a = rows_a;
+      g.rows_b = rows_b;
+      g.K = K;
+      g.bn = p.bn;
+      g.splits = p.splits;
+      g.swap = swap;
+      g.max_ctas = p.max_ctas;
+      *w = std::max(*w, tc_gemm_ws_floats(g));
+      *t = std::max(*t, ((rows_a + 127) / 128) * ((rows_b + p.bn - 1) / p.bn));
+    };
+    need(c->p_a_in, d.da, d.Ma, d.Kin, true, &ws, &tiles);
+    need(c->p_a_qkv, 3 * d.A, d.Ma, d.da, true, &ws, &tiles);
+    need(c->p_a_o, d.da, d.Ma, d.A, true, &ws, &tiles);
+    need(c->p_a_f1, d.Fa, d.Ma, d.da, true, &ws, &tiles);
+    need(c->p_a_f2, d.da, d.Ma, d.Fa, true, &ws, &tiles);
+    need(c->p_a_out, d.Pa, d.Ma, d.da, true, &ws, &tiles);
+    need(c->p_v_qkv, d.Mv, 3 * d.A, d.dv, false, &ws_v, &tiles_v);
+    need(c->p_v_o, d.Mv, d.dv, d.A, false, &ws_v, &tiles_v);
+    need(c->p_v_f1, d.Mv, d.Fv, d.dv, false, &ws_v, &tiles_v);
+    need(c->p_v_f2, d.Mv, d.dv, d.Fv, false, &ws_v, &tiles_v);
+    if (d.Pv > 0) need(c->p_v_in, d.Mv, d.dv, d.Pv, false, &ws_v, &tiles_v);
+    if (cfg->video_has_output) need(c->p_v_out, d.Mv, d.Pv, d.dv, false, &ws_v, &tiles_v);
     c->attn_splits = std::max(1, (d.Lv + d.La + 127) / 128);
   }
   RET(dalloc(c, &c->ws_gemm, ws * 4));
-  RET(dalloc(c, &c->tk_gemm, (size_t)tiles * 4));
+  RET(dalloc(c, &c->tk_gemm, (size_t)tiles * 2 * 4));
+  RET(dalloc(c, &c->ws_gemm_v, ws_v * 4));
+  RET(dalloc(c, &c->tk_gemm_v, (size_t)tiles_v * 2 * 4));
   RET(dalloc(c, &c->ws_attn, attention_ws_floats(d.B, d.H, d.Dh, d.La, c->attn_splits) * 4));
   RET(dalloc(c, &c->tk_attn, (size_t)d.B * d.H * 4));
 
@@ -928,6 +967,11 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     amap(&c->m_fa, c->f_a, d.Ma, d.Fa, bna);
     ok = ok && make_tmap_3d(&c->m_qv, c->q_v, d.Dh, d.Lv, d.B * d.H, (size_t)d.Lv * d.Dh * 2, 128);
     ok = ok && make_tmap_3d(&c->m_cache, c->kv, d.Dh, d.Ltot, 2 * d.N * d.B * d.H, (size_t)d.Ltot * d.Dh * 2, 128);
+    ok = ok && make_tmap_sw128(&c->m_xv_out, c->x_v, 4, d.dv, d.Mv, 1, 0, 32, 32);
+    ok = ok && make_tmap_sw128(&c->m_fv_out, c->f_v, 2, d.Fv, d.Mv, 1, 0, 64, 32);
+    ok = ok && make_tmap_sw128(&c->m_qv_out, c->q_v, 2, d.Dh, d.Lv, d.B * d.H, (size_t)d.Lv * d.Dh * 2, 64, 32);
+    ok = ok && make_tmap_sw128(&c->m_cache_out, c->kv, 2, d.Dh, d.Ltot, 2 * d.N * d.B * d.H,
+                               (size_t)d.Ltot * d.Dh * 2, 64, 32);
     if (!ok) return fail(c, WAM_ERR_CUDA, "tensor map creation failed");
   }
 
@@ -1234,44 +1278,51 @@ wam_status wam_op_linear(int dtype, const void* x, const void* w, const float* b
   if (dtype != WAM_BF16 || K % 64) return WAM_ERR_INVALID_ARG;
   const int bn = swap ? (M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256) : 128;
   if (swap && M > 256) return WAM_ERR_INVALID_ARG;
-  static thread_local float* ws = nullptr;
-  static thread_local int* tk = nullptr;
-  static thread_local size_t ws_cap = 0, tk_cap = 0;
-  const int rows_w = N, tiles = swap ? ((N + 127) / 128) : 1;
-  const int kb = K / 64;
-  int sp = swap ? std::max(1, std::min(splits, kb)) : 1;
-  const size_t need = swap && sp > 1 ? (size_t)tiles * sp * 128 * bn : 0;
-  if (need > ws_cap) {
-    if (ws) cudaFree(ws);
-    if (cudaMalloc(&ws, need * 4) != cudaSuccess) return WAM_ERR_OOM;
-    ws_cap = need;
-  }
-  if ((size_t)tiles > tk_cap) {
-    if (tk) cudaFree(tk);
-    if (cudaMalloc(&tk, tiles * 4) != cudaSuccess) return WAM_ERR_OOM;
-    if (cudaMemset(tk, 0, tiles * 4) != cudaSuccess) return WAM_ERR_CUDA;
-    tk_cap = tiles;
-  }
+  if (!swap && N % 32) return WAM_ERR_INVALID_ARG;
   static thread_local unsigned* status = nullptr;
   if (!status) {
     if (prepare_tc_gemm() != cudaSuccess) return WAM_ERR_CUDA;
     if (cudaMalloc(&status, 4) != cudaSuccess) return WAM_ERR_OOM;
     cudaMemset(status, 0, 4);
   }
-  CUtensorMap mx, mw;
-  if (!make_tmap_3d(&mx, x, K, M, 1, 0, swap ? bn : 128) || !make_tmap_3d(&mw, w, K, rows_w, 1, 0, swap ? 128 : bn))
-    return WAM_ERR_INVALID_ARG;
-  TcGemm g;
-  g.map_a = swap ? &mw : &mx;
-  g.map_b = swap ? &mx : &mw;
+  TcGemm g{};
   g.rows_a = swap ? N : M;
   g.rows_b = swap ? M : N;
   g.K = K;
   g.z_a = g.z_b = 0;
   g.bn = bn;
-  g.splits = sp;
+  g.splits = swap ? std::max(1, splits) : 1;
   g.swap = swap != 0;
-  g.max_ctas = 0;
+  g.max_ctas = swap ? 0 : std::max(0, splits);  // normal orientation: `splits` = persistent CTAs (0: all SMs)
+  const int tiles = 2 * ((g.rows_a + 127) / 128) * ((g.rows_b + bn - 1) / bn);  // two tickets per tile
+  static thread_local float* ws = nullptr;
+  static thread_local int* tk = nullptr;
+  static thread_local size_t ws_cap = 0, tk_cap = 0;
+  const size_t need = tc_gemm_ws_floats(g);
+  if (need > ws_cap) {
+    if (ws) cudaFree(ws);
+    ws = nullptr;
+    ws_cap = 0;
+    if (cudaMalloc(&ws, need * 4) != cudaSuccess) return WAM_ERR_OOM;
+    ws_cap = need;
+  }
+  if ((size_t)tiles > tk_cap) {
+    if (tk) cudaFree(tk);
+    tk = nullptr;
+    tk_cap = 0;
+    if (cudaMalloc(&tk, tiles * 4) != cudaSuccess) return WAM_ERR_OOM;
+    if (cudaMemset(tk, 0, tiles * 4) != cudaSuccess) return WAM_ERR_CUDA;
+    tk_cap = tiles;
+  }
+  CUtensorMap mx, mw, mo;
+  if (!make_tmap_3d(&mx, x, K, M, 1, 0, swap ? bn : 128) || !make_tmap_3d(&mw, w, K, N, 1, 0, swap ? 128 : bn))
+    return WAM_ERR_INVALID_ARG;
+  if (!swap) {
+    if (!make_tmap_sw128(&mo, out, 4, N, M, 1, 0, 32, 32)) return WAM_ERR_INVALID_ARG;
+    e.map_o = &mo;
+  }
+  g.map_a = swap ? &mw : &mx;
+  g.map_b = swap ? &mx : &mw;
   g.ws = ws;
   g.tickets = tk;
   g.status = status;

@@ -22,9 +22,14 @@ def _f32(a):
     return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(DEV)
 
 
+# Normal orientation: `splits` = persistent CTAs (0: one per SM); the
+# k-blocks of all tiles are divided evenly between them (stream-K).
 @pytest.mark.parametrize("M_,N,K,swap,splits", [
-    (200, 384, 256, False, 1),     # ragged M tail, 2 x 3 tiles
-    (1088, 256, 128, False, 1),    # 8.5 row tiles
+    (200, 384, 256, False, 1),     # ragged M tail, 2 x 3 tiles, one CTA walks all
+    (200, 384, 256, False, 0),     # 24 k-blocks on 24 CTAs: every tile in 4 pieces
+    (1088, 256, 128, False, 0),    # 8.5 row tiles
+    (1088, 1536, 1536, False, 7),  # 7 CTAs: pieces of uneven length
+    (1088, 1536, 1536, False, 0),  # out-projection shape on all SMs
     (32, 300, 512, True, 1),       # few tokens, ragged feature tail
     (32, 300, 512, True, 4),       # split-K, fixed-order reduction
     (16, 30, 768, True, 3),        # action out-projection shape
