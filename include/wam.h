@@ -241,9 +241,9 @@ wam_status wam_op_norm_mod(int dtype, const float* dev_x, void* dev_h, int M, in
  *     where s is the number of non-empty key splits (at most 32);
  *     1 <= Lq <= 64.  A call beyond them returns WAM_ERR_UNSUPPORTED and
  *     enqueues nothing.
- *   - The first call on a device looks up the array's device address (once
- *     per device, with that device current); make that first call before
- *     any stream capture.
+ *   - The first call on a device looks up the array's device address and
+ *     sets the kernel's shared-memory limit (once per device, with that
+ *     device current); make that first call before any stream capture.
  *   - Every call shares the array: calls that overlap on the GPU (other
  *     streams, other threads) race.  Each call clears the tickets it uses
  *     before its kernel runs.

@@ -17,6 +17,8 @@
 // depend on CTA timing.
 //
 // fp32 path: one warp per (query, head), exact fp32 softmax (debug precision).
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,6 +30,7 @@ constexpr int kTQ = 64;     // queries per CTA (4 warps x 16)
 constexpr int kTK = 64;     // keys per tile
 constexpr int kAttnThreads = 128;
 constexpr int kMaxSplits = 32;  // key splits of the action attention
+constexpr int kCombineBytes = 96 * 1024;  // dynamic shared memory for staging partial O rows
 
 // Row-major [64][64] bf16 tile, 16-byte chunks XOR-swizzled by row.
 __device__ __forceinline__ uint32_t tile_off(int row, int chunk) {
@@ -52,8 +55,9 @@ __global__ void __launch_bounds__(kAttnThreads)
     attn_bf16_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
                      const __nv_bfloat16* __restrict__ vc, __nv_bfloat16* __restrict__ out, int H, int Lq,
                      int Lk, int Lcache, int splits, int keys_per_split, float* __restrict__ ws,
-                     int* __restrict__ tickets) {
+                     int* __restrict__ tickets, int rows_per_pass) {
   __shared__ __align__(128) uint8_t smem[kTQ * 128 + 2 * 2 * kTK * 128];
+  extern __shared__ float4 s_comb[];  // split path: [splits][rows_per_pass][16] partial O rows
   __shared__ int s_last;
   const uint32_t sQ = smem_u32(smem);
   const uint32_t sK0 = sQ + kTQ * 128;
@@ -246,12 +250,37 @@ __global__ void __launch_bounds__(kAttnThreads)
     for (int s2 = 0; s2 < splits; ++s2) s_f[s2][tid] *= inv;
   }
   __syncthreads();
-  for (int idx = tid; idx < Lq * kD; idx += kAttnThreads) {
-    const int row = idx / kD, d = idx - row * kD;
-    float acc = 0.f;
-#pragma unroll 4
-    for (int s2 = 0; s2 < splits; ++s2) acc += s_f[s2][row] * __ldcg(cO + (size_t)s2 * kTQ * kD + row * kD + d);
-    out[(size_t)(b * Lq + row) * A + h * kD + d] = __float2bfloat16_rn(acc);
+  // Stage the partial O rows of every split in shared memory, all copies in
+  // flight at once (the reads are L2-latency bound otherwise), then sum them
+  // in split order.
+  for (int r0 = 0; r0 < Lq; r0 += rows_per_pass) {
+    const int nr = min(rows_per_pass, Lq - r0);
+    for (int i = tid; i < splits * nr * 16; i += kAttnThreads) {
+      const int s2 = i / (nr * 16), rem = i - s2 * (nr * 16);
+      const int row = rem >> 4, c4 = rem & 15;
+      cp_async16(smem_u32(s_comb + (s2 * nr + row) * 16 + c4), cO + (size_t)s2 * kTQ * kD + (r0 + row) * kD + 4 * c4,
+                 true);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    for (int i = tid; i < nr * 16; i += kAttnThreads) {
+      const int row = i >> 4, c4 = i & 15;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s2 = 0; s2 < splits; ++s2) {
+        const float f = s_f[s2][r0 + row];
+        const float4 v4 = s_comb[(s2 * nr + row) * 16 + c4];
+        acc.x += f * v4.x;
+        acc.y += f * v4.y;
+        acc.z += f * v4.z;
+        acc.w += f * v4.w;
+      }
+      uint2 w;
+      w.x = pack_bf16(acc.x, acc.y);
+      w.y = pack_bf16(acc.z, acc.w);
+      *reinterpret_cast<uint2*>(out + (size_t)(b * Lq + r0 + row) * A + h * kD + 4 * c4) = w;
+    }
+    __syncthreads();
   }
   if (tid == 0) tickets[bh] = 0;
 }
@@ -316,6 +345,10 @@ size_t attention_ws_floats(int B, int H, int Dh, int Lq, int splits) {
   return (size_t)B * H * splits * (kTQ * kD + kTQ * 2);
 }
 
+cudaError_t prepare_attention_bf16() {
+  return cudaFuncSetAttribute(attn_bf16_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kCombineBytes);
+}
+
 cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s) {
   if (a.Dh != kD) return cudaErrorInvalidValue;
   const int splits = a.splits < 1 ? 1 : a.splits;
@@ -329,11 +362,13 @@ cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s) {
   const auto* k = reinterpret_cast<const __nv_bfloat16*>(a.k);
   const auto* v = reinterpret_cast<const __nv_bfloat16*>(a.v);
   auto* o = reinterpret_cast<__nv_bfloat16*>(a.out);
-  if (used > 1)
-    return launch_k(attn_bf16_kernel<true>, grid, dim3(kAttnThreads), 0, s, q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache,
-                    used, kps, a.ws, a.tickets);
+  if (used > 1) {
+    const int rpp = std::max(1, std::min(a.Lq, kCombineBytes / (used * kD * 4)));
+    return launch_k(attn_bf16_kernel<true>, grid, dim3(kAttnThreads), (size_t)used * rpp * kD * 4, s, q, k, v, o,
+                    a.H, a.Lq, a.Lk, a.Lcache, used, kps, a.ws, a.tickets, rpp);
+  }
   return launch_k(attn_bf16_kernel<false>, grid, dim3(kAttnThreads), 0, s, q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache, 1,
-                  kps, (float*)nullptr, (int*)nullptr);
+                  kps, (float*)nullptr, (int*)nullptr, 0);
 }
 
 cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t s) {

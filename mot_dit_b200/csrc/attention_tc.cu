@@ -7,14 +7,18 @@
 //
 // Per 128-key tile j:
 //   S_j  = Q K_j^T       tcgen05.mma M=128 N=128 K=64, fp32 in TMEM (128 cols)
-//   P_j  = exp2((S_j - m_j) log2e / 8)      softmax warps, thread = query row,
+//   P_j  = exp2(S_j log2e / 8 - m)      softmax warps, thread = query row,
 //          rounded to bf16 into shared memory in the 128B-swizzled K-major
 //          layout the next MMA reads (fence.proxy.async before the hand-off)
-//   PV_j = P_j V_j       tcgen05.mma M=128 N=64 K=128, V as the MN-major B
-//          operand (the cache rows are [key][64 channels]), fp32 in TMEM
-//   O    = O alpha_j + PV_j in registers (online-softmax rescale)
-// The MMA warp issues S_{j+1} before PV_j, so the next scores are ready when
-// the softmax warps finish tile j; K/V tiles are double-buffered by TMA.
+//   O   += P_j V_j       tcgen05.mma M=128 N=64 K=128 accumulating in TMEM, V
+//          as the MN-major B operand (the cache rows are [key][64 channels])
+// The reference maximum m of a row is raised (and O and the row sum rescaled
+// in place) only when a tile's maximum exceeds it by more than 2^8: exact
+// softmax arithmetic with a stale maximum, P <= 256, and in most tiles no
+// TMEM round trip of O.  P has one buffer: P_j is written once PV_{j-1}
+// (which reads P_{j-1}) has completed.  The MMA warp issues S_{j+1}
+// before PV_j, so the next scores are ready when the softmax warps finish
+// tile j; K/V tiles are double-buffered by TMA.
 //
 // Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
 // issuer, warps 2..5 softmax / output (warp w owns TMEM lanes 32*(w%4)..+31).
@@ -32,7 +36,8 @@ constexpr int kStagesKV = 2;
 constexpr int kTileBytes = kKT * kDh * 2;  // 16 KB (one K or V tile, also the Q tile)
 constexpr int kPBytes = kQ * kKT * 2;      // 32 KB
 constexpr int kThreads = 192;
-constexpr int kTmemCols = 256;             // S: cols [0,128), PV: cols [128,192)
+constexpr int kTmemCols = 256;             // S: cols [0,128), O: cols [128,192)
+constexpr float kRescale = 8.0f;           // log2 headroom of the stale row maximum
 constexpr int kBarBytes = 128;
 // No alignment slack: two CTAs per SM need every byte (2 x (112 KB + 1 KB reserved) <= 228 KB).
 constexpr int kSmem = kTileBytes + kStagesKV * 2 * kTileBytes + kPBytes + kBarBytes;
@@ -79,6 +84,32 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 lanes x 64 columns back into TMEM, one wait.
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
+      "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
+      "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]),
+      "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]),
+      "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]),
+      "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31]), "f"(v[32]), "f"(v[33]), "f"(v[34]), "f"(v[35]), "f"(v[36]),
+      "f"(v[37]), "f"(v[38]), "f"(v[39]), "f"(v[40]), "f"(v[41]), "f"(v[42]), "f"(v[43]), "f"(v[44]), "f"(v[45]),
+      "f"(v[46]), "f"(v[47]), "f"(v[48]), "f"(v[49]), "f"(v[50]), "f"(v[51]), "f"(v[52]), "f"(v[53]), "f"(v[54]),
+      "f"(v[55]), "f"(v[56]), "f"(v[57]), "f"(v[58]), "f"(v[59]), "f"(v[60]), "f"(v[61]), "f"(v[62]), "f"(v[63])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // 2^x on the special-function unit (the hardware approximation, flushing
@@ -177,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kQ, kKT);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kQ, kDh) | (1u << 16);  // B (V) is MN-major
-      const uint32_t t_s = tmem, t_pv = tmem + 128;
+      const uint32_t t_s = tmem, t_o = tmem + 128;
       const uint32_t aq = smem_u32(sQ);
       auto issue_s = [&](int j) {
         const int s = j % kStagesKV;
@@ -200,8 +231,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t ap = smem_u32(sP), av = smem_u32(sV + s * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kKT / 16; ++kk)
-          tc_mma_bf16(t_pv, smem_desc_k128(ap + (kk >> 2) * (kQ * 128) + (kk & 3) * 32),
-                      smem_desc_mn128(av + kk * 16 * 128), idesc_pv, kk > 0 ? 1u : 0u);
+          tc_mma_bf16(t_o, smem_desc_k128(ap + (kk >> 2) * (kQ * 128) + (kk & 3) * 32),
+                      smem_desc_mn128(av + kk * 16 * 128), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(pv_full);
         tc_commit(&kv_empty[s]);
       }
@@ -214,10 +245,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int r = quad * 32 + lane;  // query row within the tile
     const uint32_t t_row = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float sl2e = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
-    float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
-    float o[kDh];
-#pragma unroll
-    for (int i = 0; i < kDh; ++i) o[i] = 0.f;
+    float mref = 0.f, l = 0.f;  // reference maximum (scaled log2 units) and row sum
     uint8_t* prow = sP + r * 128;
     const int swz = r & 7;
     bool ok = true;
@@ -228,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       tc_fence_after();
       const int kbase = j * kKT;
-      const int nvalid = min(kKT, a.Lk - kbase);  // keys of this tile inside [0, Lk)
+      const int nvalid = min(kKT, a.Lk - kbase);  // keys of this tile inside [0, Lk) (>= 1)
       // pass 1: row maximum of the valid keys
       float mx = -INFINITY;
 #pragma unroll
@@ -237,29 +265,38 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_ld64(t_row + c, v);
         if (nvalid == kKT) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) mx = fmaxf(mx, v[i]);
+          for (int i = 0; i < 64; i += 2) mx = fmax3(mx, v[i], v[i + 1]);
         } else {
 #pragma unroll
           for (int i = 0; i < 64; ++i)
             if (c + i < nvalid) mx = fmaxf(mx, v[i]);
         }
       }
-      const float m_new = fmaxf(m, mx);
-      const float alpha = ex2((m - m_new) * sl2e);  // m = -inf on the first tile: alpha = 0
-      const float mb = m_new * sl2e;
-      // O += PV_{j-1} (relative to the previous maximum); frees P and the PV columns
-      if (j > 0) {
-        if (!mbar_wait(pv_full, (j - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag)) {
+      const float mxs = mx * sl2e;
+      if (j == 0) {
+        mref = mxs;  // O is written from scratch by the first PV
+      } else {
+        // PV_{j-1} still reads P_{j-1} from the one P buffer: wait for it
+        // before P_j overwrites it (and before O may be rescaled)
+        const bool got = mbar_wait(pv_full, (j - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {  // leave together: the TMEM accesses below are warp-wide
           ok = false;
           break;
         }
         tc_fence_after();
-        float pv[64];
-        tmem_ld64(t_row + 128, pv);
+        const bool need = mxs > mref + kRescale;
+        if (__any_sync(0xffffffffu, need)) {  // tcgen05.ld / st are warp-wide
+          const float alpha = need ? ex2(mref - mxs) : 1.f;
+          if (need) mref = mxs;
+          float o[64];
+          tmem_ld64(t_row + 128, o);
 #pragma unroll
-        for (int i = 0; i < kDh; ++i) o[i] = o[i] * alpha_prev + pv[i];
+          for (int i = 0; i < kDh; ++i) o[i] *= alpha;
+          tmem_st64(t_row + 128, o);
+          l *= alpha;
+        }
       }
-      // pass 2: P = 2^(s log2e/8 - m log2e/8) as bf16 into the swizzled P tile
+      // pass 2: P = 2^(s log2e/8 - mref) as bf16 into the swizzled P tile
       float rs = 0.f;
 #pragma unroll
       for (int c = 0; c < kKT; c += 64) {
@@ -268,13 +305,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (nvalid == kKT) {
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
-            v[i] = ex2(fmaf(v[i], sl2e, -mb));
+            v[i] = ex2(fmaf(v[i], sl2e, -mref));
             rs += v[i];
           }
         } else {
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
-            v[i] = (c + i < nvalid) ? ex2(fmaf(v[i], sl2e, -mb)) : 0.f;
+            v[i] = (c + i < nvalid) ? ex2(fmaf(v[i], sl2e, -mref)) : 0.f;
             rs += v[i];
           }
         }
@@ -289,9 +326,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           *reinterpret_cast<uint4*>(blk + ((q ^ swz) << 4)) = w;
         }
       }
-      l = l * alpha + rs;
-      m = m_new;
-      alpha_prev = alpha;
+      l += rs;
       tc_fence_before();
       fence_proxy_async_smem();  // P (generic-proxy stores) -> tensor-core reads
       mbar_arrive_cta(p_full);
@@ -299,10 +334,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (ok && ntiles > 0 &&
         mbar_wait(pv_full, (ntiles - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag)) {
       tc_fence_after();
-      float pv[64];
-      tmem_ld64(t_row + 128, pv);
-#pragma unroll
-      for (int i = 0; i < kDh; ++i) o[i] = o[i] * alpha_prev + pv[i];
+      float o[64];
+      tmem_ld64(t_row + 128, o);
       const int qi = q0 + r;
       if (qi < a.Lq) {
         const float inv = 1.0f / l;

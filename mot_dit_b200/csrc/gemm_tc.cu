@@ -58,13 +58,21 @@ enum : int {
   kClassStore = 1,   // fp32 store / GELU: two output boxes per warp
   kClassRes = 2,     // gate-residual: the warp's 32 x BN residual rows (BN <= 128)
   kClassQkv = 3,     // QK-norm + RoPE: 32 cos + 32 sin rows and two output boxes per warp
+  kClassNormB = 4,   // swapped, B = RMSNorm/modulation of fp32 token rows computed in the kernel
 };
+
+// Largest reduction length of the fused-norm B operand (held whole in shared memory).
+constexpr int kNormKMax = 1024;
 
 template <int BN, bool SWAP, int EPI>
 struct TileCfg {
+  static constexpr bool kNB = EPI == kClassNormB;
+  static_assert(!kNB || (SWAP && BN <= 64), "fused-norm B operand: swapped orientation, <= 64 tokens");
   static constexpr int kABytes = BM * BK * 2;
-  static constexpr int kBBytes = BN * BK * 2;
+  static constexpr int kBBytes = kNB ? 0 : BN * BK * 2;  // per stage
   static constexpr int kStageBytes = kABytes + kBBytes;
+  // fused-norm B operand, resident: [k-block][BN rows][128 B], 128-byte swizzle
+  static constexpr int kResB = kNB ? (kNormKMax / BK) * BN * 128 : 0;
   static constexpr int kTmemCols = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
   static constexpr int kWarpStg = SWAP ? 0
                                        : (EPI == kClassStore ? 2 * kBox
@@ -73,7 +81,7 @@ struct TileCfg {
   static constexpr int kSwapStg = SWAP ? 32 * (BM + 1) * 4 : 0;  // swapped QKV staging [32 tokens][129]
   // the tile's bias slice (and gate or QK gains) in shared memory, normal orientation
   static constexpr int kVecBytes = (SWAP || EPI == kClassScalar) ? 0 : (EPI == kClassStore ? 1 : 2) * BN * 4;
-  static constexpr int kExtra = 4 * kWarpStg + kSwapStg + kVecBytes;
+  static constexpr int kExtra = kResB + 4 * kWarpStg + kSwapStg + kVecBytes;
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemMax = 232448;  // 227 KB per CTA
   static constexpr int kFit = (kSmemMax - 1024 - kBarBytes - kExtra) / kStageBytes;
@@ -333,14 +341,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kStages * C::kABytes;
-  uint8_t* sStg = smem + C::kStages * C::kStageBytes;  // epilogue staging (1024-byte aligned)
+  uint8_t* sBres = smem + C::kStages * C::kStageBytes;  // fused-norm B operand (1024-byte aligned)
+  uint8_t* sStg = sBres + C::kResB;                     // epilogue staging (1024-byte aligned)
   float* sVec = reinterpret_cast<float*>(sStg + 4 * C::kWarpStg + C::kSwapStg);  // [BN] bias, [BN] gate / gains
-  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + C::kExtra);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes + C::kExtra);
   uint64_t* empty = full + C::kStages;
   uint64_t* accf = empty + C::kStages;  // [2] accumulator ready (MMA -> epilogue)
   uint64_t* acce = accf + 2;            // [2] accumulator drained (epilogue -> MMA)
   uint64_t* redb = acce + 2;            // partial tiles copied into the ring
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redb + 1);
+  uint64_t* bready = redb + 1;          // fused-norm B operand written (epilogue warps -> MMA)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -357,13 +367,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acce[b], 4);
     }
     mbar_init(redb, 1);
+    mbar_init(bready, 1);
     *abort_flag = 0;
     *last_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&map_a);
-    prefetch_tensormap(&map_b);
+    if (!C::kNB) prefetch_tensormap(&map_b);
     if (!SWAP && EPI != kClassScalar) prefetch_tensormap(&map_o);
     if (!SWAP && EPI == kClassQkv) prefetch_tensormap(&map_o2);
   }
@@ -395,15 +406,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             tma_load_3d(sB + i * C::kBBytes, &map_b, &full[i], (sg.kb0 + i) * BK, tb * BN, g.z_b);
         }
-        pdl_wait();
-        for (int i = 0; i < pre; ++i) {
+        // with the fused norm the producer reads weights only: no wait for the previous kernel
+        if (!C::kNB) pdl_wait();
+        for (int i = 0; i < pre && !C::kNB; ++i) {
           if (SWAP)
             tma_load_3d(sB + i * C::kBBytes, &map_b, &full[i], (sg.kb0 + i) * BK, tb * BN, g.z_b);
           else
             tma_load_3d(sA + i * C::kABytes, &map_a, &full[i], (sg.kb0 + i) * BK, ta * BM, g.z_a);
         }
         issued = pre;
-      } else {
+      } else if (!C::kNB) {
         pdl_wait();
       }
       for (long long x = x_begin; x < x_end && ok;) {
@@ -420,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&full[s], C::kStageBytes);
           tma_load_3d(sA + s * C::kABytes, &map_a, &full[s], kb * BK, ta * BM, g.z_a);
-          tma_load_3d(sB + s * C::kBBytes, &map_b, &full[s], kb * BK, tb * BN, g.z_b);
+          if (!C::kNB) tma_load_3d(sB + s * C::kBBytes, &map_b, &full[s], kb * BK, tb * BN, g.z_b);
           issued = it + 1;
         }
       }
@@ -433,6 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
       int it = 0, lt = 0;
       bool ok = true;
+      if (C::kNB && x_begin < x_end) {  // the B operand is computed by the epilogue warps
+        ok = mbar_wait(bready, 0, g.status, kStatusTimeoutTmaFull, abort_flag);
+        tc_fence_after();
+      }
       for (long long x = x_begin; x < x_end && ok; ++lt) {
         const Seg sg = seg_at(g, x, x_end);
         x += sg.kb1 - sg.kb0;
@@ -451,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * C::kABytes);
-          const uint32_t b0 = smem_u32(sB + s * C::kBBytes);
+          const uint32_t b0 = C::kNB ? smem_u32(sBres + kb * (BN * 128)) : smem_u32(sB + s * C::kBBytes);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             tc_mma_bf16(d_tmem, smem_desc_k128(a0 + k * 32), smem_desc_k128(b0 + k * 32), idesc,
@@ -468,6 +484,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;
     const int row = quad * 32 + lane;  // TMEM lane = tile row
     const EpiRegs R = hoist(e);
+    if constexpr (C::kNB) {
+      // B = rms(x) * (gain or 1 + scale) + shift as bf16, in the layout a
+      // 128-byte-swizzled TMA load of [BN rows][64] would give each k-block.
+      // Four threads share a row: first every row's sum of squares over all K
+      // (loads issued 24 float4 at a time), then only the k-blocks this CTA's
+      // segments read.
+      const int K = g.K, n4 = K / 4;
+      const int te = threadIdx.x - 64;  // 0..127
+      float* sRR = reinterpret_cast<float*>(sStg);  // [BN] 1 / rms (the swapped staging is free until then)
+      for (int p = 0; p < BN / 32; ++p) {
+        const int r = p * 32 + (te >> 2), part = te & 3;
+        const bool valid = r < g.rows_b;
+        const float4* xr = reinterpret_cast<const float4*>(e.nb_x + (size_t)(valid ? r : 0) * K);
+        float ss = 0.f;
+        for (int i0 = 0; i0 < n4 / 4; i0 += 24) {
+          float4 v[24];
+#pragma unroll
+          for (int i = 0; i < 24; ++i) {
+            const int k4 = part + 4 * (i0 + i);
+            v[i] = (valid && k4 < n4) ? xr[k4] : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int i = 0; i < 24; ++i) ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+        }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        if (part == 0) sRR[r] = 1.0f / sqrtf(ss / (float)K + 1e-6f);
+      }
+      epi_bar();
+      unsigned need = 0;  // k-blocks of this CTA's segments (K <= 1024: at most 16)
+      for (long long xx = x_begin; xx < x_end;) {
+        const Seg sg = seg_at(g, xx, x_end);
+        xx += sg.kb1 - sg.kb0;
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb) need |= 1u << kb;
+      }
+      for (int kb = 0; kb < K / BK; ++kb) {
+        if (!(need >> kb & 1u)) continue;
+        const int c0 = kb * BK + (te & 3) * 16;  // this thread's 16 columns
+        float4 mul[4], add[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (e.nb_gain) {
+            mul[i] = __ldg(reinterpret_cast<const float4*>(e.nb_gain + c0) + i);
+          } else {
+            mul[i] = __ldg(reinterpret_cast<const float4*>(e.nb_scale + c0) + i);
+            mul[i].x += 1.f;
+            mul[i].y += 1.f;
+            mul[i].z += 1.f;
+            mul[i].w += 1.f;
+          }
+          add[i] = e.nb_shift ? __ldg(reinterpret_cast<const float4*>(e.nb_shift + c0) + i)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int p = 0; p < BN / 32; ++p) {
+          const int r = p * 32 + (te >> 2);
+          const bool valid = r < g.rows_b;
+          const float4* xr = reinterpret_cast<const float4*>(e.nb_x + (size_t)(valid ? r : 0) * K + c0);
+          float4 v[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) v[i] = valid ? xr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float rr = sRR[r];
+          uint32_t w[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            w[2 * i] = valid ? pack_bf16(v[i].x * rr * mul[i].x + add[i].x, v[i].y * rr * mul[i].y + add[i].y) : 0u;
+            w[2 * i + 1] = valid ? pack_bf16(v[i].z * rr * mul[i].z + add[i].z, v[i].w * rr * mul[i].w + add[i].w) : 0u;
+          }
+          const int q = (te & 3) * 2;  // two 16-byte chunks of the 128-byte row
+          uint8_t* rowp = sBres + kb * (BN * 128) + r * 128;
+          *reinterpret_cast<uint4*>(rowp + ((q ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(rowp + (((q + 1) ^ (r & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+      }
+      fence_proxy_async_smem();  // generic writes -> visible to the tensor core
+      epi_bar();                 // (the staging's 1 / rms values are read; it may be reused)
+      if (threadIdx.x == 64) mbar_arrive(bready);
+    }
     uint8_t* stg = sStg + quad * C::kWarpStg;  // this warp's staging (normal orientation)
     int nbox = 0;                              // output boxes this warp stored (double-buffer index)
     int lt = 0;
@@ -963,6 +1056,27 @@ cudaError_t launch_normal(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
 
 size_t tc_gemm_ws_floats(const TcGemm& t) { return (size_t)ctas_of(t) * 2 * BM * t.bn; }
 
+namespace {
+template <int BN, bool SWAP, int EPI>
+int ring_partials() {
+  using C = TileCfg<BN, SWAP, EPI>;
+  return C::kStages * C::kStageBytes / (BM * BN * 4);
+}
+}  // namespace
+
+int tc_gemm_ring_partials(int bn, bool swap, bool fused_norm) {
+  if (swap && fused_norm) return bn == 32 ? ring_partials<32, true, kClassNormB>() : ring_partials<64, true, kClassNormB>();
+  if (swap) {
+    switch (bn) {
+      case 32: return ring_partials<32, true, kClassScalar>();
+      case 64: return ring_partials<64, true, kClassScalar>();
+      case 128: return ring_partials<128, true, kClassScalar>();
+      default: return ring_partials<256, true, kClassScalar>();
+    }
+  }
+  return bn == 256 ? ring_partials<256, false, kClassQkv>() : ring_partials<128, false, kClassRes>();
+}
+
 cudaError_t prepare_tc_gemm() {
   cudaError_t e;
   int dev = 0;
@@ -974,6 +1088,8 @@ cudaError_t prepare_tc_gemm() {
   WAM_PREP(64, true, kClassScalar)
   WAM_PREP(128, true, kClassScalar)
   WAM_PREP(256, true, kClassScalar)
+  WAM_PREP(32, true, kClassNormB)
+  WAM_PREP(64, true, kClassNormB)
   WAM_PREP(64, false, kClassScalar)
   WAM_PREP(64, false, kClassStore)
   WAM_PREP(64, false, kClassRes)
@@ -992,6 +1108,15 @@ cudaError_t prepare_tc_gemm() {
 cudaError_t launch_tc_gemm(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
   if (g_num_sms == 0) return cudaErrorNotReady;
   if (!t.ws || !t.tickets) return cudaErrorInvalidValue;
+  if (e.nb_x) {  // fused norm of the token rows: swapped, one token tile, K <= kNormKMax
+    if (!t.swap || t.rows_b > t.bn || t.K > kNormKMax || t.K % BK)
+      return cudaErrorInvalidValue;
+    switch (t.bn) {
+      case 32: return launch_one<32, true, kClassNormB>(t, e, s);
+      case 64: return launch_one<64, true, kClassNormB>(t, e, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   if (t.swap) {
     switch (t.bn) {
       case 32: return launch_one<32, true, kClassScalar>(t, e, s);

@@ -93,6 +93,13 @@ struct EpiArgs {
   const CUtensorMap* map_o = nullptr;
   const CUtensorMap* map_o2 = nullptr;
   int zq0 = 0, zk0 = 0, zv0 = 0;
+  // Swapped orientation only: the B operand (tokens x K) is computed in the
+  // kernel as rms(nb_x) * (nb_gain or 1 + nb_scale) + nb_shift from fp32 rows
+  // nb_x [tokens][K] (ld = K) instead of being loaded; map_b is then unused.
+  const float* nb_x = nullptr;
+  const float* nb_scale = nullptr;
+  const float* nb_shift = nullptr;
+  const float* nb_gain = nullptr;
 };
 
 // C[m, n] = sum_k X[m, k] W[n, k] (+ epilogue), bf16 operands via TMA into
@@ -114,6 +121,11 @@ struct TcGemm {
 
 // Workspace floats the launch needs for K-split partial tiles.
 size_t tc_gemm_ws_floats(const TcGemm& g);
+// Partial tiles the last piece of a split tile can bring into its operand
+// ring at once (the fast reduction path); tiles split into more pieces are
+// summed from global memory instead.  Normal orientation: the smallest ring
+// of the 128- / 256-wide instances.
+int tc_gemm_ring_partials(int bn, bool swap, bool fused_norm);
 
 cudaError_t launch_tc_gemm(const TcGemm& g, const EpiArgs& e, cudaStream_t s);
 // Sets the kernels' shared-memory attributes; call once per device before any
@@ -157,6 +169,9 @@ struct AttnArgs {
   int* tickets;      // B*H counters, zero on entry, left zero
 };
 cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s);
+// Sets the split kernel's shared-memory limit; call once per device before
+// any launch (and never during stream capture).
+cudaError_t prepare_attention_bf16();
 
 // Tensor-core (tcgen05) attention for video queries: one pass over keys
 // [0, Lk) for 128-query tiles.  Q / K / V are 3-D TMA maps over [z][rows][64]

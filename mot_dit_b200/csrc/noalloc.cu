@@ -41,6 +41,8 @@ cudaError_t scratch_address(int dev, void** out) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
     if (e != cudaSuccess) return e;
+    // the split kernel's shared-memory limit is a per-device setting too
+    if ((e = wam::prepare_attention_bf16()) != cudaSuccess) return e;
     g_addr[dev] = p;
   }
   *out = g_addr[dev];

@@ -96,10 +96,9 @@ struct wam_ctx {
   GemmPlan p_v_qkv, p_v_o, p_v_f1, p_v_f2, p_v_in, p_v_out;
   GemmPlan p_a_in, p_a_qkv, p_a_o, p_a_f1, p_a_f2, p_a_out;
   int attn_splits = 1;
-  // Persistent grid of the video GEMMs while the action stream runs beside
-  // them (CEWP); otherwise they take every SM.
-  int video_ctas_overlap = 0;
-  bool video_overlap = false;
+  // The action expert's norms run inside the GEMM that consumes them (opt-in;
+  // the tokens must fit one 32/64-wide tile and K <= 1024).
+  bool fuse_norm_a = false;
 
   // TMA maps
   CUtensorMap m_hv, m_ov, m_fv, m_xvin, m_w_qkv_v, m_w_o_v, m_w_f1_v, m_w_f2_v, m_w_vin, m_w_vout;
@@ -277,7 +276,7 @@ inline void* vcache(wam_ctx* c, int i) {
 }
 
 // ------------------------------------------------------------- planning ---
-GemmPlan plan_swap(int rows_w, int tokens, int K, int bn) {
+GemmPlan plan_swap(int rows_w, int tokens, int K, int bn, bool fused_norm) {
   GemmPlan p;
   p.bn = bn;
   const int tiles = ((rows_w + 127) / 128) * ((tokens + bn - 1) / bn);
@@ -285,6 +284,10 @@ GemmPlan plan_swap(int rows_w, int tokens, int K, int bn) {
   int s = (148 + tiles - 1) / tiles;
   const int min_kb = 3;  // keep each split a few k-blocks deep
   if (s > kb / min_kb) s = kb / min_kb;
+  // a tile takes at most splits + 1 pieces; the last one's partner partials
+  // must fit its operand ring for the fast reduction
+  const int cap = tc_gemm_ring_partials(bn, true, fused_norm);
+  if (s > cap) s = cap;
   if (s < 1) s = 1;
   p.splits = s;
   return p;
@@ -304,7 +307,7 @@ wam_status run_tc(wam_ctx* c, const CUtensorMap& A, const CUtensorMap& Bm, int r
   g.bn = p.bn;
   g.splits = p.splits;
   g.swap = swap;
-  g.max_ctas = (video && c->video_overlap && p.max_ctas == 0) ? c->video_ctas_overlap : p.max_ctas;
+  g.max_ctas = p.max_ctas;
   g.ws = video ? c->ws_gemm_v : c->ws_gemm;
   g.tickets = video ? c->tk_gemm_v : c->tk_gemm;
   g.status = c->status;
@@ -397,6 +400,12 @@ wam_status norm(wam_ctx* c, const float* x, void* h, int M, int dm, const float*
   return WAM_OK;
 }
 
+// Action-expert linear layer whose input is h = rms(x_a) (gain or 1 + scale)
+// + shift: the norm is computed inside the GEMM when it fits, otherwise by
+// the norm kernel into h_a first.  `cls` is the profile class of the GEMM.
+wam_status norm_linear(wam_ctx* c, const Lin& L, EpiArgs e, const float* sc, const float* sh, const float* gain,
+                       int cls, cudaStream_t s);
+
 wam_status temb(wam_ctx* c, bool video, const float* t, cudaStream_t s) {
   const ExpertIdx& x = video ? c->ev : c->ea;
   TembArgs a;
@@ -464,6 +473,22 @@ wam_status attention(wam_ctx* c, bool video, int i, cudaStream_t s) {
     wam_status r_ = (expr);             \
     if (r_ != WAM_OK) return r_;        \
   } while (0)
+
+wam_status norm_linear(wam_ctx* c, const Lin& L, EpiArgs e, const float* sc, const float* sh, const float* gain,
+                       int cls, cudaStream_t s) {
+  const Dims& d = c->d;
+  if (c->fuse_norm_a) {
+    e.nb_x = c->x_a;
+    e.nb_scale = sc;
+    e.nb_shift = sh;
+    e.nb_gain = gain;
+  } else {
+    c->cur_cls = WAM_PROF_ACTION_NORM;
+    RET(norm(c, c->x_a, c->h_a, d.Ma, d.da, sc, sh, gain, s));
+  }
+  c->cur_cls = cls;
+  return linear(c, false, L, d.Ma, e, c->qkv_tmp_a, s);
+}
 
 // ------------------------------------------------------------- experts ----
 // Video expert: P^v_i -> record(e_i) -> Attn^v_i -> R^v_i for every block.
@@ -540,11 +565,8 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
   }
   for (int i = 0; i < d.N; ++i) {
     const float* mod = c->mod_a + (size_t)i * 6 * d.da;
-    c->cur_cls = WAM_PROF_ACTION_NORM;
-    RET(norm(c, c->x_a, c->h_a, d.Ma, d.da, mod + d.da, mod, nullptr, s));
-    c->cur_cls = WAM_PROF_ACTION_QKV;
     Lin Lq{&c->m_w_qkv_a, &c->m_ha, matp(c, blk(x, i, kQkvW)), c->h_a, 3 * d.A, d.da, i, &c->p_a_qkv};
-    RET(linear(c, false, Lq, d.Ma, epi_qkv(c, false, i), c->qkv_tmp_a, s));
+    RET(norm_linear(c, Lq, epi_qkv(c, false, i), mod + d.da, mod, nullptr, WAM_PROF_ACTION_QKV, s));
     if (ev_wait) CK(cudaStreamWaitEvent(s, ev_wait[i], 0));
     c->cur_cls = WAM_PROF_ACTION_ATTN;
     RET(attention(c, false, i, s));
@@ -554,26 +576,22 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
     eo.gate = mod + 2 * d.da;
     Lin Lo{&c->m_w_o_a, &c->m_oa, matp(c, blk(x, i, kOW)), c->o_a, d.da, d.A, i, &c->p_a_o};
     RET(linear(c, false, Lo, d.Ma, eo, nullptr, s));
-    c->cur_cls = WAM_PROF_ACTION_NORM;
-    RET(norm(c, c->x_a, c->h_a, d.Ma, d.da, mod + 4 * d.da, mod + 3 * d.da, nullptr, s));
-    c->cur_cls = WAM_PROF_ACTION_FFN_UP;
     Lin L1{&c->m_w_f1_a, &c->m_ha, matp(c, blk(x, i, kF1W)), c->h_a, d.Fa, d.da, i, &c->p_a_f1};
-    RET(linear(c, false, L1, d.Ma, epi_base(kEpiGelu, vecp(c, blk(x, i, kF1B)), nullptr, c->f_a, d.Fa), nullptr, s));
+    RET(norm_linear(c, L1, epi_base(kEpiGelu, vecp(c, blk(x, i, kF1B)), nullptr, c->f_a, d.Fa), mod + 4 * d.da,
+                    mod + 3 * d.da, nullptr, WAM_PROF_ACTION_FFN_UP, s));
     c->cur_cls = WAM_PROF_ACTION_FFN_DOWN;
     EpiArgs e2 = epi_base(kEpiGateRes, vecp(c, blk(x, i, kF2B)), c->x_a, nullptr, d.da);
     e2.gate = mod + 5 * d.da;
     Lin L2{&c->m_w_f2_a, &c->m_fa, matp(c, blk(x, i, kF2W)), c->f_a, d.da, d.Fa, i, &c->p_a_f2};
     RET(linear(c, false, L2, d.Ma, e2, nullptr, s));
   }
-  c->cur_cls = WAM_PROF_ACTION_IO;
-  RET(norm(c, c->x_a, c->h_a, d.Ma, d.da, nullptr, nullptr, vecp(c, x.fng), s));
   EpiArgs ee = epi_base(kEpiEuler, vecp(c, x.outb), c->a_state, nullptr, d.Pa);
   ee.aio = io;
   ee.step = j;
   ee.a_next = d.bf16 ? c->a_in : nullptr;
   ee.a_next_ld = d.Kin;
   Lin Lout{&c->m_w_out, &c->m_ha, matp(c, x.outw), c->h_a, d.Pa, d.da, 0, &c->p_a_out};
-  RET(linear(c, false, Lout, d.Ma, ee, nullptr, s));
+  RET(norm_linear(c, Lout, ee, nullptr, nullptr, vecp(c, x.fng), WAM_PROF_ACTION_IO, s));
   return WAM_OK;
 }
 
@@ -600,10 +618,7 @@ wam_status enqueue_chunk(wam_ctx* c, int steps, int mode, bool joint, cudaStream
   if (cewp) {
     // Enqueue the two experts interleaved block by block is not needed: the
     // streams run concurrently; the per-block events order Attn^a_i after P^v_i.
-    c->video_overlap = true;
-    const wam_status st = enqueue_video(c, sv, c->vio_chunk, joint, ev_kv, false);
-    c->video_overlap = false;
-    RET(st);
+    RET(enqueue_video(c, sv, c->vio_chunk, joint, ev_kv, false));
     for (int j = 0; j < steps; ++j) RET(enqueue_action_step(c, sa, c->aio_chunk, j, j == 0 ? ev_kv : nullptr, false));
   } else {
     RET(enqueue_video(c, sv, c->vio_chunk, joint, nullptr, false));
@@ -811,6 +826,7 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   CK(cudaGetDevice(&c->device));
   CK(prepare_tc_gemm());
   CK(prepare_attention_tc());
+  CK(prepare_attention_bf16());
   Dims& d = c->d;
   d.N = cfg->n_blocks; d.dv = cfg->d_video; d.da = cfg->d_action; d.H = cfg->n_heads; d.Dh = cfg->head_dim;
   d.A = d.H * d.Dh; d.Fv = cfg->ffn_video; d.Fa = cfg->ffn_action; d.Lc = cfg->l_cond; d.Lvid = cfg->l_video;
@@ -875,30 +891,40 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     // Video GEMMs (tokens on TMEM lanes): stream-K over a persistent grid, so
     // every CTA gets the same share of k-blocks whatever the tile count.  The
     // wide projections (QKV, FFN-up) take 256-feature tiles (half the operand
-    // traffic per flop of 128); out-proj / FFN-down keep 128 (their residual
-    // staging holds 128 columns).  Under CEWP the video GEMMs leave about a
-    // quarter of the SMs to the action stream (108 of 148 measured best on
-    // the config-2 chunk); WAM_VIDEO_GEMM_CTAS overrides the count.
+    // traffic per flop of 128); out-proj / FFN-down keep 128, their
+    // gate-residual epilogue staging the residual rows (measured: a 256-wide
+    // plain store with the residual folded into the next norm was slower
+    // overall).  The video GEMMs leave about a quarter of
+    // the SMs to the action stream that runs beside them under CEWP (108 of
+    // 148 measured best on the config-2 chunk; WAM_VIDEO_GEMM_CTAS overrides
+    // the count).  The grid is the same in every schedule: the k-range
+    // split points, and so every rounding, do not depend on the schedule.
     int nsm = 148;
     CK(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, c->device));
-    c->video_ctas_overlap = std::max(1, nsm * 73 / 100);
+    int vctas = std::max(1, nsm * 73 / 100);
     if (const char* v = getenv("WAM_VIDEO_GEMM_CTAS")) {
       const int n = atoi(v);
-      if (n > 0) c->video_ctas_overlap = std::min(n, nsm);
+      if (n > 0) vctas = std::min(n, nsm);
     }
-    c->p_v_qkv = {256, 1, 0};
-    c->p_v_o = {128, 1, 0};
-    c->p_v_f1 = {256, 1, 0};
-    c->p_v_f2 = {128, 1, 0};
-    c->p_v_in = {128, 1, 0};
-    c->p_v_out = {64, 1, 0};
+    c->p_v_qkv = {256, 1, vctas};
+    c->p_v_o = {128, 1, vctas};
+    c->p_v_f1 = {256, 1, vctas};
+    c->p_v_f2 = {128, 1, vctas};
+    c->p_v_in = {128, 1, vctas};
+    c->p_v_out = {64, 1, vctas};
     const int bn_a = d.Ma <= 32 ? 32 : (d.Ma <= 64 ? 64 : (d.Ma <= 128 ? 128 : 256));
-    c->p_a_in = plan_swap(d.da, d.Ma, d.Kin, bn_a);
-    c->p_a_qkv = plan_swap(3 * d.A, d.Ma, d.da, bn_a);
-    c->p_a_o = plan_swap(d.da, d.Ma, d.A, bn_a);
-    c->p_a_f1 = plan_swap(d.Fa, d.Ma, d.da, bn_a);
-    c->p_a_f2 = plan_swap(d.da, d.Ma, d.Fa, bn_a);
-    c->p_a_out = plan_swap(d.Pa, d.Ma, d.da, bn_a);
+    // Opt-in (WAM_FUSE_NORM=1): every CTA of the fused GEMM re-reads all of
+    // x_a for the row norms, and on the config-2/3 chunks that measured slower
+    // under CEWP (4.45 / 21.5 ms) than the separate norm kernel (4.38 / 20.4).
+    const char* fv = getenv("WAM_FUSE_NORM");
+    c->fuse_norm_a = fv && fv[0] == '1' && bn_a <= 64 && d.da <= 1024 && d.da % 64 == 0;
+    const bool fn = c->fuse_norm_a;
+    c->p_a_in = plan_swap(d.da, d.Ma, d.Kin, bn_a, false);
+    c->p_a_qkv = plan_swap(3 * d.A, d.Ma, d.da, bn_a, fn);
+    c->p_a_o = plan_swap(d.da, d.Ma, d.A, bn_a, false);
+    c->p_a_f1 = plan_swap(d.Fa, d.Ma, d.da, bn_a, fn);
+    c->p_a_f2 = plan_swap(d.da, d.Ma, d.Fa, bn_a, false);
+    c->p_a_out = plan_swap(d.Pa, d.Ma, d.da, bn_a, fn);
     // workspace and tickets of one launch: rows_a x rows_b output, reduction K
     auto need = [](const GemmPlan& p, int rows_a, int rows_b, int K, bool swap, size_t* w, int* t) {
       TcGemm g{};
@@ -1386,6 +1412,11 @@ wam_status wam_op_attention(int dtype, const void* q, const void* k, const void*
   }
   if (a.splits > 1) {
     if (Lq > 64) return WAM_ERR_INVALID_ARG;
+    static thread_local bool prepared = false;
+    if (!prepared) {
+      if (prepare_attention_bf16() != cudaSuccess) return WAM_ERR_CUDA;
+      prepared = true;
+    }
     static thread_local float* ws = nullptr;
     static thread_local int* tk = nullptr;
     static thread_local size_t cap = 0, tcap = 0;

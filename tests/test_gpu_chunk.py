@@ -48,6 +48,23 @@ def test_tiny_fp32_parity(S, mode, graph):
     check_parity(a0, inp, ref_a0, ref_veff, c.dtype)
 
 
+@pytest.mark.parametrize("batch", [1, 2])
+def test_fused_action_norm(monkeypatch, batch):
+    """Opt-in fused action norm (WAM_FUSE_NORM=1): the QKV / FFN-up / final
+    out-proj GEMMs normalise the token rows themselves (32- and 64-token
+    tiles); parity with the oracle, and CEWP == sequential bitwise."""
+    monkeypatch.setenv("WAM_FUSE_NORM", "1")
+    c = _mid().replace(batch=batch)
+    wam = W.Wam(c, seed=13)
+    inp = inputs(c, 13)
+    a0 = run_chunk(wam, inp, S=2, mode=W.CEWP, use_graph=True)
+    seq = run_chunk(wam, inp, S=2, mode=W.SEQUENTIAL, use_graph=False)
+    assert np.array_equal(a0, seq)
+    ref_a0, ref_veff = oracle_chunk(c, 13, inp, S=2)
+    check_parity(a0, inp, ref_a0, ref_veff, c.dtype)
+    wam.close()
+
+
 def test_mid_bf16_parity_and_kv_publish():
     c = _mid()
     wam = W.Wam(c, seed=11)
