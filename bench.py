@@ -53,6 +53,30 @@ def parse():
     return p.parse_args()
 
 
+GEMM_SOURCES = ["mot_dit_b200/csrc/gemm_tc.cu", "mot_dit_b200/csrc/common.cuh", "mot_dit_b200/csrc/kernels.h"]
+GEMM_PROFILE = "profiles/video_gemm_fastwam_config2.md"
+
+
+def profiled_traffic():
+    """DRAM bytes (read + write) per launch of the video GEMM class, from the
+    ncu capture summarised in the profile file, or None when the kernel
+    sources have changed since that capture."""
+    import hashlib
+    root = os.path.dirname(os.path.abspath(__file__))
+    try:
+        text = open(os.path.join(root, GEMM_PROFILE)).read()
+        h = hashlib.sha256()
+        for f in GEMM_SOURCES:
+            h.update(open(os.path.join(root, f), "rb").read())
+    except OSError:
+        return None
+    fields = dict(l.split(": ", 1) for l in text.splitlines() if l.startswith(("traffic_bytes_per_launch:",
+                                                                               "gemm_source_sha256:")))
+    if fields.get("gemm_source_sha256", "").strip() != h.hexdigest():
+        return None
+    return int(float(fields["traffic_bytes_per_launch"]))
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -320,6 +344,7 @@ def run_ours(args, rank, world, local_rank):
         return 0
 
     peaks = load_peaks()
+    traffic = profiled_traffic() if args.config == 2 else None
     w, counts, flops, bytes_ = work_model(c, S)
     gemm = ["video_qkv", "video_oproj", "video_ffn_up", "video_ffn_down"]
     g_flops = sum(w[k][0] * counts[k] for k in gemm)
@@ -354,7 +379,7 @@ def run_ours(args, rank, world, local_rank):
         "actions_per_s": round(1e3 * world * c.batch * c.l_action / ms_per_step, 1),
         "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMM, video expert (QKV/out/FFN)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_kind": f"{peaks['_kind']} bf16 sustained",
                      "launches_timed": g_launch, "method": "CUDA event-record nodes around each launch in a captured sequential chunk"},
         "chunk_roofline": {"ms": round(chunk_roof, 4), "t_tensor_ms": round(t_tc, 4), "t_hbm_ms": round(t_hbm, 4),
