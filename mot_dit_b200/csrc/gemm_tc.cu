@@ -74,9 +74,12 @@ struct TileCfg {
   // fused-norm B operand, resident: [k-block][BN rows][128 B], 128-byte swizzle
   static constexpr int kResB = kNB ? (kNormKMax / BK) * BN * 128 : 0;
   static constexpr int kTmemCols = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
+  // gate-residual: up to 128 columns the warp's whole 32 x BN residual block
+  // is prefetched; wider tiles stream it box by box through two buffers
+  static constexpr bool kResBoxes = EPI == kClassRes && BN > 128;
   static constexpr int kWarpStg = SWAP ? 0
                                        : (EPI == kClassStore ? 2 * kBox
-                                                             : (EPI == kClassRes ? 32 * BN * 4
+                                                             : (EPI == kClassRes ? (kResBoxes ? 2 * kBox : 32 * BN * 4)
                                                                                  : (EPI == kClassQkv ? 4 * kBox : 0)));
   static constexpr int kSwapStg = SWAP ? 32 * (BM + 1) * 4 : 0;  // swapped QKV staging [32 tokens][129]
   // the tile's bias slice (and gate or QK gains) in shared memory, normal orientation
@@ -84,11 +87,12 @@ struct TileCfg {
   static constexpr int kExtra = kResB + 4 * kWarpStg + kSwapStg + kVecBytes;
   static constexpr int kBarBytes = 256;
   static constexpr int kSmemMax = 232448;  // 227 KB per CTA
-  static constexpr int kFit = (kSmemMax - 1024 - kBarBytes - kExtra) / kStageBytes;
+  // no alignment slack: the dynamic shared memory of a kernel without static
+  // shared memory starts on a 1024-byte boundary (checked at run time)
+  static constexpr int kFit = (kSmemMax - kBarBytes - kExtra) / kStageBytes;
   static constexpr int kStages = kFit > 8 ? 8 : kFit;
-  static constexpr int kSmem = kStages * kStageBytes + kExtra + kBarBytes + 1024;
+  static constexpr int kSmem = kStages * kStageBytes + kExtra + kBarBytes;
   static_assert(kStages >= 3, "shared memory ring too shallow");
-  static_assert(EPI != kClassRes || BN <= 128, "residual staging holds at most 128 columns");
 };
 
 struct GemmK {
@@ -337,8 +341,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap map_o, const __grid_constant__ CUtensorMap map_o2,
                    const GemmK g, const EpiArgs e) {
   using C = TileCfg<BN, SWAP, EPI>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The 128-byte swizzle is a function of the address bits: every tile must
+  // start on a 1024-byte boundary.
+  if (smem_u32(smem_raw) & 1023) {
+    if (threadIdx.x == 0) atomicOr(g.status, kStatusTimeoutDrain);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kStages * C::kABytes;
   uint8_t* sBres = smem + C::kStages * C::kStageBytes;  // fused-norm B operand (1024-byte aligned)
@@ -605,7 +615,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (!SWAP && (EPI == kClassRes || EPI == kClassQkv)) {
         if (lane == 0) bulk_wait_read<0>();  // earlier stores have left the staging
         __syncwarp();
-        if constexpr (EPI == kClassRes) {
+        if constexpr (C::kResBoxes) {
+          // residual boxes 0 and 1 (columns [0, 64)); later boxes stream in
+          // during the epilogue
+          for (int k = lane; k < 32 * 16; k += 32) {
+            const int r = k >> 4, q4 = k & 15;
+            const int m = m0w + r, n = nb + 4 * q4;
+            const bool v = m < g.rows_a && n < g.rows_b;
+            cp_async16(smem_u32(box_chunk(stg + (q4 >> 3) * kBox, r, q4 & 7)),
+                       v ? (const void*)(R.out_f32 + (size_t)m * R.ld + n) : (const void*)R.out_f32, v);
+          }
+        } else if constexpr (EPI == kClassRes) {
           // residual rows; box b holds columns [32 b, 32 b + 32) in the store layout
           for (int k = lane; k < 32 * (BN / 4); k += 32) {
             const int r = k / (BN / 4), q4 = k % (BN / 4);
@@ -802,11 +822,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++nbox;
           }
         } else if constexpr (EPI == kClassRes) {
+          const int nvb = min(BN, g.rows_b - nb) / 32;  // boxes with valid columns
+          // box bi's residual rows into buffer bi & 1 (one cp.async group)
+          auto load_box = [&](int bi) {
+            uint8_t* dst = stg + (bi & 1) * kBox;
+            for (int k = lane; k < 32 * 8; k += 32) {
+              const int r = k >> 3, q = k & 7;
+              const int m = m0w + r, n = nb + 32 * bi + 4 * q;
+              const bool v = m < g.rows_a;
+              cp_async16(smem_u32(box_chunk(dst, r, q)),
+                         v ? (const void*)(R.out_f32 + (size_t)m * R.ld + n) : (const void*)R.out_f32, v);
+            }
+            cp_async_commit();
+          };
           for (int c = 0; c < BN; c += 32) {
+            const int bi = c >> 5;
             float v[32];
             get(c, v);
             if (!warp_rows || nb + c >= g.rows_b) continue;
-            uint8_t* box = stg + (c >> 5) * kBox;  // the prefetched residual of these columns
+            if constexpr (C::kResBoxes) {
+              if (bi >= 2) {  // loaded at the end of iteration bi - 2; bi + 1 may be in flight
+                if (bi + 1 < nvb)
+                  cp_async_wait<1>();
+                else
+                  cp_async_wait<0>();
+                __syncwarp();
+              }
+            }
+            uint8_t* box = stg + (C::kResBoxes ? (bi & 1) : bi) * kBox;  // the residual of these columns
             const float4* b4 = reinterpret_cast<const float4*>(sVec + c);
             const float4* g4 = reinterpret_cast<const float4*>(sVec + BN + c);
 #pragma unroll
@@ -824,6 +867,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) {
               tma_store_3d(&map_o, box, nb + c, m0w, 0);
               bulk_commit();
+            }
+            if constexpr (C::kResBoxes) {
+              if (bi + 2 < nvb) {  // the buffer is free once this store has read it
+                if (lane == 0) bulk_wait_read<0>();
+                __syncwarp();
+                load_box(bi + 2);
+              }
             }
           }
         } else if constexpr (EPI == kClassQkv) {
@@ -1038,12 +1088,8 @@ cudaError_t launch_normal(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
       if (!e.map_o) return cudaErrorInvalidValue;
       return launch_one<BN, false, kClassStore>(t, e, s);
     case kEpiGateRes:
-      if constexpr (BN <= 128) {
-        if (!e.map_o) return cudaErrorInvalidValue;
-        return launch_one<BN, false, kClassRes>(t, e, s);
-      } else {
-        return cudaErrorInvalidValue;
-      }
+      if (!e.map_o) return cudaErrorInvalidValue;
+      return launch_one<BN, false, kClassRes>(t, e, s);
     case kEpiQkv:
       if (!e.map_o || !e.map_o2) return cudaErrorInvalidValue;
       return launch_one<BN, false, kClassQkv>(t, e, s);
@@ -1101,6 +1147,7 @@ cudaError_t prepare_tc_gemm() {
   WAM_PREP(256, false, kClassScalar)
   WAM_PREP(256, false, kClassStore)
   WAM_PREP(256, false, kClassQkv)
+  WAM_PREP(256, false, kClassRes)
 #undef WAM_PREP
   return cudaSuccess;
 }

@@ -889,12 +889,13 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   int tiles = 1, tiles_v = 1;
   if (d.bf16) {
     // Video GEMMs (tokens on TMEM lanes): stream-K over a persistent grid, so
-    // every CTA gets the same share of k-blocks whatever the tile count.  The
-    // wide projections (QKV, FFN-up) take 256-feature tiles (half the operand
-    // traffic per flop of 128); out-proj / FFN-down keep 128, their
-    // gate-residual epilogue staging the residual rows (measured: a 256-wide
-    // plain store with the residual folded into the next norm was slower
-    // overall).  The video GEMMs leave about a quarter of
+    // every CTA gets the same share of k-blocks whatever the tile count.  QKV
+    // and FFN-up take 256-feature tiles (half the operand traffic per flop of
+    // 128).  Out-proj / FFN-down (d-wide outputs, gate-residual epilogue) take
+    // 256 only when that still leaves two tiles per CTA: with fewer, the
+    // split-tile reduction and the last tile's residual epilogue cost more
+    // than the faster MMA saves (1088 tokens: 18.9 -> 27.4 us out-proj).  The
+    // video GEMMs leave about a quarter of
     // the SMs to the action stream that runs beside them under CEWP (108 of
     // 148 measured best on the config-2 chunk; WAM_VIDEO_GEMM_CTAS overrides
     // the count).  The grid is the same in every schedule: the k-range
@@ -907,9 +908,10 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
       if (n > 0) vctas = std::min(n, nsm);
     }
     c->p_v_qkv = {256, 1, vctas};
-    c->p_v_o = {128, 1, vctas};
+    const int bn_res = ((d.Mv + 127) / 128) * (d.dv / 256) >= 2 * vctas ? 256 : 128;
+    c->p_v_o = {bn_res, 1, vctas};
     c->p_v_f1 = {256, 1, vctas};
-    c->p_v_f2 = {128, 1, vctas};
+    c->p_v_f2 = {bn_res, 1, vctas};
     c->p_v_in = {128, 1, vctas};
     c->p_v_out = {64, 1, vctas};
     const int bn_a = d.Ma <= 32 ? 32 : (d.Ma <= 64 ? 64 : (d.Ma <= 128 ? 128 : 256));
