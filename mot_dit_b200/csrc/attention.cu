@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(kAttnThreads)
     attn_bf16_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
                      const __nv_bfloat16* __restrict__ vc, __nv_bfloat16* __restrict__ out, int H, int Lq,
                      int Lk, int Lcache, int splits, int keys_per_split, float* __restrict__ ws,
-                     int* __restrict__ tickets, int rows_per_pass) {
+                     int* __restrict__ tickets, int rows_per_pass, int ldo) {
   __shared__ __align__(128) uint8_t smem[kTQ * 128 + 2 * 2 * kTK * 128];
   extern __shared__ float4 s_comb[];  // split path: [splits][rows_per_pass][16] partial O rows
   __shared__ int s_last;
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kAttnThreads)
     l += __shfl_xor_sync(0xffffffffu, l, 2);
     l_tot[r] = l;
   }
-  const int A = H * kD;
+  const int A = ldo;  // row stride of out
   if (!SPLIT) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(kAttnThreads)
 template <int D>
 __global__ void attn_f32_kernel(const float* __restrict__ q, const float* __restrict__ kc,
                                 const float* __restrict__ vc, float* __restrict__ out, int H, int Lq, int Lk,
-                                int Lcache, int total) {
+                                int Lcache, int total, int ldo) {
   const int warp_global = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (warp_global >= total) return;  // uniform per warp
   const int lane = threadIdx.x & 31;
@@ -326,8 +326,7 @@ __global__ void attn_f32_kernel(const float* __restrict__ q, const float* __rest
   l *= f;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-  const int A = H * D;
-  float* dst = out + (size_t)(b * Lq + qi) * A + h * D;
+  float* dst = out + (size_t)(b * Lq + qi) * ldo + h * D;
 #pragma unroll
   for (int d = 0; d < D; ++d) {
     float v = acc[d] * f;
@@ -351,6 +350,8 @@ cudaError_t prepare_attention_bf16() {
 
 cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s) {
   if (a.Dh != kD) return cudaErrorInvalidValue;
+  const int ldo = a.ld_out ? a.ld_out : a.H * kD;
+  if (ldo < a.H * kD || ldo % 4) return cudaErrorInvalidValue;
   const int splits = a.splits < 1 ? 1 : a.splits;
   if (splits > 1 && a.Lq > kTQ) return cudaErrorInvalidValue;
   int kps = (a.Lk + splits - 1) / splits;
@@ -365,13 +366,15 @@ cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s) {
   if (used > 1) {
     const int rpp = std::max(1, std::min(a.Lq, kCombineBytes / (used * kD * 4)));
     return launch_k(attn_bf16_kernel<true>, grid, dim3(kAttnThreads), (size_t)used * rpp * kD * 4, s, q, k, v, o,
-                    a.H, a.Lq, a.Lk, a.Lcache, used, kps, a.ws, a.tickets, rpp);
+                    a.H, a.Lq, a.Lk, a.Lcache, used, kps, a.ws, a.tickets, rpp, ldo);
   }
   return launch_k(attn_bf16_kernel<false>, grid, dim3(kAttnThreads), 0, s, q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache, 1,
-                  kps, (float*)nullptr, (int*)nullptr, 0);
+                  kps, (float*)nullptr, (int*)nullptr, 0, ldo);
 }
 
 cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t s) {
+  const int ldo = a.ld_out ? a.ld_out : a.H * a.Dh;
+  if (ldo < a.H * a.Dh) return cudaErrorInvalidValue;
   const int warps = a.B * a.H * a.Lq;
   const int per_block = 4;
   dim3 grid((warps + per_block - 1) / per_block);
@@ -380,9 +383,9 @@ cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t s) {
   const auto* v = reinterpret_cast<const float*>(a.v);
   auto* o = reinterpret_cast<float*>(a.out);
   switch (a.Dh) {
-    case 16: attn_f32_kernel<16><<<grid, 32 * per_block, 0, s>>>(q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache, warps); break;
-    case 32: attn_f32_kernel<32><<<grid, 32 * per_block, 0, s>>>(q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache, warps); break;
-    case 64: attn_f32_kernel<64><<<grid, 32 * per_block, 0, s>>>(q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache, warps); break;
+    case 16: attn_f32_kernel<16><<<grid, 32 * per_block, 0, s>>>(q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache, warps, ldo); break;
+    case 32: attn_f32_kernel<32><<<grid, 32 * per_block, 0, s>>>(q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache, warps, ldo); break;
+    case 64: attn_f32_kernel<64><<<grid, 32 * per_block, 0, s>>>(q, k, v, o, a.H, a.Lq, a.Lk, a.Lcache, warps, ldo); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

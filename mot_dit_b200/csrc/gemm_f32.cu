@@ -23,6 +23,9 @@ __device__ __forceinline__ void epi_elem_f32(const EpiArgs& e, int m, int n, flo
     case kEpiGelu:
       reinterpret_cast<float*>(e.out_act)[idx] = gelu_tanh(y);
       break;
+    case kEpiScaleAct:
+      reinterpret_cast<float*>(e.out_act)[idx] = e.scale * y;
+      break;
     case kEpiEuler: {
       const float dt = e.aio->sched[e.step] - e.aio->sched[e.step + 1];
       e.out_f32[idx] -= dt * y;
@@ -41,8 +44,9 @@ __device__ __forceinline__ void epi_elem_f32(const EpiArgs& e, int m, int n, flo
   }
 }
 
-__global__ void __launch_bounds__(256) f32_gemm_kernel(const float* __restrict__ X, const float* __restrict__ W,
-                                                       int M, int N, int K, const EpiArgs e) {
+__global__ void __launch_bounds__(256) f32_gemm_kernel(const float* __restrict__ X, int ldx,
+                                                       const float* __restrict__ W, int M, int N, int K,
+                                                       const EpiArgs e) {
   __shared__ float sX[TK][T + 4];
   __shared__ float sW[TK][T + 4];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -52,7 +56,7 @@ __global__ void __launch_bounds__(256) f32_gemm_kernel(const float* __restrict__
     for (int i = threadIdx.x; i < T * TK; i += 256) {
       const int r = i / TK, c = i % TK;
       const int m = m0 + r, n = n0 + r, k = k0 + c;
-      sX[c][r] = (m < M && k < K) ? X[(size_t)m * K + k] : 0.f;
+      sX[c][r] = (m < M && k < K) ? X[(size_t)m * ldx + k] : 0.f;
       sW[c][r] = (n < N && k < K) ? W[(size_t)n * K + k] : 0.f;
     }
     __syncthreads();
@@ -116,10 +120,10 @@ __global__ void qkv_post_f32_kernel(const float* __restrict__ qkv, int M, const 
 
 }  // namespace
 
-cudaError_t launch_f32_gemm(const float* X, const float* W, int M, int N, int K, const EpiArgs& e,
+cudaError_t launch_f32_gemm(const float* X, int ldx, const float* W, int M, int N, int K, const EpiArgs& e,
                             cudaStream_t s) {
   dim3 grid((N + T - 1) / T, (M + T - 1) / T);
-  f32_gemm_kernel<<<grid, 256, 0, s>>>(X, W, M, N, K, e);
+  f32_gemm_kernel<<<grid, 256, 0, s>>>(X, ldx, W, M, N, K, e);
   return cudaGetLastError();
 }
 

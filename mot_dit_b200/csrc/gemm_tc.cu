@@ -301,6 +301,9 @@ __device__ __forceinline__ void epi_elem(const EpiArgs& e, int m, int n, float y
     case kEpiGelu:
       reinterpret_cast<__nv_bfloat16*>(e.out_act)[idx] = __float2bfloat16_rn(gelu_tanh(y));
       break;
+    case kEpiScaleAct:
+      reinterpret_cast<__nv_bfloat16*>(e.out_act)[idx] = __float2bfloat16_rn(e.scale * y);
+      break;
     case kEpiEuler: {
       const float dt = e.aio->sched[e.step] - e.aio->sched[e.step + 1];
       const float a = e.out_f32[idx] - dt * y;
@@ -994,6 +997,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j) {
               const int m = mb + c + j;
               if (m < g.rows_b) R.out_act[(size_t)m * R.ld + n] = __float2bfloat16_rn(gelu_tanh(v[j] + bias));
+            }
+          } else if (n_ok && R.kind == kEpiScaleAct) {
+            const float sc = e.scale;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int m = mb + c + j;
+              if (m < g.rows_b) R.out_act[(size_t)m * R.ld + n] = __float2bfloat16_rn(sc * (v[j] + bias));
             }
           } else if (n_ok) {
 #pragma unroll

@@ -61,10 +61,12 @@ enum Epi : int {
   kEpiQkv = 3,       // bias, per-head QK-RMSNorm with gains, RoPE, scatter to Q and the KV cache
   kEpiEuler = 4,     // a[m, n] -= (t_j - t_{j-1}) * (acc + bias[n]); also writes the next in-proj input
   kEpiVideoOut = 5,  // joint variant: video endpoint f^v = c_skip x + c_out (x - sigma v)
+  kEpiScaleAct = 6,  // out_act[m, n] = scale * (acc + bias[n]) (act dtype): the LoRA down-projection s x A^T
 };
 
 struct EpiArgs {
   int kind = 0;
+  float scale = 1.f;  // kEpiScaleAct
   const float* bias = nullptr;
   const float* gate = nullptr;
   float* out_f32 = nullptr;
@@ -132,16 +134,18 @@ cudaError_t launch_tc_gemm(const TcGemm& g, const EpiArgs& e, cudaStream_t s);
 // launch (and never during stream capture).
 cudaError_t prepare_tc_gemm();
 
-// fp32 SIMT GEMM (debug precision): C = X W^T + epilogue; X [M, K] (ld = K), W [N, K].
-cudaError_t launch_f32_gemm(const float* X, const float* W, int M, int N, int K, const EpiArgs& e,
+// fp32 SIMT GEMM (debug precision): C = X W^T + epilogue; X [M, K] with row
+// stride ldx, W [N, K] (row stride K).
+cudaError_t launch_f32_gemm(const float* X, int ldx, const float* W, int M, int N, int K, const EpiArgs& e,
                             cudaStream_t s);
 
 // fp32 path: per-head QK-RMSNorm + RoPE + scatter of a raw projection [M, 3A].
 cudaError_t launch_qkv_post_f32(const float* qkv, int M, const EpiArgs& e, cudaStream_t s);
 
-// h[m, :] = rms(x[m, :]) * (gain ? gain : 1 + scale) + (shift ? shift : 0)
+// h[m, :] = rms(x[m, :]) * (gain ? gain : 1 + scale) + (shift ? shift : 0);
+// h rows ldh apart (0: d).
 cudaError_t launch_norm_mod(const float* x, void* h, bool h_bf16, int M, int d, const float* scale,
-                            const float* shift, const float* gain, cudaStream_t s);
+                            const float* shift, const float* gain, cudaStream_t s, int ldh = 0);
 
 // Timestep conditioning of one expert: tau(t) -> c -> m, then mod[i] = m + T_i
 // for every block.  t = io_t[0] (device scalar); weights in `bf16` or fp32.
@@ -165,6 +169,7 @@ struct AttnArgs {
   const void* q; const void* k; const void* v; void* out;
   int B, H, Dh, Lq, Lk, Lcache;
   int splits;        // key splits (1 = single pass)
+  int ld_out = 0;    // row stride of out (0: H * Dh)
   float* ws;         // partial O / m / l when splits > 1
   int* tickets;      // B*H counters, zero on entry, left zero
 };

@@ -26,7 +26,7 @@ constexpr int kNormV = 12;
 template <bool BF16>
 __global__ void __launch_bounds__(32 * kNormWarps)
     norm_mod_kernel(const float* __restrict__ x, void* __restrict__ h, int M, int d, const float* __restrict__ scale,
-                    const float* __restrict__ shift, const float* __restrict__ gain) {
+                    const float* __restrict__ shift, const float* __restrict__ gain, int ldh) {
   pdl_trigger();
   pdl_wait();
   const int row = blockIdx.x * kNormWarps + (threadIdx.x >> 5);
@@ -70,9 +70,9 @@ __global__ void __launch_bounds__(32 * kNormWarps)
       uint2 p;
       p.x = pack_bf16(y[0], y[1]);
       p.y = pack_bf16(y[2], y[3]);
-      reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(h) + (size_t)row * d)[i] = p;
+      reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(h) + (size_t)row * ldh)[i] = p;
     } else {
-      reinterpret_cast<float4*>(reinterpret_cast<float*>(h) + (size_t)row * d)[i] = make_float4(y[0], y[1], y[2], y[3]);
+      reinterpret_cast<float4*>(reinterpret_cast<float*>(h) + (size_t)row * ldh)[i] = make_float4(y[0], y[1], y[2], y[3]);
     }
   }
 }
@@ -280,11 +280,14 @@ int grid_for(size_t n, int threads) {
 }  // namespace
 
 cudaError_t launch_norm_mod(const float* x, void* h, bool h_bf16, int M, int d, const float* scale,
-                            const float* shift, const float* gain, cudaStream_t s) {
+                            const float* shift, const float* gain, cudaStream_t s, int ldh) {
+  if (ldh == 0) ldh = d;
+  if (ldh < d || ldh % 4) return cudaErrorInvalidValue;
   if (d % 4 != 0 || d > 32 * 4 * kNormV) return cudaErrorInvalidValue;
   dim3 grid((M + kNormWarps - 1) / kNormWarps);
-  if (h_bf16) return launch_k(norm_mod_kernel<true>, grid, dim3(32 * kNormWarps), 0, s, x, h, M, d, scale, shift, gain);
-  return launch_k(norm_mod_kernel<false>, grid, dim3(32 * kNormWarps), 0, s, x, h, M, d, scale, shift, gain);
+  if (h_bf16)
+    return launch_k(norm_mod_kernel<true>, grid, dim3(32 * kNormWarps), 0, s, x, h, M, d, scale, shift, gain, ldh);
+  return launch_k(norm_mod_kernel<false>, grid, dim3(32 * kNormWarps), 0, s, x, h, M, d, scale, shift, gain, ldh);
 }
 
 cudaError_t launch_temb(const TembArgs& a, cudaStream_t s) {

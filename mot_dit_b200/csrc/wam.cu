@@ -32,6 +32,9 @@ struct PEntry {
   int rows, cols, ld;
   bool matrix, ones;
   size_t off;  // elements into wmat (matrix) or wvec (vector)
+  // LoRA B factors live inside their layer's weight matrix: columns
+  // [col_off, col_off + cols) of matrix `alias` (same ld), see add_expert
+  int alias = -1, col_off = 0;
   size_t count() const { return (size_t)rows * cols; }
 };
 
@@ -49,6 +52,9 @@ struct ExpertIdx {
 
 struct Dims {
   int N, dv, da, H, Dh, A, Fv, Fa, Lc, Lvid, Lv, La, Pa, Pv, B, r, Ltot, Mv, Ma, Kin;
+  // row strides of the action GEMM inputs h_a, o_a, f_a: each row carries the
+  // layer input and, with LoRA, the r columns of s x A^T after it
+  int lh, lo, lf;
   bool bf16;
 };
 
@@ -77,6 +83,7 @@ struct wam_ctx {
   void* kv = nullptr;                                 // [N][2][B][H][Ltot][Dh]
   float *mod_v = nullptr, *mod_a = nullptr, *temb_v = nullptr, *temb_a = nullptr;
   float *rope_cos = nullptr, *rope_sin = nullptr;
+  float* zero_r = nullptr;   // r zeros: the (absent) bias of the LoRA down-projection
   float* ws_gemm = nullptr;  // action-stream GEMM partial tiles / tickets
   int* tk_gemm = nullptr;
   float* ws_gemm_v = nullptr;  // video-stream GEMM partial tiles / tickets (the streams overlap)
@@ -95,6 +102,7 @@ struct wam_ctx {
   // plans
   GemmPlan p_v_qkv, p_v_o, p_v_f1, p_v_f2, p_v_in, p_v_out;
   GemmPlan p_a_in, p_a_qkv, p_a_o, p_a_f1, p_a_f2, p_a_out;
+  GemmPlan p_u_qkv, p_u_o, p_u_f1, p_u_f2;  // LoRA down-projections u = s x A^T
   int attn_splits = 1;
   // The action expert's norms run inside the GEMM that consumes them (opt-in;
   // the tokens must fit one 32/64-wide tile and K <= 1024).
@@ -103,6 +111,7 @@ struct wam_ctx {
   // TMA maps
   CUtensorMap m_hv, m_ov, m_fv, m_xvin, m_w_qkv_v, m_w_o_v, m_w_f1_v, m_w_f2_v, m_w_vin, m_w_vout;
   CUtensorMap m_w_in, m_w_qkv_a, m_w_o_a, m_w_f1_a, m_w_f2_a, m_w_out, m_ain, m_ha, m_oa, m_fa;
+  CUtensorMap m_la_qkv, m_la_o, m_la_f1, m_la_f2;  // LoRA A factors [r, in] per block
   CUtensorMap m_qv, m_cache;  // video-attention operands
   // video GEMM outputs (TMA stores, 32-row boxes): x_v fp32, f_v bf16, Q, the K/V cache
   CUtensorMap m_xv_out, m_fv_out, m_qv_out, m_cache_out;
@@ -210,25 +219,36 @@ void add_expert(wam_ctx* c, bool video) {
     const std::string b = p + "blk" + std::to_string(i) + ".";
     const int first = add(b + "T", 6, dm, false, false);
     if (i == 0) ix.blk0 = first;
-    add(b + "qkv.w", 3 * A, dm, true, false);
+    const int wq = add(b + "qkv.w", 3 * A, dm, true, false);
     add(b + "qkv.b", 1, 3 * A, false, false);
     add(b + "qn.g", 1, A, false, true);
     add(b + "kn.g", 1, A, false, true);
-    add(b + "o.w", dm, A, true, false);
+    const int wo = add(b + "o.w", dm, A, true, false);
     add(b + "o.b", 1, dm, false, false);
-    add(b + "ffn1.w", F, dm, true, false);
+    const int w1 = add(b + "ffn1.w", F, dm, true, false);
     add(b + "ffn1.b", 1, F, false, false);
-    add(b + "ffn2.w", dm, F, true, false);
+    const int w2 = add(b + "ffn2.w", dm, F, true, false);
     add(b + "ffn2.b", 1, dm, false, false);
     if (lora) {
+      // Unmerged LoRA y = x W^T + b + s (x A^T) B^T as one GEMM over the
+      // concatenated reduction [x | s x A^T] . [W | B]^T: B sits in columns
+      // [K, K + r) of W's rows (W's leading dimension grows by r).
+      auto lb = [&](const std::string& n, int w) {
+        const int k = c->params[w].ld, rows = c->params[w].rows;
+        c->params[w].ld = k + d.r;
+        const int e = add(n, rows, d.r, true, false);  // (may reallocate the table)
+        c->params[e].ld = k + d.r;
+        c->params[e].alias = w;
+        c->params[e].col_off = k;
+      };
       add(b + "qkv.la", d.r, dm, true, false);
-      add(b + "qkv.lb", 3 * A, d.r, true, false);
+      lb(b + "qkv.lb", wq);
       add(b + "o.la", d.r, A, true, false);
-      add(b + "o.lb", dm, d.r, true, false);
+      lb(b + "o.lb", wo);
       add(b + "ffn1.la", d.r, dm, true, false);
-      add(b + "ffn1.lb", F, d.r, true, false);
+      lb(b + "ffn1.lb", w1);
       add(b + "ffn2.la", d.r, F, true, false);
-      add(b + "ffn2.lb", dm, d.r, true, false);
+      lb(b + "ffn2.lb", w2);
     }
     if (i == 0) ix.per_blk = (int)c->params.size() - first;
   }
@@ -247,7 +267,9 @@ void add_expert(wam_ctx* c, bool video) {
 void layout_params(wam_ctx* c) {
   size_t om = 0, ov = 0;
   for (auto& e : c->params) {
-    if (e.matrix) {
+    if (e.matrix && e.alias >= 0) {
+      e.off = c->params[e.alias].off + e.col_off;
+    } else if (e.matrix) {
       e.off = om;
       om += ((size_t)e.rows * e.ld + 127) / 128 * 128;
     } else {
@@ -274,6 +296,12 @@ inline void* vcache(wam_ctx* c, int i) {
   const size_t per = (size_t)c->d.B * c->d.H * c->d.Ltot * c->d.Dh;
   return (char*)c->kv + (size_t)(2 * i + 1) * per * c->esz;
 }
+
+#define RET(expr)                       \
+  do {                                  \
+    wam_status r_ = (expr);             \
+    if (r_ != WAM_OK) return r_;        \
+  } while (0)
 
 // ------------------------------------------------------------- planning ---
 GemmPlan plan_swap(int rows_w, int tokens, int K, int bn, bool fused_norm) {
@@ -352,15 +380,35 @@ struct Lin {
   const CUtensorMap* map_w;  // weight map (bf16)
   const CUtensorMap* map_x;  // activation map (bf16)
   const void* w;             // fp32 path: weight pointer
-  const void* x;             // fp32 path: activation pointer
+  const void* x;             // activation pointer (rows ldx apart; 0: K)
   int n_out, K;              // output features, reduction length
   int z;                     // block index in the weight map
   const GemmPlan* plan;
+  int ldx = 0;
+  // unmerged LoRA (action expert): the A factor [r, K] of this layer
+  const CUtensorMap* map_la = nullptr;
+  const void* la = nullptr;
+  const GemmPlan* plan_u = nullptr;
 };
 
 wam_status linear(wam_ctx* c, bool video, const Lin& L, int M, const EpiArgs& e_in, float* qkv_tmp, cudaStream_t s) {
   const Dims& d = c->d;
   ProfScope ps(c, s);
+  const int ldx = L.ldx ? L.ldx : L.K;
+  int K = L.K;
+  if (L.la) {
+    // LoRA: u = s x A^T into columns [K, K + r) of the input rows, then one
+    // GEMM over the concatenated reduction [x | u] . [W | B]^T
+    EpiArgs eu = epi_base(kEpiScaleAct, c->zero_r, nullptr, (char*)L.x + (size_t)L.K * c->esz, ldx);
+    eu.scale = c->cfg.lora_scale;
+    if (d.bf16) {
+      RET(run_tc(c, *L.map_la, *L.map_x, d.r, M, L.K, L.z, 0, *L.plan_u, true, eu, s, false));
+    } else {
+      c->launches++;
+      CK(launch_f32_gemm((const float*)L.x, ldx, (const float*)L.la, M, d.r, L.K, eu, s));
+    }
+    K += d.r;
+  }
   if (d.bf16) {
     if (video) {  // tokens on TMEM lanes; outputs leave through TMA stores
       EpiArgs e = e_in;
@@ -375,28 +423,28 @@ wam_status linear(wam_ctx* c, bool video, const Lin& L, int M, const EpiArgs& e_
       } else if (e.kind == kEpiStoreF32 || e.kind == kEpiGateRes) {
         e.map_o = &c->m_xv_out;
       }
-      return run_tc(c, *L.map_x, *L.map_w, M, L.n_out, L.K, 0, L.z, *L.plan, false, e, s, true);
+      return run_tc(c, *L.map_x, *L.map_w, M, L.n_out, K, 0, L.z, *L.plan, false, e, s, true);
     }
-    return run_tc(c, *L.map_w, *L.map_x, L.n_out, M, L.K, L.z, 0, *L.plan, true, e_in, s, false);
+    return run_tc(c, *L.map_w, *L.map_x, L.n_out, M, K, L.z, 0, *L.plan, true, e_in, s, false);
   }
   if (e_in.kind == kEpiQkv) {
     EpiArgs st = epi_base(kEpiStoreF32, e_in.bias, qkv_tmp, nullptr, 3 * d.A);
     c->launches++;
-    CK(launch_f32_gemm((const float*)L.x, (const float*)L.w, M, L.n_out, L.K, st, s));
+    CK(launch_f32_gemm((const float*)L.x, ldx, (const float*)L.w, M, L.n_out, K, st, s));
     c->launches++;
     CK(launch_qkv_post_f32(qkv_tmp, M, e_in, s));
     return WAM_OK;
   }
   c->launches++;
-  CK(launch_f32_gemm((const float*)L.x, (const float*)L.w, M, L.n_out, L.K, e_in, s));
+  CK(launch_f32_gemm((const float*)L.x, ldx, (const float*)L.w, M, L.n_out, K, e_in, s));
   return WAM_OK;
 }
 
 wam_status norm(wam_ctx* c, const float* x, void* h, int M, int dm, const float* sc, const float* sh, const float* g,
-                cudaStream_t s) {
+                cudaStream_t s, int ldh = 0) {
   c->launches++;
   ProfScope ps(c, s);
-  CK(launch_norm_mod(x, h, c->d.bf16, M, dm, sc, sh, g, s));
+  CK(launch_norm_mod(x, h, c->d.bf16, M, dm, sc, sh, g, s, ldh));
   return WAM_OK;
 }
 
@@ -443,6 +491,7 @@ wam_status attention(wam_ctx* c, bool video, int i, cudaStream_t s) {
   a.Lk = video ? d.Lv : d.Lv + d.La;
   a.Lcache = d.Ltot;
   a.splits = video ? 1 : c->attn_splits;
+  a.ld_out = video ? 0 : d.lo;
   a.ws = c->ws_attn;
   a.tickets = c->tk_attn;
   c->launches++;
@@ -468,12 +517,6 @@ wam_status attention(wam_ctx* c, bool video, int i, cudaStream_t s) {
   return WAM_OK;
 }
 
-#define RET(expr)                       \
-  do {                                  \
-    wam_status r_ = (expr);             \
-    if (r_ != WAM_OK) return r_;        \
-  } while (0)
-
 wam_status norm_linear(wam_ctx* c, const Lin& L, EpiArgs e, const float* sc, const float* sh, const float* gain,
                        int cls, cudaStream_t s) {
   const Dims& d = c->d;
@@ -484,7 +527,7 @@ wam_status norm_linear(wam_ctx* c, const Lin& L, EpiArgs e, const float* sc, con
     e.nb_gain = gain;
   } else {
     c->cur_cls = WAM_PROF_ACTION_NORM;
-    RET(norm(c, c->x_a, c->h_a, d.Ma, d.da, sc, sh, gain, s));
+    RET(norm(c, c->x_a, c->h_a, d.Ma, d.da, sc, sh, gain, s, d.lh));
   }
   c->cur_cls = cls;
   return linear(c, false, L, d.Ma, e, c->qkv_tmp_a, s);
@@ -551,6 +594,14 @@ wam_status enqueue_video(wam_ctx* c, cudaStream_t s, const VideoIo* io, bool joi
   return WAM_OK;
 }
 
+// Attach block i's LoRA A factor (action expert) to a linear layer.
+void lora(wam_ctx* c, Lin& L, int i, int local, const CUtensorMap* map, const GemmPlan* plan) {
+  if (c->d.r == 0) return;
+  L.map_la = map;
+  L.la = matp(c, blk(c->ea, i, local));
+  L.plan_u = plan;
+}
+
 // One Euler step j of the action expert: P^a_i -> wait(e_i) -> Attn^a_i -> R^a_i.
 wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, int j, const cudaEvent_t* ev_wait,
                                bool record_used) {
@@ -565,7 +616,8 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
   }
   for (int i = 0; i < d.N; ++i) {
     const float* mod = c->mod_a + (size_t)i * 6 * d.da;
-    Lin Lq{&c->m_w_qkv_a, &c->m_ha, matp(c, blk(x, i, kQkvW)), c->h_a, 3 * d.A, d.da, i, &c->p_a_qkv};
+    Lin Lq{&c->m_w_qkv_a, &c->m_ha, matp(c, blk(x, i, kQkvW)), c->h_a, 3 * d.A, d.da, i, &c->p_a_qkv, d.lh};
+    lora(c, Lq, i, kQkvLa, &c->m_la_qkv, &c->p_u_qkv);
     RET(norm_linear(c, Lq, epi_qkv(c, false, i), mod + d.da, mod, nullptr, WAM_PROF_ACTION_QKV, s));
     if (ev_wait) CK(cudaStreamWaitEvent(s, ev_wait[i], 0));
     c->cur_cls = WAM_PROF_ACTION_ATTN;
@@ -574,15 +626,18 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
     c->cur_cls = WAM_PROF_ACTION_OPROJ;
     EpiArgs eo = epi_base(kEpiGateRes, vecp(c, blk(x, i, kOB)), c->x_a, nullptr, d.da);
     eo.gate = mod + 2 * d.da;
-    Lin Lo{&c->m_w_o_a, &c->m_oa, matp(c, blk(x, i, kOW)), c->o_a, d.da, d.A, i, &c->p_a_o};
+    Lin Lo{&c->m_w_o_a, &c->m_oa, matp(c, blk(x, i, kOW)), c->o_a, d.da, d.A, i, &c->p_a_o, d.lo};
+    lora(c, Lo, i, kOLa, &c->m_la_o, &c->p_u_o);
     RET(linear(c, false, Lo, d.Ma, eo, nullptr, s));
-    Lin L1{&c->m_w_f1_a, &c->m_ha, matp(c, blk(x, i, kF1W)), c->h_a, d.Fa, d.da, i, &c->p_a_f1};
-    RET(norm_linear(c, L1, epi_base(kEpiGelu, vecp(c, blk(x, i, kF1B)), nullptr, c->f_a, d.Fa), mod + 4 * d.da,
+    Lin L1{&c->m_w_f1_a, &c->m_ha, matp(c, blk(x, i, kF1W)), c->h_a, d.Fa, d.da, i, &c->p_a_f1, d.lh};
+    lora(c, L1, i, kF1La, &c->m_la_f1, &c->p_u_f1);
+    RET(norm_linear(c, L1, epi_base(kEpiGelu, vecp(c, blk(x, i, kF1B)), nullptr, c->f_a, d.lf), mod + 4 * d.da,
                     mod + 3 * d.da, nullptr, WAM_PROF_ACTION_FFN_UP, s));
     c->cur_cls = WAM_PROF_ACTION_FFN_DOWN;
     EpiArgs e2 = epi_base(kEpiGateRes, vecp(c, blk(x, i, kF2B)), c->x_a, nullptr, d.da);
     e2.gate = mod + 5 * d.da;
-    Lin L2{&c->m_w_f2_a, &c->m_fa, matp(c, blk(x, i, kF2W)), c->f_a, d.da, d.Fa, i, &c->p_a_f2};
+    Lin L2{&c->m_w_f2_a, &c->m_fa, matp(c, blk(x, i, kF2W)), c->f_a, d.da, d.Fa, i, &c->p_a_f2, d.lf};
+    lora(c, L2, i, kF2La, &c->m_la_f2, &c->p_u_f2);
     RET(linear(c, false, L2, d.Ma, e2, nullptr, s));
   }
   EpiArgs ee = epi_base(kEpiEuler, vecp(c, x.outb), c->a_state, nullptr, d.Pa);
@@ -590,7 +645,7 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
   ee.step = j;
   ee.a_next = d.bf16 ? c->a_in : nullptr;
   ee.a_next_ld = d.Kin;
-  Lin Lout{&c->m_w_out, &c->m_ha, matp(c, x.outw), c->h_a, d.Pa, d.da, 0, &c->p_a_out};
+  Lin Lout{&c->m_w_out, &c->m_ha, matp(c, x.outw), c->h_a, d.Pa, d.da, 0, &c->p_a_out, d.lh};
   RET(norm_linear(c, Lout, ee, nullptr, nullptr, vecp(c, x.fng), WAM_PROF_ACTION_IO, s));
   return WAM_OK;
 }
@@ -807,7 +862,7 @@ void wam_destroy(wam_ctx* c) {
   if (c->cap_a) cudaStreamDestroy(c->cap_a);
   void* bufs[] = {c->wmat, c->wvec, c->x_v, c->x_a, c->a_state, c->x_sigma, c->h_v, c->q_v, c->o_v, c->f_v,
                   c->x_vin, c->h_a, c->q_a, c->o_a, c->f_a, c->a_in, c->qkv_tmp_v, c->qkv_tmp_a, c->kv,
-                  c->mod_v, c->mod_a, c->temb_v, c->temb_a, c->rope_cos, c->rope_sin, c->ws_gemm, c->tk_gemm, c->ws_gemm_v, c->tk_gemm_v,
+                  c->mod_v, c->mod_a, c->temb_v, c->temb_a, c->rope_cos, c->rope_sin, c->ws_gemm, c->tk_gemm, c->ws_gemm_v, c->tk_gemm_v, c->zero_r,
                   c->ws_attn, c->tk_attn, c->status, c->vio_chunk, c->vio_eager, c->aio_chunk, c->aio_eager,
                   c->h_video, c->h_cond, c->h_noise, c->h_out, c->j_vout, c->j_aout};
   for (void* p : bufs)
@@ -819,7 +874,6 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   if (!cfg || !out) return WAM_ERR_INVALID_ARG;
   std::string why;
   if (!check_cfg(cfg, &why)) return WAM_ERR_INVALID_ARG;
-  if (cfg->lora_rank > 0 && cfg->dtype == WAM_BF16) return WAM_ERR_UNSUPPORTED;
   std::unique_ptr<wam_ctx> holder(new wam_ctx());
   wam_ctx* c = holder.get();
   c->cfg = *cfg;
@@ -834,6 +888,9 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   d.B = cfg->batch; d.r = cfg->lora_rank; d.Ltot = d.Lv + d.La; d.Mv = d.B * d.Lv; d.Ma = d.B * d.La;
   d.bf16 = cfg->dtype == WAM_BF16;
   d.Kin = d.bf16 ? (d.Pa + 63) / 64 * 64 : d.Pa;
+  d.lh = d.da + d.r;
+  d.lo = d.A + d.r;
+  d.lf = d.Fa + d.r;
   c->esz = d.bf16 ? 2 : 4;
 
   add_expert(c, true);
@@ -856,10 +913,11 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   RET(dalloc(c, &c->o_v, (size_t)d.Mv * d.A * ae));
   RET(dalloc(c, &c->f_v, (size_t)d.Mv * d.Fv * ae));
   RET(dalloc(c, &c->x_a, (size_t)d.Ma * d.da * 4));
-  RET(dalloc(c, &c->h_a, (size_t)d.Ma * d.da * ae));
+  RET(dalloc(c, &c->h_a, (size_t)d.Ma * d.lh * ae));
   RET(dalloc(c, &c->q_a, (size_t)d.Ma * d.A * ae));
-  RET(dalloc(c, &c->o_a, (size_t)d.Ma * d.A * ae));
-  RET(dalloc(c, &c->f_a, (size_t)d.Ma * d.Fa * ae));
+  RET(dalloc(c, &c->o_a, (size_t)d.Ma * d.lo * ae));
+  RET(dalloc(c, &c->f_a, (size_t)d.Ma * d.lf * ae));
+  RET(dalloc(c, &c->zero_r, (size_t)std::max(d.r, 1) * 4));
   RET(dalloc(c, &c->a_state, (size_t)d.Ma * d.Pa * 4));
   RET(dalloc(c, &c->a_in, (size_t)d.Ma * d.Kin * ae));
   if (d.Pv > 0) {
@@ -919,13 +977,19 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     // x_a for the row norms, and on the config-2/3 chunks that measured slower
     // under CEWP (4.45 / 21.5 ms) than the separate norm kernel (4.38 / 20.4).
     const char* fv = getenv("WAM_FUSE_NORM");
-    c->fuse_norm_a = fv && fv[0] == '1' && bn_a <= 64 && d.da <= 1024 && d.da % 64 == 0;
+    c->fuse_norm_a = fv && fv[0] == '1' && bn_a <= 64 && d.da <= 1024 && d.da % 64 == 0 && d.r == 0;
     const bool fn = c->fuse_norm_a;
     c->p_a_in = plan_swap(d.da, d.Ma, d.Kin, bn_a, false);
-    c->p_a_qkv = plan_swap(3 * d.A, d.Ma, d.da, bn_a, fn);
-    c->p_a_o = plan_swap(d.da, d.Ma, d.A, bn_a, false);
-    c->p_a_f1 = plan_swap(d.Fa, d.Ma, d.da, bn_a, fn);
-    c->p_a_f2 = plan_swap(d.da, d.Ma, d.Fa, bn_a, false);
+    c->p_a_qkv = plan_swap(3 * d.A, d.Ma, d.da + d.r, bn_a, fn);
+    c->p_a_o = plan_swap(d.da, d.Ma, d.A + d.r, bn_a, false);
+    c->p_a_f1 = plan_swap(d.Fa, d.Ma, d.da + d.r, bn_a, fn);
+    c->p_a_f2 = plan_swap(d.da, d.Ma, d.Fa + d.r, bn_a, false);
+    if (d.r > 0) {
+      c->p_u_qkv = plan_swap(d.r, d.Ma, d.da, bn_a, false);
+      c->p_u_o = plan_swap(d.r, d.Ma, d.A, bn_a, false);
+      c->p_u_f1 = plan_swap(d.r, d.Ma, d.da, bn_a, false);
+      c->p_u_f2 = plan_swap(d.r, d.Ma, d.Fa, bn_a, false);
+    }
     c->p_a_out = plan_swap(d.Pa, d.Ma, d.da, bn_a, fn);
     // workspace and tickets of one launch: rows_a x rows_b output, reduction K
     auto need = [](const GemmPlan& p, int rows_a, int rows_b, int K, bool swap, size_t* w, int* t) {
@@ -941,10 +1005,16 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
       *t = std::max(*t, ((rows_a + 127) / 128) * ((rows_b + p.bn - 1) / p.bn));
     };
     need(c->p_a_in, d.da, d.Ma, d.Kin, true, &ws, &tiles);
-    need(c->p_a_qkv, 3 * d.A, d.Ma, d.da, true, &ws, &tiles);
-    need(c->p_a_o, d.da, d.Ma, d.A, true, &ws, &tiles);
-    need(c->p_a_f1, d.Fa, d.Ma, d.da, true, &ws, &tiles);
-    need(c->p_a_f2, d.da, d.Ma, d.Fa, true, &ws, &tiles);
+    need(c->p_a_qkv, 3 * d.A, d.Ma, d.da + d.r, true, &ws, &tiles);
+    need(c->p_a_o, d.da, d.Ma, d.A + d.r, true, &ws, &tiles);
+    need(c->p_a_f1, d.Fa, d.Ma, d.da + d.r, true, &ws, &tiles);
+    need(c->p_a_f2, d.da, d.Ma, d.Fa + d.r, true, &ws, &tiles);
+    if (d.r > 0) {
+      need(c->p_u_qkv, d.r, d.Ma, d.da, true, &ws, &tiles);
+      need(c->p_u_o, d.r, d.Ma, d.A, true, &ws, &tiles);
+      need(c->p_u_f1, d.r, d.Ma, d.da, true, &ws, &tiles);
+      need(c->p_u_f2, d.r, d.Ma, d.Fa, true, &ws, &tiles);
+    }
     need(c->p_a_out, d.Pa, d.Ma, d.da, true, &ws, &tiles);
     need(c->p_v_qkv, d.Mv, 3 * d.A, d.dv, false, &ws_v, &tiles_v);
     need(c->p_v_o, d.Mv, d.dv, d.A, false, &ws_v, &tiles_v);
@@ -984,15 +1054,21 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     }
     if (cfg->video_has_output) amap(&c->m_w_vout, matp(c, c->ev.outw), d.Pv, d.dv, c->p_v_out.bn);
     amap(&c->m_w_in, matp(c, c->ea.inw), d.da, d.Kin, 128);
-    wmap(&c->m_w_qkv_a, c->ea, kQkvW, 3 * d.A, d.da, 128);
-    wmap(&c->m_w_o_a, c->ea, kOW, d.da, d.A, 128);
-    wmap(&c->m_w_f1_a, c->ea, kF1W, d.Fa, d.da, 128);
-    wmap(&c->m_w_f2_a, c->ea, kF2W, d.da, d.Fa, 128);
+    wmap(&c->m_w_qkv_a, c->ea, kQkvW, 3 * d.A, d.da + d.r, 128);
+    wmap(&c->m_w_o_a, c->ea, kOW, d.da, d.A + d.r, 128);
+    wmap(&c->m_w_f1_a, c->ea, kF1W, d.Fa, d.da + d.r, 128);
+    wmap(&c->m_w_f2_a, c->ea, kF2W, d.da, d.Fa + d.r, 128);
+    if (d.r > 0) {
+      wmap(&c->m_la_qkv, c->ea, kQkvLa, d.r, d.da, 128);
+      wmap(&c->m_la_o, c->ea, kOLa, d.r, d.A, 128);
+      wmap(&c->m_la_f1, c->ea, kF1La, d.r, d.da, 128);
+      wmap(&c->m_la_f2, c->ea, kF2La, d.r, d.Fa, 128);
+    }
     amap(&c->m_w_out, matp(c, c->ea.outw), d.Pa, d.da, 128);
     amap(&c->m_ain, c->a_in, d.Ma, d.Kin, bna);
-    amap(&c->m_ha, c->h_a, d.Ma, d.da, bna);
-    amap(&c->m_oa, c->o_a, d.Ma, d.A, bna);
-    amap(&c->m_fa, c->f_a, d.Ma, d.Fa, bna);
+    amap(&c->m_ha, c->h_a, d.Ma, d.lh, bna);
+    amap(&c->m_oa, c->o_a, d.Ma, d.lo, bna);
+    amap(&c->m_fa, c->f_a, d.Ma, d.lf, bna);
     ok = ok && make_tmap_3d(&c->m_qv, c->q_v, d.Dh, d.Lv, d.B * d.H, (size_t)d.Lv * d.Dh * 2, 128);
     ok = ok && make_tmap_3d(&c->m_cache, c->kv, d.Dh, d.Ltot, 2 * d.N * d.B * d.H, (size_t)d.Ltot * d.Dh * 2, 128);
     ok = ok && make_tmap_sw128(&c->m_xv_out, c->x_v, 4, d.dv, d.Mv, 1, 0, 32, 32);
@@ -1238,17 +1314,20 @@ wam_status wam_import_params(wam_ctx* c, const float* host, size_t nbytes) {
       CK(cudaMemcpy(vecp(c, (int)p), v.data(), e.count() * 4, cudaMemcpyHostToDevice));
       continue;
     }
+    // rows of `cols` values into rows of pitch ld (other columns of the rows,
+    // e.g. the LoRA B factor inside a weight matrix, are left alone)
     if (c->d.bf16) {
-      hb.assign((size_t)e.rows * e.ld, 0);
-      for (int r = 0; r < e.rows; ++r)
-        for (int k = 0; k < e.cols; ++k) {
-          uint32_t b;
-          memcpy(&b, &src[(size_t)r * e.cols + k], 4);
-          hb[(size_t)r * e.ld + k] = (uint16_t)((b + 0x7FFFu + ((b >> 16) & 1u)) >> 16);
-        }
-      CK(cudaMemcpy(matp(c, (int)p), hb.data(), hb.size() * 2, cudaMemcpyHostToDevice));
+      hb.assign((size_t)e.rows * e.cols, 0);
+      for (size_t i = 0; i < hb.size(); ++i) {
+        uint32_t b;
+        memcpy(&b, &src[i], 4);
+        hb[i] = (uint16_t)((b + 0x7FFFu + ((b >> 16) & 1u)) >> 16);
+      }
+      CK(cudaMemcpy2D(matp(c, (int)p), (size_t)e.ld * 2, hb.data(), (size_t)e.cols * 2, (size_t)e.cols * 2, e.rows,
+                      cudaMemcpyHostToDevice));
     } else {
-      CK(cudaMemcpy(matp(c, (int)p), src, e.count() * 4, cudaMemcpyHostToDevice));
+      CK(cudaMemcpy2D(matp(c, (int)p), (size_t)e.ld * 4, src, (size_t)e.cols * 4, (size_t)e.cols * 4, e.rows,
+                      cudaMemcpyHostToDevice));
     }
   }
   return WAM_OK;
@@ -1302,7 +1381,7 @@ wam_status wam_op_linear(int dtype, const void* x, const void* w, const float* b
   e.bias = bias;
   e.out_f32 = out;
   e.ld_out = N;
-  if (dtype == WAM_FP32) return launch_f32_gemm((const float*)x, (const float*)w, M, N, K, e, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
+  if (dtype == WAM_FP32) return launch_f32_gemm((const float*)x, K, (const float*)w, M, N, K, e, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
   if (dtype != WAM_BF16 || K % 64) return WAM_ERR_INVALID_ARG;
   const int bn = swap ? (M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256) : 128;
   if (swap && M > 256) return WAM_ERR_INVALID_ARG;
