@@ -20,8 +20,12 @@
 // before PV_j, so the next scores are ready when the softmax warps finish
 // tile j; K/V tiles are double-buffered by TMA.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
-// issuer, warps 2..5 softmax / output (warp w owns TMEM lanes 32*(w%4)..+31).
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer, warps 2..9 softmax in two warpgroups: warp w reads TMEM lanes
+// 32*(w%4)..+31 (its 32 query rows), warpgroup g = (w-2)/4 takes keys
+// [64 g, 64 g + 64) of every tile.  The two warps of a row quadrant swap their
+// partial row maxima through a spare TMEM column and a 64-thread named
+// barrier; each keeps its own partial row sum.
 // Every wait is bounded (see common.cuh).
 #include "common.cuh"
 #include "kernels.h"
@@ -35,9 +39,10 @@ constexpr int kDh = 64;
 constexpr int kStagesKV = 2;
 constexpr int kTileBytes = kKT * kDh * 2;  // 16 KB (one K or V tile, also the Q tile)
 constexpr int kPBytes = kQ * kKT * 2;      // 32 KB
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA, two softmax warpgroups
 constexpr int kTmemCols = 256;             // S: cols [0,128), O: cols [128,192)
 constexpr float kRescale = 8.0f;           // log2 headroom of the stale row maximum
+constexpr int kXchg = 192;                 // TMEM columns 192, 193: partial row maxima / sums of the two halves
 constexpr int kBarBytes = 128;
 // No alignment slack: two CTAs per SM need every byte (2 x (112 KB + 1 KB reserved) <= 228 KB).
 constexpr int kSmem = kTileBytes + kStagesKV * 2 * kTileBytes + kPBytes + kBarBytes;
@@ -105,6 +110,23 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) 
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// One 32-bit TMEM column of the warp's 32 lanes (thread i: lane base + i).
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "f"(v) : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  return __uint_as_float(r);
+}
+
+// The two softmax warps of TMEM row quadrant q (warps 2 + q' with q' % 4 == q).
+__device__ __forceinline__ void pair_bar(int quad) {
+  asm volatile("bar.sync %0, 64;" ::"r"(2 + quad) : "memory");
+}
+
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -164,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&kv_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(p_full, 256);
     mbar_init(pv_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -242,97 +264,105 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ------------------------------------------------------ softmax warps
     pdl_wait();
     const int quad = warp & 3;
+    const int wg = (warp - 2) >> 2;  // key half of every tile
     const int r = quad * 32 + lane;  // query row within the tile
     const uint32_t t_row = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t t_mine = t_row + kXchg + wg, t_peer = t_row + kXchg + (wg ^ 1);
     const float sl2e = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
-    float mref = 0.f, l = 0.f;  // reference maximum (scaled log2 units) and row sum
-    uint8_t* prow = sP + r * 128;
+    float mref = 0.f, l = 0.f;  // reference maximum (scaled log2 units), partial row sum
+    uint8_t* prow = sP + wg * (kQ * 128) + r * 128;  // this warpgroup's 64-key block of P
     const int swz = r & 7;
+    const int c0 = wg * 64;
+    // Every iteration runs to its end, error or not: the named barrier of the
+    // quadrant must see both of its warps the same number of times (a failed
+    // wait only marks ok = false; garbage then flows to no output).
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      if (!mbar_wait(s_full, j & 1, a.status, kStatusTimeoutAccum, abort_flag)) {
-        ok = false;
-        break;
-      }
+      ok = mbar_wait(s_full, j & 1, a.status, kStatusTimeoutAccum, abort_flag) && ok;
       tc_fence_after();
-      const int kbase = j * kKT;
-      const int nvalid = min(kKT, a.Lk - kbase);  // keys of this tile inside [0, Lk) (>= 1)
-      // pass 1: row maximum of the valid keys
+      const int nvalid = min(kKT, a.Lk - j * kKT) - c0;  // keys of this half inside [0, Lk) (may be <= 0)
+      // pass 1: partial row maximum, swapped with the other half's
       float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kKT; c += 64) {
+      {
         float v[64];
-        tmem_ld64(t_row + c, v);
-        if (nvalid == kKT) {
+        tmem_ld64(t_row + c0, v);
+        if (nvalid >= 64) {
 #pragma unroll
           for (int i = 0; i < 64; i += 2) mx = fmax3(mx, v[i], v[i + 1]);
         } else {
 #pragma unroll
           for (int i = 0; i < 64; ++i)
-            if (c + i < nvalid) mx = fmaxf(mx, v[i]);
+            if (i < nvalid) mx = fmaxf(mx, v[i]);
         }
       }
+      tmem_st1(t_mine, mx);
+      tc_fence_before();
+      pair_bar(quad);
+      tc_fence_after();
+      mx = fmaxf(mx, tmem_ld1(t_peer));
       const float mxs = mx * sl2e;
       if (j == 0) {
         mref = mxs;  // O is written from scratch by the first PV
       } else {
         // PV_{j-1} still reads P_{j-1} from the one P buffer: wait for it
         // before P_j overwrites it (and before O may be rescaled)
-        const bool got = mbar_wait(pv_full, (j - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) {  // leave together: the TMEM accesses below are warp-wide
-          ok = false;
-          break;
-        }
+        ok = mbar_wait(pv_full, (j - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag) && ok;
         tc_fence_after();
-        const bool need = mxs > mref + kRescale;
-        if (__any_sync(0xffffffffu, need)) {  // tcgen05.ld / st are warp-wide
+        const bool need = mxs > mref + kRescale;  // the same decision in both halves
+        if (__any_sync(0xffffffffu, need)) {     // tcgen05.ld / st are warp-wide
           const float alpha = need ? ex2(mref - mxs) : 1.f;
           if (need) mref = mxs;
-          float o[64];
-          tmem_ld64(t_row + 128, o);
+          if (wg == 0) {  // O belongs to the first half
+            float o[64];
+            tmem_ld64(t_row + 128, o);
 #pragma unroll
-          for (int i = 0; i < kDh; ++i) o[i] *= alpha;
-          tmem_st64(t_row + 128, o);
+            for (int i = 0; i < kDh; ++i) o[i] *= alpha;
+            tmem_st64(t_row + 128, o);
+          }
           l *= alpha;
         }
       }
-      // pass 2: P = 2^(s log2e/8 - mref) as bf16 into the swizzled P tile
+      // pass 2: P = 2^(s log2e/8 - mref) as bf16 into this half's P block
       float rs = 0.f;
+      float v[64];
+      tmem_ld64(t_row + c0, v);
+      if (nvalid >= 64) {
 #pragma unroll
-      for (int c = 0; c < kKT; c += 64) {
-        float v[64];
-        tmem_ld64(t_row + c, v);
-        if (nvalid == kKT) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            v[i] = ex2(fmaf(v[i], sl2e, -mref));
-            rs += v[i];
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            v[i] = (c + i < nvalid) ? ex2(fmaf(v[i], sl2e, -mref)) : 0.f;
-            rs += v[i];
-          }
+        for (int i = 0; i < 64; ++i) {
+          v[i] = ex2(fmaf(v[i], sl2e, -mref));
+          rs += v[i];
         }
-        uint8_t* blk = prow + (c >> 6) * (kQ * 128);
+      } else {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint4 w;
-          w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-          w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-          w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-          w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-          *reinterpret_cast<uint4*>(blk + ((q ^ swz) << 4)) = w;
+        for (int i = 0; i < 64; ++i) {
+          v[i] = (i < nvalid) ? ex2(fmaf(v[i], sl2e, -mref)) : 0.f;
+          rs += v[i];
         }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint4 w;
+        w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+        w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+        w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+        w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+        *reinterpret_cast<uint4*>(prow + ((q ^ swz) << 4)) = w;
       }
       l += rs;
       tc_fence_before();
       fence_proxy_async_smem();  // P (generic-proxy stores) -> tensor-core reads
       mbar_arrive_cta(p_full);
     }
-    if (ok && ntiles > 0 &&
-        mbar_wait(pv_full, (ntiles - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag)) {
+    // the full row sum: the two partial sums through the exchange columns,
+    // after both halves have read the last maxima there
+    pair_bar(quad);
+    tmem_st1(t_mine, l);
+    tc_fence_before();
+    pair_bar(quad);
+    tc_fence_after();
+    l += tmem_ld1(t_peer);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && wg == 0 && mbar_wait(pv_full, (ntiles - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag)) {
       tc_fence_after();
       float o[64];
       tmem_ld64(t_row + 128, o);
@@ -341,13 +371,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float inv = 1.0f / l;
         uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)b * a.Lq + qi) * (a.H * kDh) + h * kDh);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int jj = 0; jj < 8; ++jj) {
           uint4 w;
-          w.x = pack_bf16(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
-          w.y = pack_bf16(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
-          w.z = pack_bf16(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
-          w.w = pack_bf16(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
-          dst[j] = w;
+          w.x = pack_bf16(o[8 * jj + 0] * inv, o[8 * jj + 1] * inv);
+          w.y = pack_bf16(o[8 * jj + 2] * inv, o[8 * jj + 3] * inv);
+          w.z = pack_bf16(o[8 * jj + 4] * inv, o[8 * jj + 5] * inv);
+          w.w = pack_bf16(o[8 * jj + 6] * inv, o[8 * jj + 7] * inv);
+          dst[jj] = w;
         }
       }
     }
