@@ -5,27 +5,26 @@
 // RealtimeWAM summary page, 前置知识 "Mixture-of-Transformers": video queries
 // see video keys only).
 //
-// Per 128-key tile j:
-//   S_j  = Q K_j^T       tcgen05.mma M=128 N=128 K=64, fp32 in TMEM (128 cols)
-//   P_j  = exp2(S_j log2e / 8 - m)      softmax warps, thread = query row,
-//          rounded to bf16 into shared memory in the 128B-swizzled K-major
-//          layout the next MMA reads (fence.proxy.async before the hand-off)
-//   O   += P_j V_j       tcgen05.mma M=128 N=64 K=128 accumulating in TMEM, V
+// Two independent flash-attention streams share one CTA: softmax warpgroup g
+// (g = 0, 1) owns the key tiles j = g, g + 2, g + 4, ... (64 keys each), with
+// its own S buffer, P buffer, O accumulator, row maximum and row sum; the two
+// are merged at the end (log-sum-exp weights, as for split keys).  For tile j
+// of stream g:
+//   S_j  = Q K_j^T      tcgen05.mma M=128 N=64 K=64, fp32 into TMEM S_g
+//   P_j  = exp2(S_j log2e / 8 - m_g)   thread = query row (64 keys), bf16
+//          into the 128B-swizzled K-major P_g tile (fence.proxy.async)
+//   O_g += P_j V_j      tcgen05.mma M=128 N=64 K=64 accumulating in TMEM, V
 //          as the MN-major B operand (the cache rows are [key][64 channels])
-// The reference maximum m of a row is raised (and O and the row sum rescaled
-// in place) only when a tile's maximum exceeds it by more than 2^8: exact
-// softmax arithmetic with a stale maximum, P <= 256, and in most tiles no
-// TMEM round trip of O.  P has one buffer: P_j is written once PV_{j-1}
-// (which reads P_{j-1}) has completed.  The MMA warp issues S_{j+1}
-// before PV_j, so the next scores are ready when the softmax warps finish
-// tile j; K/V tiles are double-buffered by TMA.
+// m_g is raised (and O_g and the row sum rescaled in place) only when a tile's
+// maximum exceeds it by more than 2^8: exact softmax arithmetic with a stale
+// maximum, P <= 256, and in most tiles no TMEM round trip of O.  The MMA warp
+// issues S_{j+2} right after PV_j, so while one warpgroup exponentiates tile
+// j the tensor core already holds the other's tile j+1 and its own tile j+2;
+// K/V tiles are 4-stage buffered by TMA.
 //
 // Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
-// issuer, warps 2..9 softmax in two warpgroups: warp w reads TMEM lanes
-// 32*(w%4)..+31 (its 32 query rows), warpgroup g = (w-2)/4 takes keys
-// [64 g, 64 g + 64) of every tile.  The two warps of a row quadrant swap their
-// partial row maxima through a spare TMEM column and a 64-thread named
-// barrier; each keeps its own partial row sum.
+// issuer, warps 2..9 softmax: warp w reads TMEM lanes 32*(w%4)..+31 (its 32
+// query rows) of its warpgroup (w-2)/4's S and O columns.
 // Every wait is bounded (see common.cuh).
 #include "common.cuh"
 #include "kernels.h"
@@ -34,18 +33,18 @@ namespace wam {
 namespace {
 
 constexpr int kQ = 128;       // queries per CTA
-constexpr int kKT = 128;      // keys per tile
+constexpr int kKT = 64;       // keys per tile
 constexpr int kDh = 64;
-constexpr int kStagesKV = 2;
-constexpr int kTileBytes = kKT * kDh * 2;  // 16 KB (one K or V tile, also the Q tile)
-constexpr int kPBytes = kQ * kKT * 2;      // 32 KB
-constexpr int kThreads = 320;  // producer, MMA, two softmax warpgroups
-constexpr int kTmemCols = 256;             // S: cols [0,128), O: cols [128,192)
+constexpr int kStagesKV = 4;
+constexpr int kQBytes = kQ * kDh * 2;      // 16 KB
+constexpr int kKVBytes = kKT * kDh * 2;    // 8 KB (one K or V tile)
+constexpr int kPBytes = kQ * kKT * 2;      // 16 KB (one P tile)
+constexpr int kThreads = 320;              // producer, MMA, two softmax warpgroups
+constexpr int kTmemCols = 256;             // S_0 [0,64), S_1 [64,128), O_0 [128,192), O_1 [192,256)
 constexpr float kRescale = 8.0f;           // log2 headroom of the stale row maximum
-constexpr int kXchg = 192;                 // TMEM columns 192, 193: partial row maxima / sums of the two halves
 constexpr int kBarBytes = 128;
 // No alignment slack: two CTAs per SM need every byte (2 x (112 KB + 1 KB reserved) <= 228 KB).
-constexpr int kSmem = kTileBytes + kStagesKV * 2 * kTileBytes + kPBytes + kBarBytes;
+constexpr int kSmem = kQBytes + kStagesKV * 2 * kKVBytes + 2 * kPBytes + kBarBytes;
 
 // Shared-memory descriptor of an MN-major bf16 operand stored as rows of 128
 // bytes (64 elements along N) with the 128-byte swizzle, consecutive K rows
@@ -110,23 +109,6 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) 
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// One 32-bit TMEM column of the warp's 32 lanes (thread i: lane base + i).
-__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "f"(v) : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
-  uint32_t r;
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-  return __uint_as_float(r);
-}
-
-// The two softmax warps of TMEM row quadrant q (warps 2 + q' with q' % 4 == q).
-__device__ __forceinline__ void pair_bar(int quad) {
-  asm volatile("bar.sync %0, 64;" ::"r"(2 + quad) : "memory");
-}
-
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -159,19 +141,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (threadIdx.x == 0) atomicOr(a.status, kStatusTimeoutDrain);
     return;
   }
-  uint8_t* smem = smem_raw;
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kTileBytes;                       // [stage] K tiles
-  uint8_t* sV = sK + kStagesKV * kTileBytes;           // [stage] V tiles
-  uint8_t* sP = sV + kStagesKV * kTileBytes;           // two 64-key blocks of [128][128 B]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sP + kPBytes);
+  uint8_t* sQ = smem_raw;
+  uint8_t* sK = sQ + kQBytes;                  // [stage] K tiles
+  uint8_t* sV = sK + kStagesKV * kKVBytes;     // [stage] V tiles
+  uint8_t* sP = sV + kStagesKV * kKVBytes;     // [stream] P tiles [128][128 B]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sP + 2 * kPBytes);
   uint64_t* q_full = bar + 0;
-  uint64_t* kv_full = bar + 1;   // [2]
-  uint64_t* kv_empty = bar + 3;  // [2]
-  uint64_t* s_full = bar + 5;
-  uint64_t* p_full = bar + 6;
-  uint64_t* pv_full = bar + 7;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 8);
+  uint64_t* kv_full = bar + 1;   // [4]
+  uint64_t* kv_empty = bar + 5;  // [4]
+  uint64_t* s_full = bar + 9;    // [2] S_g written (MMA -> softmax g)
+  uint64_t* p_full = bar + 11;   // [2] P_g written, S_g read (softmax g -> MMA)
+  uint64_t* pv_full = bar + 13;  // [2] PV into O_g complete (MMA -> softmax g)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -185,9 +166,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 256);
-    mbar_init(pv_full, 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&s_full[g], 1);
+      mbar_init(&p_full[g], 128);
+      mbar_init(&pv_full[g], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -209,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 0) {
     if (lane == 0) {
       pdl_wait();
-      mbar_arrive_expect_tx(q_full, kTileBytes);
+      mbar_arrive_expect_tx(q_full, kQBytes);
       tma_load_3d(sQ, &map_q, q_full, 0, q0, a.zq0 + bh);
       int issued = 0;
       for (int j = 0; j < ntiles; ++j) {
@@ -217,9 +200,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (j >= kStagesKV &&
             !mbar_wait(&kv_empty[s], ((j / kStagesKV) - 1) & 1, a.status, kStatusTimeoutTmaEmpty, abort_flag))
           break;
-        mbar_arrive_expect_tx(&kv_full[s], 2 * kTileBytes);
-        tma_load_3d(sK + s * kTileBytes, &map_k, &kv_full[s], 0, j * kKT, a.zk0 + bh);
-        tma_load_3d(sV + s * kTileBytes, &map_v, &kv_full[s], 0, j * kKT, a.zv0 + bh);
+        mbar_arrive_expect_tx(&kv_full[s], 2 * kKVBytes);
+        tma_load_3d(sK + s * kKVBytes, &map_k, &kv_full[s], 0, j * kKT, a.zk0 + bh);
+        tma_load_3d(sV + s * kKVBytes, &map_v, &kv_full[s], 0, j * kKT, a.zv0 + bh);
         issued = j + 1;
       }
       mbar_wait(q_full, 0, a.status, kStatusTimeoutDrain, nullptr);
@@ -230,33 +213,37 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kQ, kKT);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kQ, kDh) | (1u << 16);  // B (V) is MN-major
-      const uint32_t t_s = tmem, t_o = tmem + 128;
       const uint32_t aq = smem_u32(sQ);
+      // S_j into S_{j & 1} (TMEM columns 64 (j & 1) ..)
       auto issue_s = [&](int j) {
         const int s = j % kStagesKV;
         if (!mbar_wait(&kv_full[s], (j / kStagesKV) & 1, a.status, kStatusTimeoutTmaFull, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t ak = smem_u32(sK + s * kTileBytes);
+        const uint32_t ak = smem_u32(sK + s * kKVBytes);
 #pragma unroll
         for (int kk = 0; kk < kDh / 16; ++kk)
-          tc_mma_bf16(t_s, smem_desc_k128(aq + kk * 32), smem_desc_k128(ak + kk * 32), idesc_s, kk > 0 ? 1u : 0u);
-        tc_commit(s_full);
+          tc_mma_bf16(tmem + (j & 1) * kKT, smem_desc_k128(aq + kk * 32), smem_desc_k128(ak + kk * 32), idesc_s,
+                      kk > 0 ? 1u : 0u);
+        tc_commit(&s_full[j & 1]);
         return true;
       };
-      bool ok = mbar_wait(q_full, 0, a.status, kStatusTimeoutTmaFull, abort_flag) && issue_s(0);
+      bool ok = mbar_wait(q_full, 0, a.status, kStatusTimeoutTmaFull, abort_flag);
+      ok = ok && issue_s(0);
+      if (ntiles > 1) ok = ok && issue_s(1);
       for (int j = 0; j < ntiles && ok; ++j) {
-        // P_j written (and S_j, PV_{j-1} read) by the softmax warps
-        if (!mbar_wait(p_full, j & 1, a.status, kStatusTimeoutAccum, abort_flag)) break;
+        const int g = j & 1, t = j >> 1;  // stream, its tile count
+        // P_j written (and S_j read) by softmax warpgroup g
+        if (!mbar_wait(&p_full[g], t & 1, a.status, kStatusTimeoutAccum, abort_flag)) break;
         tc_fence_after();
-        if (j + 1 < ntiles && !issue_s(j + 1)) break;
         const int s = j % kStagesKV;
-        const uint32_t ap = smem_u32(sP), av = smem_u32(sV + s * kTileBytes);
+        const uint32_t ap = smem_u32(sP + g * kPBytes), av = smem_u32(sV + s * kKVBytes);
 #pragma unroll
         for (int kk = 0; kk < kKT / 16; ++kk)
-          tc_mma_bf16(t_o, smem_desc_k128(ap + (kk >> 2) * (kQ * 128) + (kk & 3) * 32),
-                      smem_desc_mn128(av + kk * 16 * 128), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(pv_full);
-        tc_commit(&kv_empty[s]);
+          tc_mma_bf16(tmem + 128 + g * kDh, smem_desc_k128(ap + kk * 32), smem_desc_mn128(av + kk * 16 * 128),
+                      idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&pv_full[g]);
+        tc_commit(&kv_empty[s]);  // K_j and V_j are read
+        if (j + 2 < ntiles && !issue_s(j + 2)) break;
       }
     }
     __syncwarp();
@@ -264,29 +251,28 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ------------------------------------------------------ softmax warps
     pdl_wait();
     const int quad = warp & 3;
-    const int wg = (warp - 2) >> 2;  // key half of every tile
+    const int g = (warp - 2) >> 2;   // stream: key tiles g, g + 2, ...
     const int r = quad * 32 + lane;  // query row within the tile
-    const uint32_t t_row = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    const uint32_t t_mine = t_row + kXchg + wg, t_peer = t_row + kXchg + (wg ^ 1);
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t t_s = t_lane + g * kKT, t_o = t_lane + 128 + g * kDh;
     const float sl2e = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
-    float mref = 0.f, l = 0.f;  // reference maximum (scaled log2 units), partial row sum
-    uint8_t* prow = sP + wg * (kQ * 128) + r * 128;  // this warpgroup's 64-key block of P
+    float mref = -INFINITY, l = 0.f;  // reference maximum (scaled log2 units) and row sum of the stream
+    uint8_t* prow = sP + g * kPBytes + r * 128;
     const int swz = r & 7;
-    const int c0 = wg * 64;
-    // Every iteration runs to its end, error or not: the named barrier of the
-    // quadrant must see both of its warps the same number of times (a failed
-    // wait only marks ok = false; garbage then flows to no output).
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      ok = mbar_wait(s_full, j & 1, a.status, kStatusTimeoutAccum, abort_flag) && ok;
+    int t = 0;
+    for (int j = g; j < ntiles; j += 2, ++t) {
+      if (!mbar_wait(&s_full[g], t & 1, a.status, kStatusTimeoutAccum, abort_flag)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      const int nvalid = min(kKT, a.Lk - j * kKT) - c0;  // keys of this half inside [0, Lk) (may be <= 0)
-      // pass 1: partial row maximum, swapped with the other half's
+      const int nvalid = min(kKT, a.Lk - j * kKT);  // keys of this tile inside [0, Lk) (>= 1)
       float mx = -INFINITY;
       {
         float v[64];
-        tmem_ld64(t_row + c0, v);
-        if (nvalid >= 64) {
+        tmem_ld64(t_s, v);
+        if (nvalid == kKT) {
 #pragma unroll
           for (int i = 0; i < 64; i += 2) mx = fmax3(mx, v[i], v[i + 1]);
         } else {
@@ -295,38 +281,34 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (i < nvalid) mx = fmaxf(mx, v[i]);
         }
       }
-      tmem_st1(t_mine, mx);
-      tc_fence_before();
-      pair_bar(quad);
-      tc_fence_after();
-      mx = fmaxf(mx, tmem_ld1(t_peer));
       const float mxs = mx * sl2e;
-      if (j == 0) {
-        mref = mxs;  // O is written from scratch by the first PV
+      if (t == 0) {
+        mref = mxs;  // O_g is written from scratch by the stream's first PV
       } else {
-        // PV_{j-1} still reads P_{j-1} from the one P buffer: wait for it
-        // before P_j overwrites it (and before O may be rescaled)
-        ok = mbar_wait(pv_full, (j - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag) && ok;
+        // PV of the stream's previous tile still reads P_g: wait for it before
+        // P_j overwrites it (and before O_g may be rescaled)
+        const bool got = mbar_wait(&pv_full[g], (t - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {  // leave together: the TMEM accesses below are warp-wide
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const bool need = mxs > mref + kRescale;  // the same decision in both halves
-        if (__any_sync(0xffffffffu, need)) {     // tcgen05.ld / st are warp-wide
+        const bool need = mxs > mref + kRescale;
+        if (__any_sync(0xffffffffu, need)) {  // tcgen05.ld / st are warp-wide
           const float alpha = need ? ex2(mref - mxs) : 1.f;
           if (need) mref = mxs;
-          if (wg == 0) {  // O belongs to the first half
-            float o[64];
-            tmem_ld64(t_row + 128, o);
+          float o[64];
+          tmem_ld64(t_o, o);
 #pragma unroll
-            for (int i = 0; i < kDh; ++i) o[i] *= alpha;
-            tmem_st64(t_row + 128, o);
-          }
+          for (int i = 0; i < kDh; ++i) o[i] *= alpha;
+          tmem_st64(t_o, o);
           l *= alpha;
         }
       }
-      // pass 2: P = 2^(s log2e/8 - mref) as bf16 into this half's P block
       float rs = 0.f;
       float v[64];
-      tmem_ld64(t_row + c0, v);
-      if (nvalid >= 64) {
+      tmem_ld64(t_s, v);
+      if (nvalid == kKT) {
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           v[i] = ex2(fmaf(v[i], sl2e, -mref));
@@ -351,33 +333,55 @@ __global__ void __launch_bounds__(kThreads, 2)
       l += rs;
       tc_fence_before();
       fence_proxy_async_smem();  // P (generic-proxy stores) -> tensor-core reads
-      mbar_arrive_cta(p_full);
+      mbar_arrive_cta(&p_full[g]);
     }
-    // the full row sum: the two partial sums through the exchange columns,
-    // after both halves have read the last maxima there
-    pair_bar(quad);
-    tmem_st1(t_mine, l);
-    tc_fence_before();
-    pair_bar(quad);
-    tc_fence_after();
-    l += tmem_ld1(t_peer);
+    // The stream's last PV; then stream 1 hands (m, l) over in the idle P_1
+    // tile and stream 0 merges: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) /
+    // (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)), M = max(m_0, m_1).
+    const int nt = (ntiles - g + 1) / 2;  // tiles of this stream
+    if (ok && nt > 0) ok = mbar_wait(&pv_full[g], (nt - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag);
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && wg == 0 && mbar_wait(pv_full, (ntiles - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag)) {
-      tc_fence_after();
-      float o[64];
-      tmem_ld64(t_row + 128, o);
+    tc_fence_after();
+    float* xch = reinterpret_cast<float*>(sP + kPBytes);  // [128] m_1, [128] l_1, [128] ok_1
+    if (g == 1) {
+      xch[r] = nt > 0 ? mref : -INFINITY;
+      xch[kQ + r] = l;
+      xch[2 * kQ + r] = ok ? 1.f : 0.f;
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");  // both streams, every path
+    // (warp-uniform: stream 1's flag is the same for the 32 rows of a quadrant)
+    const bool has1 = ntiles > 1;
+    if (g == 0 && __all_sync(0xffffffffu, ok && xch[2 * kQ + r] != 0.f)) {
+      const float m1 = xch[r], l1 = xch[kQ + r];
+      const float M = has1 ? fmaxf(mref, m1) : mref;
+      const float f0 = ex2(mref - M), f1 = has1 ? ex2(m1 - M) : 0.f;
+      const float den = l * f0 + l1 * f1;
+      const float inv = 1.0f / den;
       const int qi = q0 + r;
-      if (qi < a.Lq) {
-        const float inv = 1.0f / l;
-        uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)b * a.Lq + qi) * (a.H * kDh) + h * kDh);
+      uint4* dst = reinterpret_cast<uint4*>(a.out + ((size_t)b * a.Lq + qi) * (a.H * kDh) + h * kDh);
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          uint4 w;
-          w.x = pack_bf16(o[8 * jj + 0] * inv, o[8 * jj + 1] * inv);
-          w.y = pack_bf16(o[8 * jj + 2] * inv, o[8 * jj + 3] * inv);
-          w.z = pack_bf16(o[8 * jj + 4] * inv, o[8 * jj + 5] * inv);
-          w.w = pack_bf16(o[8 * jj + 6] * inv, o[8 * jj + 7] * inv);
-          dst[jj] = w;
+      for (int half = 0; half < 2; ++half) {  // 32 channels at a time (registers)
+        float o0[32];
+        tmem_ld32(t_o + 32 * half, o0);
+        if (has1) {
+          float o1[32];
+          tmem_ld32(t_lane + 128 + kDh + 32 * half, o1);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o0[i] = o0[i] * f0 + o1[i] * f1;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o0[i] *= f0;
+        }
+        if (qi < a.Lq) {
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            uint4 w;
+            w.x = pack_bf16(o0[8 * jj + 0] * inv, o0[8 * jj + 1] * inv);
+            w.y = pack_bf16(o0[8 * jj + 2] * inv, o0[8 * jj + 3] * inv);
+            w.z = pack_bf16(o0[8 * jj + 4] * inv, o0[8 * jj + 5] * inv);
+            w.w = pack_bf16(o0[8 * jj + 6] * inv, o0[8 * jj + 7] * inv);
+            dst[4 * half + jj] = w;
+          }
         }
       }
     }
@@ -386,7 +390,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    if (lane == 0 && ntiles > 0) mbar_wait(pv_full, (ntiles - 1) & 1, a.status, kStatusTimeoutDrain, nullptr);
+    if (lane == 0) {
+      for (int g = 0; g < 2; ++g) {
+        const int nt = (ntiles - g + 1) / 2;
+        if (nt > 0) mbar_wait(&pv_full[g], (nt - 1) & 1, a.status, kStatusTimeoutDrain, nullptr);
+      }
+    }
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

@@ -180,7 +180,8 @@ cudaError_t prepare_attention_bf16();
 
 // Tensor-core (tcgen05) attention for video queries: one pass over keys
 // [0, Lk) for 128-query tiles.  Q / K / V are 3-D TMA maps over [z][rows][64]
-// bf16 (box 64 x 128); (b, h) reads matrix z0 + b*H + h of each map.
+// bf16 (Q box 64 x 128 rows, K / V box 64 x 64 rows); (b, h) reads matrix
+// z0 + b*H + h of each map.
 struct AttnTc {
   const CUtensorMap* map_q;
   const CUtensorMap* map_k;

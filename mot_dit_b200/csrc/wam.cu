@@ -1070,7 +1070,7 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     amap(&c->m_oa, c->o_a, d.Ma, d.lo, bna);
     amap(&c->m_fa, c->f_a, d.Ma, d.lf, bna);
     ok = ok && make_tmap_3d(&c->m_qv, c->q_v, d.Dh, d.Lv, d.B * d.H, (size_t)d.Lv * d.Dh * 2, 128);
-    ok = ok && make_tmap_3d(&c->m_cache, c->kv, d.Dh, d.Ltot, 2 * d.N * d.B * d.H, (size_t)d.Ltot * d.Dh * 2, 128);
+    ok = ok && make_tmap_3d(&c->m_cache, c->kv, d.Dh, d.Ltot, 2 * d.N * d.B * d.H, (size_t)d.Ltot * d.Dh * 2, 64);
     ok = ok && make_tmap_sw128(&c->m_xv_out, c->x_v, 4, d.dv, d.Mv, 1, 0, 32, 32);
     ok = ok && make_tmap_sw128(&c->m_fv_out, c->f_v, 2, d.Fv, d.Mv, 1, 0, 64, 32);
     ok = ok && make_tmap_sw128(&c->m_qv_out, c->q_v, 2, d.Dh, d.Lv, d.B * d.H, (size_t)d.Lv * d.Dh * 2, 64, 32);
@@ -1475,8 +1475,8 @@ wam_status wam_op_attention(int dtype, const void* q, const void* k, const void*
     }
     CUtensorMap mq, mk, mv;
     if (!make_tmap_3d(&mq, q, 64, Lq, B * H, (size_t)Lq * 128, 128) ||
-        !make_tmap_3d(&mk, k, 64, Lcache, B * H, (size_t)Lcache * 128, 128) ||
-        !make_tmap_3d(&mv, v, 64, Lcache, B * H, (size_t)Lcache * 128, 128))
+        !make_tmap_3d(&mk, k, 64, Lcache, B * H, (size_t)Lcache * 128, 64) ||
+        !make_tmap_3d(&mv, v, 64, Lcache, B * H, (size_t)Lcache * 128, 64))
       return WAM_ERR_INVALID_ARG;
     AttnTc t;
     t.map_q = &mq;
