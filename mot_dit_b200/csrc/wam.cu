@@ -304,14 +304,19 @@ inline void* vcache(wam_ctx* c, int i) {
   } while (0)
 
 // ------------------------------------------------------------- planning ---
-GemmPlan plan_swap(int rows_w, int tokens, int K, int bn, bool fused_norm) {
+GemmPlan plan_swap(int rows_w, int tokens, int K, int bn, bool fused_norm, int target_ctas) {
   GemmPlan p;
   p.bn = bn;
   const int tiles = ((rows_w + 127) / 128) * ((tokens + bn - 1) / bn);
   const int kb = (K + 63) / 64;
-  int s = (148 + tiles - 1) / tiles;
+  int s = (target_ctas + tiles - 1) / tiles;
   const int min_kb = 3;  // keep each split a few k-blocks deep
   if (s > kb / min_kb) s = kb / min_kb;
+  // With 24 or more feature tiles the weights already stream from as many
+  // SMs; splitting further only adds the partial-tile hand-off (action QKV /
+  // FFN-up at 32 tokens: 4 splits 16.6 us, none 14.5 us per launch in the
+  // 10-step chunk).
+  if (tiles >= 24) s = 1;
   // a tile takes at most splits + 1 pieces; the last one's partner partials
   // must fit its operand ring for the fast reduction
   const int cap = tc_gemm_ring_partials(bn, true, fused_norm);
@@ -989,18 +994,25 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     const char* fv = getenv("WAM_FUSE_NORM");
     c->fuse_norm_a = fv && fv[0] == '1' && bn_a <= 64 && d.da <= 1024 && d.da % 64 == 0 && d.r == 0;
     const bool fn = c->fuse_norm_a;
-    c->p_a_in = plan_swap(d.da, d.Ma, d.Kin, bn_a, false);
-    c->p_a_qkv = plan_swap(3 * d.A, d.Ma, d.da + d.r, bn_a, fn);
-    c->p_a_o = plan_swap(d.da, d.Ma, d.A + d.r, bn_a, false);
-    c->p_a_f1 = plan_swap(d.Fa, d.Ma, d.da + d.r, bn_a, fn);
-    c->p_a_f2 = plan_swap(d.da, d.Ma, d.Fa + d.r, bn_a, false);
-    if (d.r > 0) {
-      c->p_u_qkv = plan_swap(d.r, d.Ma, d.da, bn_a, false);
-      c->p_u_o = plan_swap(d.r, d.Ma, d.A, bn_a, false);
-      c->p_u_f1 = plan_swap(d.r, d.Ma, d.da, bn_a, false);
-      c->p_u_f2 = plan_swap(d.r, d.Ma, d.Fa, bn_a, false);
+    // CTAs per action GEMM (tiles x splits, about): the weight stream spread
+    // over this many SMs; WAM_ACTION_CTAS overrides.
+    int actas = nsm;
+    if (const char* v = getenv("WAM_ACTION_CTAS")) {
+      const int n = atoi(v);
+      if (n > 0) actas = n;
     }
-    c->p_a_out = plan_swap(d.Pa, d.Ma, d.da, bn_a, fn);
+    c->p_a_in = plan_swap(d.da, d.Ma, d.Kin, bn_a, false, actas);
+    c->p_a_qkv = plan_swap(3 * d.A, d.Ma, d.da + d.r, bn_a, fn, actas);
+    c->p_a_o = plan_swap(d.da, d.Ma, d.A + d.r, bn_a, false, actas);
+    c->p_a_f1 = plan_swap(d.Fa, d.Ma, d.da + d.r, bn_a, fn, actas);
+    c->p_a_f2 = plan_swap(d.da, d.Ma, d.Fa + d.r, bn_a, false, actas);
+    if (d.r > 0) {
+      c->p_u_qkv = plan_swap(d.r, d.Ma, d.da, bn_a, false, actas);
+      c->p_u_o = plan_swap(d.r, d.Ma, d.A, bn_a, false, actas);
+      c->p_u_f1 = plan_swap(d.r, d.Ma, d.da, bn_a, false, actas);
+      c->p_u_f2 = plan_swap(d.r, d.Ma, d.Fa, bn_a, false, actas);
+    }
+    c->p_a_out = plan_swap(d.Pa, d.Ma, d.da, bn_a, fn, actas);
     // workspace and tickets of one launch: rows_a x rows_b output, reduction K
     auto need = [](const GemmPlan& p, int rows_a, int rows_b, int K, bool swap, size_t* w, int* t) {
       TcGemm g{};
