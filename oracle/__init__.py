@@ -22,6 +22,8 @@ Modules:
     config  -- model shapes and the five synthetic presets
     params  -- seeded parameter generation (N(0, 0.02) weights, unit gains)
     model   -- float64 forward: video expert, action expert, Euler / endpoints
+    tacd    -- TACD training targets, forward only: teacher K-step rollout,
+               interval-average velocity, student / EMA endpoints, L_TA, L_CD
 """
 from .config import WamConfig, preset  # noqa: F401
 from .params import generate_params, param_specs  # noqa: F401

@@ -53,12 +53,14 @@ def _normal(seed: int, name: str, shape) -> np.ndarray:
 
 
 def make_inputs(seed: int, *, batch: int, l_cond: int, l_video: int, video_width: int,
-                l_action: int, action_dim: int, patch_input: bool = False) -> dict:
+                l_action: int, action_dim: int, patch_input: bool = False, action_clean: bool = False) -> dict:
     """Draw one chunk's inputs.
 
     ``video_width`` is d_v for embedded tokens or P_v when ``patch_input``.
     ``l_cond`` conditioning tokens have width ``video_width`` (only used when
-    not ``patch_input``).
+    not ``patch_input``).  ``action_clean`` also draws a clean action chunk
+    (always drawn with ``patch_input``); every array has its own stream, so
+    asking for it changes none of the others.
     """
     out = {
         "video": _normal(seed, "video", (batch, l_video, video_width)),
@@ -66,9 +68,10 @@ def make_inputs(seed: int, *, batch: int, l_cond: int, l_video: int, video_width
     }
     out["cond"] = (_normal(seed, "cond", (batch, l_cond, video_width))
                    if l_cond > 0 else np.zeros((batch, 0, video_width), np.float32))
+    if patch_input or action_clean:
+        out["action_clean"] = _normal(seed, "action_clean", (batch, l_action, action_dim))
     if patch_input:
         out["video_eps"] = _normal(seed, "video_eps", (batch, l_video, video_width))
-        out["action_clean"] = _normal(seed, "action_clean", (batch, l_action, action_dim))
         out["u_video"] = float(child_rng(seed, "u_video").uniform())
         out["u_action"] = float(child_rng(seed, "u_action").uniform())
     return out
