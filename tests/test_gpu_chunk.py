@@ -2,7 +2,10 @@
 oracle: seeded parameters, the fp32 debug path (rel. L2 <= 1e-4), the bf16
 path (rel. L2 <= 1e-2) on a_0 and v_eff = a_1 - a_0, CEWP == sequential
 bitwise, graph == eager bitwise, the per-block K/V publish, the closed-form
-constant-velocity case and the eager video/action API."""
+constant-velocity case and the eager video/action API (also under stream
+delays)."""
+import time
+
 import numpy as np
 import pytest
 
@@ -89,7 +92,7 @@ def test_mid_bf16_parity_and_kv_publish():
 def test_cewp_equals_sequential_bitwise(cfg):
     c = W.preset(1) if cfg == "tiny" else _mid()
     wam = W.Wam(c, seed=3)
-    for seed in (0, 1, 2):
+    for seed in (0, 1, 2, 3, 4):
         inp = inputs(c, seed)
         outs = [run_chunk(wam, inp, S=S, mode=m, use_graph=g)
                 for S in (1, 3) for m, g in ((W.CEWP, True), (W.SEQUENTIAL, True), (W.CEWP, False),
@@ -101,8 +104,48 @@ def test_cewp_equals_sequential_bitwise(cfg):
     # repeated graph launches stay bitwise stable
     inp = inputs(c, 9)
     first = run_chunk(wam, inp, S=1)
-    for _ in range(20):
+    for _ in range(100):
         assert np.array_equal(run_chunk(wam, inp, S=1), first)
+    wam.close()
+
+
+@pytest.mark.parametrize("delay", ["video", "action", "host"])
+def test_eager_chunks_under_stream_delays(delay):
+    """Two back-to-back chunks through the eager API, with one stream held
+    back by a sleep kernel (or the host pausing between enqueues).  Action
+    attention i waits for video block i's K/V, and the next chunk's video
+    block i waits until the last action attention i has read the cache, so
+    the order comes from events, not timing: both chunks equal the pipelined
+    graph bitwise.  A missing consumed-K/V wait shows under the action delay
+    (chunk 1's video would overwrite K/V that chunk 0 has not read yet)."""
+    c = _mid()
+    wam = W.Wam(c, seed=17)
+    ins = [inputs(c, 40 + k) for k in range(2)]
+    refs = [run_chunk(wam, inp, S=2) for inp in ins]
+    dev = torch.device("cuda", 0)
+    vids = [(torch.from_numpy(inp["video"]).to(dev), torch.from_numpy(inp["cond"]).to(dev)) for inp in ins]
+    acts = [torch.from_numpy(inp["noise"]).to(dev) for inp in ins]
+    sv, sa = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    spin = 20_000_000   # clock cycles (about 10 ms): longer than a whole chunk of this model
+    for k in range(2):
+        if delay == "video":
+            with torch.cuda.stream(sv):
+                torch.cuda._sleep(spin)
+        wam.video_forward(*vids[k], 0.0, stream=sv)
+        if delay == "host":
+            time.sleep(0.01)
+        if delay == "action":
+            with torch.cuda.stream(sa):
+                torch.cuda._sleep(spin)
+        wam.action_step(acts[k], 1.0, 0.5, stream=sa)
+        wam.action_step(acts[k], 0.5, 0.0, stream=sa)
+    sa.synchronize()
+    sv.synchronize()
+    wam.check_device_status()
+    for k in range(2):
+        assert np.array_equal(acts[k].cpu().numpy(), refs[k]), k
+    wam.close()
 
 
 @pytest.mark.parametrize("cfg,S", [("tiny", 1), ("tiny", 8), ("mid", 1), ("mid", 8)])
