@@ -107,6 +107,32 @@ def _ptr(x):
     return x.data_ptr()  # torch.Tensor
 
 
+def _io(x, n: int, where: str, name: str, device: bool = True):
+    """Pointer of a chunk I/O buffer after checking what the C ABI assumes of
+    it: float32, C-contiguous, exactly n elements, in device memory (a CUDA
+    tensor) for the device entry points or host memory (a numpy array or CPU
+    tensor) for the host ones.  None and raw integer addresses pass through
+    unchecked (the library rejects a missing required buffer)."""
+    if x is None or isinstance(x, int):
+        return x
+    if isinstance(x, np.ndarray):
+        ok = not device and x.dtype == np.float32 and x.flags.c_contiguous and x.size == n
+        got = f"numpy {x.dtype}, {x.size} elements"
+    else:  # torch.Tensor
+        ok = (bool(x.is_cuda) == device and str(x.dtype) == "torch.float32" and x.is_contiguous()
+              and x.numel() == n)
+        got = f"{'CUDA' if x.is_cuda else 'CPU'} tensor {x.dtype}, {x.numel()} elements"
+    if not ok:
+        where_mem = "device" if device else "host"
+        raise WamError(1, where, f"{name}: need a C-contiguous float32 {where_mem} buffer of {n} elements, got {got}")
+    return _ptr(x)
+
+
+def _check_sched(t, S: int, where: str):
+    if t is not None and len(t) != S + 1:
+        raise WamError(1, where, f"t_sched has {len(t)} values, S + 1 = {S + 1} needed")
+
+
 def _stream(s):
     if s is None:
         return None
@@ -145,37 +171,60 @@ class Wam:
 
     __del__ = close
 
+    def io_sizes(self):
+        """Element counts of one chunk's (video, cond, actions) buffers:
+        [B, l_video, d_video or video_patch_dim], [B, l_cond, d_video] and
+        [B, l_action, action_dim]."""
+        c = self.cfg
+        return (c.batch * c.l_video * (c.video_patch_dim or c.d_video), c.batch * c.l_cond * c.d_video,
+                c.batch * c.l_action * c.action_dim)
+
+    def _chunk_ptrs(self, where, video, cond, noise, out, device=True):
+        nv, nc, na = self.io_sizes()
+        return (_io(video, nv, where, "video", device), _io(cond, nc, where, "cond", device),
+                _io(noise, na, where, "noise", device), _io(out, na, where, "out", device))
+
     def video_forward(self, video, cond, t_video=0.0, stream=None):
-        self._check(self._lib.wam_video_forward(self._h, _ptr(video), _ptr(cond), t_video, _stream(stream)),
-                    "wam_video_forward")
+        nv, nc, _ = self.io_sizes()
+        w = "wam_video_forward"
+        self._check(self._lib.wam_video_forward(self._h, _io(video, nv, w, "video"), _io(cond, nc, w, "cond"),
+                                                t_video, _stream(stream)), w)
 
     def action_step(self, actions, t_from, t_to, stream=None):
-        self._check(self._lib.wam_action_step(self._h, _ptr(actions), t_from, t_to, _stream(stream)),
-                    "wam_action_step")
+        w = "wam_action_step"
+        self._check(self._lib.wam_action_step(self._h, _io(actions, self.io_sizes()[2], w, "actions"), t_from, t_to,
+                                              _stream(stream)), w)
 
     def infer_chunk(self, video, cond, noise, out, S=1, t_sched=None, mode=CEWP, use_graph=True,
                     stream_video=None, stream_action=None):
+        w = "wam_infer_chunk"
+        ptrs = self._chunk_ptrs(w, video, cond, noise, out)
+        _check_sched(t_sched, S, w)
         p, keep = _sched(t_sched)
-        self._check(self._lib.wam_infer_chunk(self._h, _ptr(video), _ptr(cond), _ptr(noise), _ptr(out), S, p,
-                                              mode, int(use_graph), _stream(stream_video),
-                                              _stream(stream_action)), "wam_infer_chunk")
+        self._check(self._lib.wam_infer_chunk(self._h, *ptrs, S, p, mode, int(use_graph), _stream(stream_video),
+                                              _stream(stream_action)), w)
         del keep
 
     def infer_chunk_host(self, video, cond, noise, out, S=1, t_sched=None, mode=CEWP, use_graph=True,
                          stream_video=None, stream_action=None):
+        w = "wam_infer_chunk_host"
+        ptrs = self._chunk_ptrs(w, video, cond, noise, out, device=False)
+        _check_sched(t_sched, S, w)
         p, keep = _sched(t_sched)
-        self._check(self._lib.wam_infer_chunk_host(self._h, _ptr(video), _ptr(cond), _ptr(noise), _ptr(out), S, p,
-                                                   mode, int(use_graph), _stream(stream_video),
-                                                   _stream(stream_action)), "wam_infer_chunk_host")
+        self._check(self._lib.wam_infer_chunk_host(self._h, *ptrs, S, p, mode, int(use_graph),
+                                                   _stream(stream_video), _stream(stream_action)), w)
         del keep
 
     def joint_one_step(self, video_clean, video_eps, action_clean, action_eps, u_video, u_action,
                        video_out, action_out, shift_video=5.0, shift_action=1.0, mode=CEWP, use_graph=True,
                        stream_video=None, stream_action=None):
+        w = "wam_joint_one_step"
+        nv, _, na = self.io_sizes()
         self._check(self._lib.wam_joint_one_step(
-            self._h, _ptr(video_clean), _ptr(video_eps), _ptr(action_clean), _ptr(action_eps), u_video, u_action,
-            shift_video, shift_action, _ptr(video_out), _ptr(action_out), mode, int(use_graph),
-            _stream(stream_video), _stream(stream_action)), "wam_joint_one_step")
+            self._h, _io(video_clean, nv, w, "video_clean"), _io(video_eps, nv, w, "video_eps"),
+            _io(action_clean, na, w, "action_clean"), _io(action_eps, na, w, "action_eps"), u_video, u_action,
+            shift_video, shift_action, _io(video_out, nv, w, "video_out"), _io(action_out, na, w, "action_out"),
+            mode, int(use_graph), _stream(stream_video), _stream(stream_action)), w)
 
     def export_params(self) -> np.ndarray:
         n = C.c_size_t(0)
@@ -207,9 +256,10 @@ class Wam:
         sequential chunk (see PROF_CLASSES)."""
         ms = np.zeros(len(PROF_CLASSES), np.float32)
         cnt = np.zeros(len(PROF_CLASSES), np.int32)
-        self._check(self._lib.wam_profile_chunk(self._h, _ptr(video), _ptr(cond), _ptr(noise), _ptr(out), S,
-                                                _stream(stream), ms.ctypes.data, cnt.ctypes.data),
-                    "wam_profile_chunk")
+        w = "wam_profile_chunk"
+        ptrs = self._chunk_ptrs(w, video, cond, noise, out)
+        self._check(self._lib.wam_profile_chunk(self._h, *ptrs, S, _stream(stream), ms.ctypes.data, cnt.ctypes.data),
+                    w)
         return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(PROF_CLASSES)}
 
 

@@ -60,3 +60,47 @@ def test_status_strings():
     assert L.wam_status_str(0) == b"ok"
     assert L.wam_status_str(5) == b"device wait timed out"
     assert L.wam_last_error(None) == b""
+
+
+# ---------------------------------------------------------------- binding
+def _shell(k):
+    """A Wam object with preset k's shapes and no device context: the
+    binding's buffer checks run, and a call that gets past them reaches the
+    library with a NULL context (WAM_ERR_INVALID_ARG, nothing enqueued)."""
+    w = W.Wam.__new__(W.Wam)
+    w.cfg = W.preset(k)
+    w._lib = W.lib()
+    w._h = None
+    return w
+
+
+def test_binding_io_sizes_follow_the_config():
+    assert _shell(2).io_sizes() == (1024 * 1536, 64 * 1536, 32 * 30)
+    assert _shell(4).io_sizes() == (8 * 2048 * 1536, 8 * 64 * 1536, 8 * 32 * 30)
+    assert _shell(5).io_sizes() == (1024 * 192, 0, 16 * 30)
+
+
+def test_binding_rejects_buffers_the_library_would_misread():
+    import numpy as np
+    import torch
+    w = _shell(1)
+    nv, nc, na = w.io_sizes()
+    video, noise = torch.zeros(nv), torch.zeros(na)
+    with pytest.raises(W.WamError, match="device buffer") as e:      # host memory for a device entry point
+        w.infer_chunk(video, None, noise, torch.zeros(na))
+    assert e.value.status == 1
+    with pytest.raises(W.WamError, match="device buffer"):
+        w.action_step(noise, 1.0, 0.0)
+    hv, hn, ho = (np.zeros(n, np.float32) for n in (nv, na, na))
+    with pytest.raises(W.WamError, match="out: need"):                # wrong size
+        w.infer_chunk_host(hv, None, hn, np.zeros(na + 1, np.float32))
+    with pytest.raises(W.WamError, match="noise: need"):              # wrong dtype
+        w.infer_chunk_host(hv, None, hn.astype(np.float64), ho)
+    with pytest.raises(W.WamError, match="video: need"):              # not contiguous
+        w.infer_chunk_host(torch.zeros(nv, 2)[:, 0], None, hn, ho)
+    with pytest.raises(W.WamError, match="t_sched has 2 values"):
+        w.infer_chunk_host(hv, None, hn, ho, S=2, t_sched=[1.0, 0.0])
+    # well-formed host buffers pass the checks and reach the library
+    with pytest.raises(W.WamError) as e:
+        w.infer_chunk_host(hv, None, hn, ho, S=2, t_sched=[1.0, 0.5, 0.0])
+    assert e.value.status == 1 and "need" not in str(e.value)
