@@ -64,7 +64,11 @@ typedef enum { WAM_SCHED_SEQUENTIAL = 0, WAM_SCHED_CEWP = 1 } wam_sched;
  * expert's QKV / out / FFN projections.  video_has_output: the video expert's
  * last block and output map run (joint variant).  dtype: WAM_BF16 (bf16
  * weights and GEMM operands, fp32 accumulation and residual stream, head_dim
- * 64) or WAM_FP32 (fp32 everywhere, debug precision). */
+ * 64) or WAM_FP32 (fp32 everywhere, debug precision).  wam_init rejects
+ * (WAM_ERR_INVALID_ARG) shapes its kernels do not cover: expert widths above
+ * 1536; on the bf16 path widths that are not multiples of 64 (128 for
+ * ffn_video and the attention width), more than 64 action tokens per sample
+ * or 256 per chunk, and a LoRA rank that is not a multiple of 64. */
 typedef struct {
   int n_blocks, d_video, d_action, n_heads, head_dim, ffn_video, ffn_action;
   int l_cond, l_video, l_action, action_dim, video_patch_dim;

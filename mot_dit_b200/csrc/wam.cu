@@ -776,6 +776,8 @@ bool check_cfg(const wam_config* g, std::string* why) {
   if (g->l_video < 1 || g->l_action < 1 || g->l_cond < 0 || g->batch < 1 || g->action_dim < 1) return bad("token counts");
   if (g->head_dim % 2) return bad("head_dim must be even");
   if (g->d_video % 8 || g->d_action % 8 || g->ffn_video % 8 || g->ffn_action % 8) return bad("widths must be multiples of 8");
+  // the norm / modulation prologue keeps a whole row in one warp's registers
+  if (g->d_video > 1536 || g->d_action > 1536) return bad("expert widths above 1536 are not supported");
   if (g->video_has_output && g->video_patch_dim <= 0) return bad("a video output needs patch input");
   if (g->video_patch_dim > 0 && g->l_cond != 0) return bad("patch input takes no conditioning tokens");
   if (g->lora_rank < 0) return bad("lora_rank");

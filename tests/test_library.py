@@ -46,6 +46,7 @@ def test_unknown_preset_rejected():
 @pytest.mark.parametrize("bad", [
     dict(n_blocks=0), dict(head_dim=48, dtype=W.BF16), dict(head_dim=15), dict(l_action=0),
     dict(video_has_output=1), dict(d_video=100, dtype=W.BF16), dict(dtype=7), dict(batch=0),
+    dict(d_video=2048, dtype=W.BF16), dict(d_action=1600),
 ])
 def test_init_rejects_bad_config_without_device(bad):
     base = W.preset(2) if bad.get("dtype") == W.BF16 else W.preset(1)
