@@ -189,6 +189,36 @@ def test_joint_attention_equals_masked_full_sequence():
     np.testing.assert_allclose(oa, full[:, :, Lv:], rtol=1e-12, atol=1e-13)
 
 
+def _naive_attention_row(q, keys, vals):
+    """softmax(q . k / sqrt(Dh)) V for one query, in plain Python loops."""
+    scale = 1.0 / math.sqrt(len(q))
+    scores = [sum(qi * ki for qi, ki in zip(q, k)) * scale for k in keys]
+    m = max(scores)
+    w = [math.exp(x - m) for x in scores]
+    z = sum(w)
+    return [sum(wj * v[c] for wj, v in zip(w, vals)) / z for c in range(len(vals[0]))]
+
+
+def test_joint_attention_against_naive_loops():
+    """The O(n^2) definition, loop by loop, on a tiny shape: video queries over
+    video keys only, action queries over [video; action] keys."""
+    rng = np.random.default_rng(15)
+    H, Lv, La, Dh = 2, 5, 3, 4
+    qv, kv_, vv = (rng.standard_normal((1, H, Lv, Dh)) for _ in range(3))
+    qa, ka, va = (rng.standard_normal((1, H, La, Dh)) for _ in range(3))
+    ov = M.attention(qv, kv_, vv)
+    oa = M.attention(qa, np.concatenate([kv_, ka], 2), np.concatenate([vv, va], 2))
+    for h in range(H):
+        keys_v, vals_v = kv_[0, h].tolist(), vv[0, h].tolist()
+        for i in range(Lv):
+            want = _naive_attention_row(qv[0, h, i].tolist(), keys_v, vals_v)
+            np.testing.assert_allclose(ov[0, h, i], want, rtol=1e-12, atol=1e-14)
+        keys_j, vals_j = keys_v + ka[0, h].tolist(), vals_v + va[0, h].tolist()
+        for i in range(La):
+            want = _naive_attention_row(qa[0, h, i].tolist(), keys_j, vals_j)
+            np.testing.assert_allclose(oa[0, h, i], want, rtol=1e-12, atol=1e-14)
+
+
 def test_mot_block_equals_joint_sequence_formulation():
     """One MoT block of the action expert written as a single masked attention
     over the joint token sequence (per-token expert weights, positions 0..L_v+L_a-1)."""
