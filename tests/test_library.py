@@ -105,3 +105,26 @@ def test_binding_rejects_buffers_the_library_would_misread():
     with pytest.raises(W.WamError) as e:
         w.infer_chunk_host(hv, None, hn, ho, S=2, t_sched=[1.0, 0.5, 0.0])
     assert e.value.status == 1 and "need" not in str(e.value)
+
+
+def test_header_compiles_as_c_and_links_from_c():
+    """include/wam.h is a C header: a C99 program (tests/c_abi/abi_check.c)
+    compiles with -pedantic -Werror, links against the library and gets the
+    documented argument errors without a device."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(W.library_path())
+    W.lib()  # raises if the library has not been built
+    out_dir = os.path.join(lib_dir, "_build")
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "abi_check")
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+           os.path.join(ROOT, "tests", "c_abi", "abi_check.c"), "-L", lib_dir, "-lmotdit",
+           f"-Wl,-rpath,{lib_dir}", "-o", exe]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and "c abi ok" in r.stdout, r.stdout + r.stderr
