@@ -861,7 +861,8 @@ void wam_destroy(wam_ctx* c) {
   cudaDeviceSynchronize();
   for (auto& kv : c->graphs) cudaGraphExecDestroy(kv.second);
   for (auto* v : {&c->ev_kv, &c->ev_kv_cap, &c->ev_used})
-    for (auto e : *v) cudaEventDestroy(e);
+    for (auto e : *v)
+      if (e) cudaEventDestroy(e);
   for (auto e : {c->ev_fork, c->ev_join, c->ev_pre, c->ev_post})
     if (e) cudaEventDestroy(e);
   for (auto e : c->prof_pool) cudaEventDestroy(e);
@@ -881,7 +882,8 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   if (!cfg || !out) return WAM_ERR_INVALID_ARG;
   std::string why;
   if (!check_cfg(cfg, &why)) return WAM_ERR_INVALID_ARG;
-  std::unique_ptr<wam_ctx> holder(new wam_ctx());
+  // on any failure below, wam_destroy releases what was created so far
+  std::unique_ptr<wam_ctx, void (*)(wam_ctx*)> holder(new wam_ctx(), wam_destroy);
   wam_ctx* c = holder.get();
   c->cfg = *cfg;
   CK(cudaGetDevice(&c->device));

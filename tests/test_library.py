@@ -56,6 +56,18 @@ def test_init_rejects_bad_config_without_device(bad):
     assert st == 1 and not h.value
 
 
+def test_init_without_a_device_fails_cleanly():
+    """A valid config on a host with no GPU: WAM_ERR_CUDA, *out left NULL,
+    and the half-built context released (a second call behaves the same)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    cfg = W.preset(1)
+    for _ in range(2):
+        h = C.c_void_p()
+        assert W.lib().wam_init(C.byref(cfg), 0, C.byref(h)) == 4 and not h.value
+
+
 def test_status_strings():
     L = W.lib()
     assert L.wam_status_str(0) == b"ok"
