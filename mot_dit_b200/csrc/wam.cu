@@ -1187,12 +1187,12 @@ wam_status wam_infer_chunk_host(wam_ctx* c, const float* hv, const float* hc, co
   if (!c || !hv || !hn || !hout || (c->d.Lc > 0 && !hc)) return fail(c, WAM_ERR_INVALID_ARG, "null host buffer");
   const Dims& d = c->d;
   const size_t nv = (size_t)d.B * d.Lvid * d.dv, nc = (size_t)d.B * d.Lc * d.dv, nn = (size_t)d.Ma * d.Pa;
-  if (!c->h_video) {
-    RET(dalloc(c, &c->h_video, nv * 4));
-    RET(dalloc(c, &c->h_cond, nc * 4));
-    RET(dalloc(c, &c->h_noise, nn * 4));
-    RET(dalloc(c, &c->h_out, nn * 4));
-  }
+  // staging allocated on first use; each buffer on its own, so a failed
+  // allocation is retried by the next call instead of leaving a gap
+  if (!c->h_video) RET(dalloc(c, &c->h_video, nv * 4));
+  if (!c->h_cond) RET(dalloc(c, &c->h_cond, nc * 4));
+  if (!c->h_noise) RET(dalloc(c, &c->h_noise, nn * 4));
+  if (!c->h_out) RET(dalloc(c, &c->h_out, nn * 4));
   cudaStream_t sv = (cudaStream_t)stream_video;
   CK(cudaMemcpyAsync(c->h_video, hv, nv * 4, cudaMemcpyHostToDevice, sv));
   if (nc) CK(cudaMemcpyAsync(c->h_cond, hc, nc * 4, cudaMemcpyHostToDevice, sv));
