@@ -22,9 +22,13 @@ def _mid():
     return W.WamConfig(**MID_BF16)
 
 
-@pytest.mark.parametrize("cfg", ["tiny", "mid"])
+@pytest.mark.parametrize("cfg", ["tiny", "mid", "tiny_lora", "mid_lora"])
 def test_seeded_params_match_oracle_generator(cfg):
-    c = W.preset(1) if cfg == "tiny" else _mid()
+    """Every parameter the library generated on the device (LoRA factors
+    included: B lives inside its layer's weight matrix) equals the oracle's."""
+    c = W.preset(1) if cfg.startswith("tiny") else _mid()
+    if cfg.endswith("lora"):
+        c = c.replace(lora_rank=64)
     wam = W.Wam(c, seed=1234)
     flat = wam.export_params()
     P = PR.generate_params(ocfg(c), 1234)
