@@ -147,6 +147,8 @@ class ClockSampler:
 
     def stop(self):
         if not self.proc:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
             return None
         self.proc.terminate()
         try:
@@ -264,6 +266,13 @@ def max_over_ranks(ms, dist, device):
     return float(t.item())
 
 
+def step_percentiles(ms):
+    """Median, p10 and p90 of per-step times (numpy's linear interpolation)."""
+    import numpy as np
+    q = np.percentile(np.asarray(ms, dtype=np.float64), [50, 10, 90])
+    return {"median": round(float(q[0]), 4), "p10": round(float(q[1]), 4), "p90": round(float(q[2]), 4)}
+
+
 def job_ms_per_chunk(ms_per_step, world):
     """Whole-job time per chunk: each of the `world` replicas makes one chunk
     per step (independent problems, weak scaling), so the job makes `world`
@@ -318,15 +327,18 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]  # end of each step
     e0.record(sv)
-    for _ in range(args.steps):
+    for i in range(args.steps):
         step()
+        marks[i].record(sv)
     e1.record(sv)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     wam.check_device_status()
     elapsed = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    per_step = [(marks[i - 1] if i else e0).elapsed_time(marks[i]) for i in range(args.steps)]
     ms_per_step = elapsed / args.steps
     launches_per_chunk = wam.chunk_kernel_count(S)
 
@@ -399,6 +411,7 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "schedule": args.schedule + ("+graph" if use_graph else "+eager"),
                    "l2": "no flush: each chunk streams 2.1 GB of weights, > 126 MB L2"},
+        "step_ms": dict(step_percentiles(per_step), note="this rank's per-step times (rank 0)"),
         "chunks_per_s": round(1e3 * world / ms_per_step, 2),
         "actions_per_s": round(1e3 * world * c.batch * c.l_action / ms_per_step, 1),
         "roofline": {"bound": "tensor", "kernel": "tcgen05 GEMM, video expert (QKV/out/FFN)",

@@ -54,3 +54,8 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
         config, seed, warmup, steps, gpus = 2, 0, 0, 1, 2
     assert bench.run_reference(A(), rank=1, world=2) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_step_percentiles():
+    q = bench.step_percentiles([4.0, 4.1, 3.9, 4.05, 5.0])
+    assert q == {"median": 4.05, "p10": 3.94, "p90": 4.64}
