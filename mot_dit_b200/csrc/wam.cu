@@ -676,8 +676,8 @@ wam_status enqueue_chunk(wam_ctx* c, int steps, int mode, bool joint, cudaStream
     CK(launch_init_action(c->aio_chunk, c->a_state, d.bf16 ? c->a_in : nullptr, d.bf16, d.Ma, d.Pa, d.Kin, s_act));
   }
   if (cewp) {
-    // Enqueue the two experts interleaved block by block is not needed: the
-    // streams run concurrently; the per-block events order Attn^a_i after P^v_i.
+    // The experts need not be enqueued interleaved block by block: the two
+    // streams run concurrently, and the per-block events order Attn^a_i after P^v_i.
     RET(enqueue_video(c, sv, c->vio_chunk, joint, ev_kv, false));
     for (int j = 0; j < steps; ++j) RET(enqueue_action_step(c, sa, c->aio_chunk, j, j == 0 ? ev_kv : nullptr, false));
   } else {
