@@ -432,6 +432,14 @@ def run_ours(args, rank, world, local_rank):
         ms_cpu, sample = cpu_oracle_sample(args.config, args.seed)
         line["cpu_baseline"] = {"value": round(ms_cpu, 1), "unit": "ms", "cores": oracle_threads(), "kind": "oracle",
                                 "sample": sample + f"; {cpu_info()}"}
+        try:  # the same sample on one thread (BLAS pool limited to 1)
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1, user_api="blas"):
+                ms_1t, sample_1t = cpu_oracle_sample(args.config, args.seed, reps=1)
+            line["cpu_baseline_1thread"] = {"value": round(ms_1t, 1), "unit": "ms", "cores": 1, "kind": "oracle",
+                                            "sample": sample_1t}
+        except ImportError:
+            pass
     print(json.dumps(line), flush=True)
     if dist:
         dist.destroy_process_group()
