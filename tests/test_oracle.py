@@ -419,3 +419,140 @@ def test_joint_one_step_composition():
     r0 = M.joint_one_step(cfg, P0, inp)
     assert np.abs(r0["f_action"] - r["f_action"]).max() > 1e-8
     np.testing.assert_array_equal(r0["f_video"], r["f_video"])   # LoRA is on the action expert only
+
+
+# --------------------------------------------------------------------------
+# P_i's QK-norm + RoPE, the timestep MLP and the FFN: closed forms with
+# hand-chosen weights (summary page, 方法步骤详情: the fused "RMSNorm/RoPE"
+# operator and the merged QKV projection; the AdaLN timestep modulation and
+# the GELU FFN of the shared block definition)
+# --------------------------------------------------------------------------
+
+def test_project_qkv_per_head_norm_then_rope_closed_form():
+    """Two heads of two channels, every weight zero, so q/k/v are the bias.
+    Head 0's q = (3, 4) with gain (1, 0), head 1's q = (-2, 0) with gain (1, 1),
+    one token at position pi/2 (RoPE turns channel pair (0, 1) by pi/2).
+
+    Per-head RMS: head 0 has mean square 12.5, head 1 has 2.  Norm, then
+    gain, then a quarter turn (x, y) -> (-y, x):
+      head 0: (3, 4)/sqrt(12.5+eps) -> gain -> (3r0, 0) -> (0, 3r0)
+      head 1: (-2, 0)/sqrt(2+eps)   -> gain -> (-2r1, 0) -> (0, -2r1).
+    RoPE first would give head 0 (-4r0, 0); a norm over both heads (mean
+    square 7.25) gives other magnitudes; v is the raw projection."""
+    cfg = _tiny(n_heads=2, head_dim=2)
+    P = _zero_params(cfg)
+    b = "video.blk0."
+    q_vals = [3.0, 4.0, -2.0, 0.0]
+    k_vals = [0.0, 5.0, 1.0, 1.0]
+    v_vals = [0.25, -0.5, 1.5, -2.0]
+    P[b + "qkv.b"] = np.array(q_vals + k_vals + v_vals, np.float32)
+    P[b + "qn.g"] = np.array([1.0, 0.0, 1.0, 1.0], np.float32)
+    P[b + "kn.g"] = np.array([2.0, 1.0, 1.0, 1.0], np.float32)
+    h = np.zeros((1, 1, cfg.d_video))
+    q, k, v = M.project_qkv(cfg, P, b, h, np.array([math.pi / 2]), 1.0)
+    r0, r1 = 1.0 / math.sqrt(12.5 + 1e-6), 1.0 / math.sqrt(2.0 + 1e-6)
+    np.testing.assert_allclose(q[0, 0, 0], [0.0, 3.0 * r0], atol=1e-15)
+    np.testing.assert_allclose(q[0, 1, 0], [0.0, -2.0 * r1], atol=1e-15)
+    # k head 0 = (0, 5): mean square 12.5, gain (2, 1) -> (0, 5 r0) -> (-5 r0, 0);
+    # k head 1 = (1, 1): mean square 1 -> (1, 1)/sqrt(1+eps) -> (-1, 1)/sqrt(1+eps)
+    rk = 1.0 / math.sqrt(1.0 + 1e-6)
+    np.testing.assert_allclose(k[0, 0, 0], [-5.0 * r0, 0.0], atol=1e-15)
+    np.testing.assert_allclose(k[0, 1, 0], [-rk, rk], atol=1e-15)
+    np.testing.assert_array_equal(v[0, :, 0].ravel(), v_vals)
+
+
+def test_project_qkv_norm_is_per_head_and_per_token():
+    """Unit gains at position 0 (RoPE = identity): every (token, head) slice
+    of q and k has mean square ms/(ms+eps) of its own pre-norm mean square ms;
+    scaling one head's rows of W_qkv by 10 changes no other head's q or k."""
+    cfg = _tiny()
+    P = {k: v.astype(np.float64) for k, v in PR.generate_params(cfg, 21).items()}
+    b = "video.blk0."
+    rng = np.random.default_rng(22)
+    h = rng.standard_normal((2, 5, cfg.d_video))
+    pos = np.zeros(5)
+    q, k, v = M.project_qkv(cfg, P, b, h, pos, 1.0)
+    A, H, Dh = cfg.attn_dim, cfg.n_heads, cfg.head_dim
+    raw = h @ P[b + "qkv.w"].T + P[b + "qkv.b"]
+    for sec, got in ((0, q), (1, k)):
+        pre = raw[..., sec * A:(sec + 1) * A].reshape(2, 5, H, Dh).transpose(0, 2, 1, 3)
+        ms = np.mean(pre ** 2, -1)
+        np.testing.assert_allclose(np.mean(got ** 2, -1), ms / (ms + 1e-6), rtol=1e-12)
+    np.testing.assert_allclose(v, raw[..., 2 * A:].reshape(2, 5, H, Dh).transpose(0, 2, 1, 3), rtol=1e-13)
+    # head 2's q and k rows (weights and bias) scaled by 10
+    P2 = dict(P)
+    w, bb = P[b + "qkv.w"].copy(), P[b + "qkv.b"].copy()
+    for sec in (0, 1):
+        rows = slice(sec * A + 2 * Dh, sec * A + 3 * Dh)
+        w[rows] *= 10.0
+        bb[rows] *= 10.0
+    P2[b + "qkv.w"], P2[b + "qkv.b"] = w, bb
+    q2, k2, _ = M.project_qkv(cfg, P2, b, h, pos, 1.0)
+    for hh in range(H):
+        # head 2 itself moves only through eps (relative change about eps / ms, ms ~ 0.03 here)
+        tol = 2e-3 if hh == 2 else 0.0
+        np.testing.assert_allclose(q2[:, hh], q[:, hh], rtol=tol, atol=0)
+        np.testing.assert_allclose(k2[:, hh], k[:, hh], rtol=tol, atol=0)
+
+
+def test_modulation_mlp_closed_form():
+    """tau(t) -> c = W_t2 SiLU(W_t1 tau + b_t1) + b_t2 -> m = W_m SiLU(c) + b_m
+    with selection weights.  At t = pi/2000 feature 128 (sin(1000 t w_0)) is 1
+    and feature 0 (cos) is 0.  W_t1 picks 2 x feature 128 plus bias 0.5 into
+    unit 0; W_t2 = I with bias -1; W_m copies unit 0 into outputs 0 and 7,
+    with bias 0.25 on output 7.  So
+      c_0 = silu(2.5) - 1,  m_0 = silu(c_0),  m_7 = silu(c_0) + 0.25,
+    and every other output is 0.  A SiLU dropped, doubled or moved changes m_0."""
+    cfg = _tiny(n_blocks=1)
+    P = _zero_params(cfg)
+    d = cfg.d_action
+    P["action.t1.w"][0, 128] = 2.0
+    P["action.t1.b"][0] = 0.5
+    P["action.t2.w"] = np.eye(d, dtype=np.float32)
+    P["action.t2.b"][0] = -1.0
+    P["action.mod.w"][0, 0] = 1.0
+    P["action.mod.w"][7, 0] = 1.0
+    P["action.mod.b"][7] = 0.25
+    m = M.modulation(cfg, P, "action", math.pi / 2000.0)
+
+    def silu(z):
+        return z / (1.0 + math.exp(-z))
+    c0 = silu(2.5) - 1.0
+    want = np.zeros(6 * d)
+    want[0] = silu(c0)
+    want[7] = silu(c0) + 0.25
+    np.testing.assert_allclose(m, want, rtol=1e-13, atol=1e-13)
+    # a dropped SiLU before the modulation map would give c_0 itself
+    assert abs(m[0] - c0) > 0.2
+
+
+def test_block_rest_ffn_activation_between_the_two_layers():
+    """R_i with selection weights and (1 + sc2) = 0, so h2 = sh2 exactly.
+    sh2_0 = -0.75 reaches hidden unit 0 through ffn1 (w = e_0 e_0^T, no bias);
+    ffn2 copies hidden unit 0 into output 3 and adds b2.  The out-projection is
+    zero apart from its bias, so x += g1 b_o + g2 (GELU_tanh(-0.75) e_3 + b2).
+    GELU_tanh comes from torch; SiLU (-0.256), the identity (-0.75) or GELU
+    after ffn2 would all give other values."""
+    cfg = _tiny(n_blocks=1)
+    P = _zero_params(cfg)
+    d, F = cfg.d_action, cfg.ffn_action
+    b = "action.blk0."
+    rng = np.random.default_rng(23)
+    P[b + "o.b"] = rng.standard_normal(d).astype(np.float32)
+    P[b + "ffn1.w"][0, 0] = 1.0
+    P[b + "ffn2.w"][3, 0] = 1.0
+    P[b + "ffn2.b"] = rng.standard_normal(d).astype(np.float32)
+    sh1, sc1, g1 = (rng.standard_normal(d) for _ in range(3))
+    sh2 = np.zeros(d)
+    sh2[0] = -0.75
+    sc2 = -np.ones(d)
+    g2 = rng.standard_normal(d)
+    x = rng.standard_normal((1, 2, d))
+    o = np.zeros((1, cfg.n_heads, 2, cfg.head_dim))
+    got = M.block_rest(cfg, P, b, x, o, (sh1, sc1, g1, sh2, sc2, g2), 1.0)
+    gelu = float(torch.nn.functional.gelu(torch.tensor(-0.75, dtype=torch.float64), approximate="tanh"))
+    f = P[b + "ffn2.b"].astype(np.float64).copy()
+    f[3] += gelu
+    want = x + g1 * P[b + "o.b"] + g2 * f
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-14)
+    assert abs(gelu - (-0.75 / (1 + math.exp(0.75)))) > 0.05 and abs(gelu + 0.75) > 0.5
