@@ -94,7 +94,10 @@ wam_status wam_preset(int k, wam_config* out);
  * weights / biases / modulation tables / LoRA factors, 1 for norm gains;
  * rounded to bf16 for bf16 models), allocates the K/V cache, the
  * activations and the workspaces, and creates the per-block events.
- * Synchronous.  *out is set only on WAM_OK. */
+ * Synchronous.  *out is set only on WAM_OK.  WAM_ERR_OOM when a device
+ * allocation fails, or would take the context past the byte budget given in
+ * the environment variable WAM_DEVICE_MEMORY_LIMIT (unset or 0: no budget);
+ * everything allocated so far is released. */
 wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out);
 
 /* Release everything the context owns (device memory, events, graphs).
@@ -248,6 +251,9 @@ wam_status wam_op_norm_mod(int dtype, const float* dev_x, void* dev_h, int M, in
  *   - The first call on a device looks up the array's device address and
  *     sets the kernel's shared-memory limit (once per device, with that
  *     device current); make that first call before any stream capture.
+ *     Both are kept for the life of the process: after a cudaDeviceReset
+ *     that device's cached address is stale, so do not call this entry point
+ *     again on a device that has been reset.
  *   - Every call shares the array: calls that overlap on the GPU (other
  *     streams, other threads) race.  Each call clears the tickets it uses
  *     before its kernel runs.

@@ -125,6 +125,8 @@ struct wam_ctx {
   bool video_done = false;
   int launches = 0;
   std::string last_error;
+  // device-memory budget of the context (WAM_DEVICE_MEMORY_LIMIT, bytes; 0 = none)
+  size_t mem_limit = 0, mem_used = 0;
 
   // per-launch timing (wam_profile_chunk)
   bool prof_on = false;
@@ -757,12 +759,16 @@ bool valid_schedule(const float* t, int S) {
 template <typename T>
 wam_status dalloc(wam_ctx* c, T** p, size_t bytes) {
   if (bytes == 0) bytes = 256;
+  if (c->mem_limit && c->mem_used + bytes > c->mem_limit)
+    return fail(c, WAM_ERR_OOM, "allocation of %zu bytes exceeds the context's device memory limit (%zu of %zu used)",
+                bytes, c->mem_used, c->mem_limit);
   cudaError_t e = cudaMalloc((void**)p, bytes);
   if (e == cudaErrorMemoryAllocation) {
     cudaGetLastError();
     return fail(c, WAM_ERR_OOM, "cudaMalloc(%zu) failed: out of device memory", bytes);
   }
   CK(e);
+  c->mem_used += bytes;
   CK(cudaMemset(*p, 0, bytes));
   return WAM_OK;
 }
@@ -886,6 +892,7 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   std::unique_ptr<wam_ctx, void (*)(wam_ctx*)> holder(new wam_ctx(), wam_destroy);
   wam_ctx* c = holder.get();
   c->cfg = *cfg;
+  if (const char* v = getenv("WAM_DEVICE_MEMORY_LIMIT")) c->mem_limit = strtoull(v, nullptr, 10);
   CK(cudaGetDevice(&c->device));
   CK(prepare_tc_gemm());
   CK(prepare_attention_tc());
@@ -1312,6 +1319,7 @@ wam_status wam_export_params(wam_ctx* c, float* host, size_t* nbytes) {
     at += e.count();
   }
   cudaFree(tmp);
+  c->mem_used -= mx * 4;
   *nbytes = total * 4;
   return st;
 }
@@ -1374,6 +1382,7 @@ wam_status wam_read_kv(wam_ctx* c, int block, int which, float* host, size_t* nb
   cudaError_t ce = launch_to_f32(which ? vcache(c, block) : kcache(c, block), d.bf16, tmp, n, 1, 1, 0);
   if (ce == cudaSuccess) ce = cudaMemcpy(host, tmp, n * 4, cudaMemcpyDeviceToHost);
   cudaFree(tmp);
+  c->mem_used -= n * 4;
   CK(ce);
   return WAM_OK;
 }

@@ -231,3 +231,24 @@ def test_argument_errors_enqueue_nothing():
         fresh.action_step(out, 1.0, 0.0)
     assert e.value.status == 6
     wam.check_device_status()
+
+
+def test_device_memory_limit_reports_oom(monkeypatch):
+    """A context whose allocations would pass WAM_DEVICE_MEMORY_LIMIT fails
+    with WAM_ERR_OOM before calling cudaMalloc, leaves *out NULL and releases
+    what it had allocated; the same config builds and runs without the limit."""
+    import ctypes as C
+    c = _mid()
+    monkeypatch.setenv("WAM_DEVICE_MEMORY_LIMIT", str(1 << 20))   # far below the model's weights
+    h = C.c_void_p()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        assert W.lib().wam_init(C.byref(c), 0, C.byref(h)) == 3 and not h.value
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] >= free0 - (64 << 20)   # nothing left behind
+    monkeypatch.delenv("WAM_DEVICE_MEMORY_LIMIT")
+    wam = W.Wam(c, seed=0)
+    inp = inputs(c, 0)
+    a0 = run_chunk(wam, inp, S=1)
+    assert np.isfinite(a0).all()
+    wam.close()

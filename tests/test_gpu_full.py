@@ -59,6 +59,8 @@ def test_batch8_sampled_elements(oracle_params):
     wam = W.Wam(c, seed=0)
     inp = inputs(c, 2)
     a0 = run_chunk(wam, inp, S=1, mode=W.CEWP, use_graph=True)
+    seq = run_chunk(wam, inp, S=1, mode=W.SEQUENTIAL, use_graph=True)
+    assert np.array_equal(a0, seq)   # the wavefront reordering is exact at this shape too
     oc1 = ocfg(c).with_(batch=1)
     for b in (0, 7):
         one = {k: (v[b:b + 1] if isinstance(v, np.ndarray) else v) for k, v in inp.items()}

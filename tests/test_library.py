@@ -140,3 +140,25 @@ def test_header_compiles_as_c_and_links_from_c():
     assert r.returncode == 0, r.stderr
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and "c abi ok" in r.stdout, r.stdout + r.stderr
+
+
+def test_noalloc_attention_refusals_without_a_device():
+    """wam_op_attention_noalloc checks its arguments and its scratch limits
+    before any CUDA call, so every refusal path runs on a host without a GPU
+    (the pointers are dummies that are never dereferenced)."""
+    L = W.lib()
+    p = C.c_void_p(0x1000)
+
+    def call(B=1, H=24, Lq=32, Lk=1120, Lc=1120, splits=9, ptrs=(p, p, p, p)):
+        return L.wam_op_attention_noalloc(*ptrs, B, H, Lq, Lk, Lc, splits, None)
+    assert call(splits=1) == 1                 # split-KV needs at least two splits
+    assert call(Lq=65) == 1                    # at most 64 queries per (sample, head)
+    assert call(Lq=0) == 1 and call(Lk=0) == 1 and call(B=0) == 1 and call(H=0) == 1
+    assert call(Lk=1121) == 1                  # keys beyond the cache rows
+    assert call(ptrs=(None, p, p, p)) == 1 and call(ptrs=(p, p, p, None)) == 1
+    assert call(Lk=64 * 33, Lc=64 * 33, splits=33) == 2     # 33 non-empty splits: more than the combine holds
+    assert call(B=8, H=64, Lq=64, Lk=128, Lc=128, splits=2) == 2   # 8*64*2 slots * 4224 floats > 2^21
+    # more (sample, head) pairs than the 1024 tickets: the partials' limit
+    # (at least two splits of 4224 floats each) already refuses beyond 248 pairs
+    assert call(B=1025, H=1, Lq=1, Lk=128, Lc=128, splits=2) == 2
+    assert call(B=248, H=1, Lq=1, Lk=128, Lc=128, splits=2, ptrs=(None, p, p, p)) == 1

@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 
 import mot_dit_b200 as W
+from oracle import model as M
 from oracle.params import round_bf16
 from wam_testlib import rel_l2
 
@@ -28,17 +29,25 @@ def _case(B, H, Lq, Lc, seed):
 
 
 def test_noalloc_attention_matches_allocating_entry_point_twice():
+    """Two calls in a row.  The second has fewer (sample, head, split) slots
+    than the first (24 against 216), so partials the first call left in the
+    shared scratch would show up if the second read any of them.  Both entry
+    points run the same kernel with the same split rule and a fixed-order
+    combine: their outputs are bitwise equal, and both match the oracle."""
     cases = [(1, 24, 32, 1120, 1120, 9, 0), (2, 4, 16, 300, 310, 3, 1)]
-    for B, H, Lq, Lk, Lc, splits, seed in cases:   # two calls in a row, different shapes
+    for B, H, Lq, Lk, Lc, splits, seed in cases:
         q, k, v = _case(B, H, Lq, Lc, seed)
         ref = torch.full((B * Lq, H * 64), float("nan"), device=DEV, dtype=torch.bfloat16)
         got = torch.full_like(ref, float("nan"))
         W.op_attention(W.BF16, q, k, v, ref, B, H, 64, Lq, Lk, Lc, splits=splits)
         W.op_attention_noalloc(q, k, v, got, B, H, Lq, Lk, Lc, splits)
         torch.cuda.synchronize()
-        r, g = ref.float().cpu().numpy(), got.float().cpu().numpy()
+        assert torch.equal(got, ref)
+        g = got.float().cpu().numpy()
         assert np.isfinite(g).all()
-        assert rel_l2(g, r) <= 1e-2
+        f64 = lambda t: t.float().cpu().numpy().astype(np.float64)
+        want = M.merge_heads(M.attention(f64(q), f64(k)[:, :, :Lk], f64(v)[:, :, :Lk])).reshape(B * Lq, H * 64)
+        assert rel_l2(g, want) <= 1e-2
 
 
 def test_noalloc_attention_refuses_beyond_its_scratch():
