@@ -24,6 +24,8 @@ Modules:
     model   -- float64 forward: video expert, action expert, Euler / endpoints
     tacd    -- TACD training targets, forward only: teacher K-step rollout,
                interval-average velocity, student / EMA endpoints, L_TA, L_CD
+    multistep -- chunk with a multi-step video expert: N_v Euler steps of the
+               video latents, the action expert on the last forward's K/V
 """
 from .config import WamConfig, preset  # noqa: F401
 from .params import generate_params, param_specs  # noqa: F401
