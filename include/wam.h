@@ -161,6 +161,53 @@ wam_status wam_joint_one_step(wam_ctx* ctx, const float* dev_video_clean, const 
                               float* dev_action_out, int mode, int use_graph, void* stream_video,
                               void* stream_action);
 
+/* Chunk with a multi-step video expert (RealtimeWAM summary page, 未来方向
+ * (2): the wavefront carried over to a video expert that keeps several
+ * denoising steps).  Requires video_patch_dim > 0 and video_has_output.
+ * The video latents start from dev_video_eps (level 1) and take n_video
+ * flow-matching Euler steps x <- x - (s_j - s_{j-1}) v^v(x, s_j) along
+ * host_sched_video (n_video + 1 levels falling from 1 to the last, within
+ * [0, 1]; NULL = uniform j / n_video), each a full forward of the video
+ * expert; the result x_0 goes to dev_video_out [B, l_video, video_patch_dim].
+ * The action expert then takes S Euler steps from dev_noise along
+ * host_t_sched (as in wam_infer_chunk) over the K/V of the LAST video forward:
+ * under WAM_SCHED_CEWP only that forward records the per-block events, and
+ * action block i's attention waits for video block i of it.  mode, use_graph
+ * and the streams as in wam_infer_chunk; 1 <= n_video, S <= 64. */
+wam_status wam_infer_chunk_multistep(wam_ctx* ctx, const float* dev_video_eps, const float* dev_noise,
+                                     float* dev_video_out, float* dev_actions_out, int n_video,
+                                     const float* host_sched_video, int S, const float* host_t_sched, int mode,
+                                     int use_graph, void* stream_video, void* stream_action);
+
+/* TACD target forward (Teacher-Anchored Consistency Distillation, forward
+ * only: the targets one training step of the action expert's LoRA is fitted
+ * to; RealtimeWAM summary page, sections 前置知识 "一致性蒸馏", 核心方法 and
+ * 方法步骤详情).  On `stream`, with device buffers:
+ *   a_t = (1 - t) a_clean + t eps;
+ *   the video expert once (t_v = 0) on dev_video / dev_cond, its K/V shared
+ *   by all three networks;
+ *   the frozen teacher -- the student's base weights, LoRA off -- runs K
+ *   Euler steps from (a_t, t) over the uniform grid t_k = t k / K down to 0:
+ *   a_0^T, and its first state a~_s at s = t (K - 1) / K;
+ *   the student (the LoRA model `student`) gives the endpoint
+ *   f(a_t, t) = a_t - t v, so v_student = (a_t - f) / t;
+ *   the EMA target (the LoRA model `ema`; it may be `student` itself) gives
+ *   f^-(a~_s, s) (for s = 0 the endpoint map is the identity);
+ *   u_TA = (a_t - a_0^T) / t, u_CD = (a_t - f^-) / t;
+ *   losses[0] = L_TA = E||v_student - u_TA||^2, losses[1] = L_CD =
+ *   E||v_student - u_CD||^2 (squared L2 over one sample's [l_action,
+ *   action_dim], mean over the batch), losses[2] = L_CD + lambda L_TA.
+ * dev_action_clean, dev_eps and the optional outputs dev_u_ta, dev_v_student,
+ * dev_u_cd, dev_a_t, dev_a0_teacher are [B, l_action, action_dim]; losses is
+ * 3 floats (required).  student and ema: contexts of the same config with
+ * lora_rank > 0 on one device; the EMA's K/V cache is overwritten with the
+ * student's.  0 < t <= 1, 1 <= K <= 64, else WAM_ERR_INVALID_ARG.  Buffers
+ * for the intermediate states are allocated in `student` on first use. */
+wam_status wam_tacd_targets(wam_ctx* student, wam_ctx* ema, const float* dev_video, const float* dev_cond,
+                            const float* dev_action_clean, const float* dev_eps, float t, int K, float lambda,
+                            float* dev_u_ta, float* dev_v_student, float* dev_u_cd, float* dev_losses,
+                            float* dev_a_t, float* dev_a0_teacher, void* stream);
+
 /* Copy every parameter, in generation order, as fp32 into host_buf (matrix
  * padding removed).  With host_buf == NULL only *nbytes is set.  Synchronous.
  * WAM_ERR_INVALID_ARG if *nbytes is too small. */
@@ -179,6 +226,17 @@ wam_status wam_read_kv(wam_ctx* ctx, int block, int which, float* host_buf, size
  * bounded waits (WAM_ERR_TIMEOUT, then clears the flag) or CUDA errors. */
 wam_status wam_check_device_status(wam_ctx* ctx);
 
+/* Failure-path test hook (tests only; every context of the process on the
+ * current device).  With extra > 0, the last piece of a split GEMM tile that
+ * is its CTA's final segment waits for `extra` more partial tiles than exist,
+ * giving up after limit_ns nanoseconds: the bounded wait runs out on a count
+ * nothing raises, the CTA winds down (its copies and MMAs drained, TMEM
+ * released), and wam_check_device_status then reports WAM_ERR_TIMEOUT and
+ * clears the tickets, so the next call is clean.  extra = 0 restores the
+ * normal wait (2 s limit, never reached).  Synchronous; call it outside
+ * stream capture.  No GPU fault is involved. */
+wam_status wam_test_peer_wait(int extra, unsigned long long limit_ns);
+
 /* Number of kernel launches one chunk enqueues for (S, mode) (graph or not). */
 int wam_chunk_kernel_count(wam_ctx* ctx, int S);
 
@@ -188,6 +246,7 @@ typedef enum {
   WAM_PROF_VIDEO_FFN_UP, WAM_PROF_VIDEO_FFN_DOWN, WAM_PROF_VIDEO_TEMB, WAM_PROF_VIDEO_IO,
   WAM_PROF_ACTION_NORM, WAM_PROF_ACTION_QKV, WAM_PROF_ACTION_ATTN, WAM_PROF_ACTION_OPROJ,
   WAM_PROF_ACTION_FFN_UP, WAM_PROF_ACTION_FFN_DOWN, WAM_PROF_ACTION_TEMB, WAM_PROF_ACTION_IO,
+  WAM_PROF_ACTION_BLOCK, /* persistent action-block launches (attention + R_i + next P_i, one per block) */
   WAM_PROF_CLASSES
 } wam_prof_class;
 
@@ -200,6 +259,28 @@ typedef enum {
  * count the whole projection; the fp32 path's QK-norm kernel is part of QKV.) */
 wam_status wam_profile_chunk(wam_ctx* ctx, const float* dev_video, const float* dev_cond, const float* dev_noise,
                              float* dev_actions_out, int S, void* stream, float* host_ms, int* host_counts);
+
+/* Kinds of wam_trace_chunk records. */
+typedef enum {
+  WAM_TRACE_START = 0,        /* chunk start (video stream) */
+  WAM_TRACE_VIDEO_KV = 1,     /* video block i's projection done: K^v_i / V^v_i published, e_i recorded */
+  WAM_TRACE_VIDEO_END = 2,    /* video block i's remainder done */
+  WAM_TRACE_ACTION_ATTN = 3,  /* action stream reaches Attn^a_i (after its wait on e_i) */
+  WAM_TRACE_ACTION_END = 4,   /* action block i done (its remainder, and the next block's projection on the
+                                 persistent path) */
+  WAM_TRACE_END = 5           /* chunk end (video stream, after the join) */
+} wam_trace_kind;
+
+/* Measurement of the wavefront: the chunk (S uniform steps, `mode`) captured
+ * into a CUDA graph with a timing event at every block boundary of both
+ * streams (the event nodes replace the dependent-launch overlap at those
+ * points), replayed once to warm up and once timed.  Writes up to `capacity`
+ * records of 4 floats (kind, block, Euler step, ms since the start record)
+ * into host_ms and the number of records into *count.  Synchronises
+ * stream_video.  Arguments otherwise as in wam_infer_chunk. */
+wam_status wam_trace_chunk(wam_ctx* ctx, const float* dev_video, const float* dev_cond, const float* dev_noise,
+                           float* dev_actions_out, int S, int mode, void* stream_video, void* stream_action,
+                           float* host_ms, int capacity, int* count);
 
 const char* wam_status_str(wam_status s);
 const char* wam_last_error(wam_ctx* ctx);

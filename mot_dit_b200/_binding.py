@@ -10,7 +10,9 @@ FP32, BF16 = 0, 1
 SEQUENTIAL, CEWP = 0, 1
 PROF_CLASSES = ("video_norm", "video_qkv", "video_attn", "video_oproj", "video_ffn_up", "video_ffn_down",
                 "video_temb", "video_io", "action_norm", "action_qkv", "action_attn", "action_oproj",
-                "action_ffn_up", "action_ffn_down", "action_temb", "action_io")
+                "action_ffn_up", "action_ffn_down", "action_temb", "action_io", "action_block")
+
+TRACE_KINDS = ("start", "video_kv", "video_end", "action_attn", "action_end", "end")
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "out of device memory", 4: "CUDA error",
            5: "device wait timed out", 6: "invalid call order"}
@@ -67,12 +69,17 @@ def lib():
         "wam_infer_chunk_host": (C.c_int, [_P, _P, _P, _P, _P, C.c_int, _F, C.c_int, C.c_int, _P, _P]),
         "wam_joint_one_step": (C.c_int, [_P, _P, _P, _P, _P, C.c_float, C.c_float, C.c_float, C.c_float, _P, _P,
                                          C.c_int, C.c_int, _P, _P]),
+        "wam_infer_chunk_multistep": (C.c_int, [_P, _P, _P, _P, _P, C.c_int, _F, C.c_int, _F, C.c_int, C.c_int, _P,
+                                                _P]),
+        "wam_tacd_targets": (C.c_int, [_P, _P, _P, _P, _P, _P, C.c_float, C.c_int, C.c_float] + [_P] * 6 + [_P]),
         "wam_export_params": (C.c_int, [_P, _P, C.POINTER(C.c_size_t)]),
         "wam_import_params": (C.c_int, [_P, _P, C.c_size_t]),
         "wam_read_kv": (C.c_int, [_P, C.c_int, C.c_int, _P, C.POINTER(C.c_size_t)]),
         "wam_check_device_status": (C.c_int, [_P]),
         "wam_chunk_kernel_count": (C.c_int, [_P, C.c_int]),
         "wam_profile_chunk": (C.c_int, [_P, _P, _P, _P, _P, C.c_int, _P, _P, _P]),
+        "wam_trace_chunk": (C.c_int, [_P, _P, _P, _P, _P, C.c_int, C.c_int, _P, _P, _P, C.c_int, _P]),
+        "wam_test_peer_wait": (C.c_int, [C.c_int, C.c_uint64]),
         "wam_status_str": (C.c_char_p, [C.c_int]),
         "wam_last_error": (C.c_char_p, [_P]),
         "wam_op_linear": (C.c_int, [C.c_int, _P, _P, _P, _P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _P]),
@@ -226,6 +233,34 @@ class Wam:
             shift_video, shift_action, _io(video_out, nv, w, "video_out"), _io(action_out, na, w, "action_out"),
             mode, int(use_graph), _stream(stream_video), _stream(stream_action)), w)
 
+    def infer_chunk_multistep(self, video_eps, noise, video_out, actions_out, n_video=1, sched_video=None, S=1,
+                              t_sched=None, mode=CEWP, use_graph=True, stream_video=None, stream_action=None):
+        w = "wam_infer_chunk_multistep"
+        nv, _, na = self.io_sizes()
+        _check_sched(sched_video, n_video, w)
+        _check_sched(t_sched, S, w)
+        pv, keep_v = _sched(sched_video)
+        pa, keep_a = _sched(t_sched)
+        self._check(self._lib.wam_infer_chunk_multistep(
+            self._h, _io(video_eps, nv, w, "video_eps"), _io(noise, na, w, "noise"), _io(video_out, nv, w, "video_out"),
+            _io(actions_out, na, w, "actions_out"), n_video, pv, S, pa, mode, int(use_graph), _stream(stream_video),
+            _stream(stream_action)), w)
+        del keep_v, keep_a
+
+    def tacd_targets(self, ema, video, cond, action_clean, eps, t, K, lam, u_ta, v_student, u_cd, losses,
+                     a_t=None, a0_teacher=None, stream=None):
+        """TACD target forward (wam_tacd_targets): this context is the student
+        (its base weights are the teacher), `ema` the EMA target (may be self)."""
+        w = "wam_tacd_targets"
+        nv, nc, na = self.io_sizes()
+        ema_h = ema._h if ema is not None else None
+        self._check(self._lib.wam_tacd_targets(
+            self._h, ema_h, _io(video, nv, w, "video"), _io(cond, nc, w, "cond"),
+            _io(action_clean, na, w, "action_clean"), _io(eps, na, w, "eps"), t, K, lam,
+            _io(u_ta, na, w, "u_ta"), _io(v_student, na, w, "v_student"), _io(u_cd, na, w, "u_cd"),
+            _io(losses, 3, w, "losses"), _io(a_t, na, w, "a_t"), _io(a0_teacher, na, w, "a0_teacher"),
+            _stream(stream)), w)
+
     def export_params(self) -> np.ndarray:
         n = C.c_size_t(0)
         self._check(self._lib.wam_export_params(self._h, None, C.byref(n)), "wam_export_params")
@@ -250,6 +285,19 @@ class Wam:
 
     def chunk_kernel_count(self, S: int) -> int:
         return self._lib.wam_chunk_kernel_count(self._h, S)
+
+    def trace_chunk(self, video, cond, noise, out, S=1, mode=CEWP, stream_video=None, stream_action=None):
+        """Block-boundary timestamps of one graph-replayed chunk: a list of
+        (kind, block, step, ms) with kind in TRACE_KINDS."""
+        w = "wam_trace_chunk"
+        ptrs = self._chunk_ptrs(w, video, cond, noise, out)
+        cap = 8 * (self.cfg.n_blocks + 2) * (S + 1)
+        buf = np.zeros(4 * cap, np.float32)
+        n = C.c_int(0)
+        self._check(self._lib.wam_trace_chunk(self._h, *ptrs, S, mode, _stream(stream_video), _stream(stream_action),
+                                              buf.ctypes.data, cap, C.byref(n)), w)
+        rec = buf[:4 * min(n.value, cap)].reshape(-1, 4)
+        return [(TRACE_KINDS[int(k)], int(b), int(j), float(t)) for k, b, j, t in rec]
 
     def profile_chunk(self, video, cond, noise, out, S=1, stream=None):
         """Per-class summed launch durations (ms) and launch counts of one eager

@@ -39,6 +39,14 @@ __device__ __forceinline__ void epi_elem_f32(const EpiArgs& e, int m, int n, flo
       e.vio->video_out[idx] = cs * xs + co * (xs - sigma * y);
       break;
     }
+    case kEpiVideoEuler: {
+      const float ds = e.vio->vsched[e.step] - e.vio->vsched[e.step + 1];
+      const float xn = e.out_f32[idx] - ds * y;
+      e.out_f32[idx] = xn;
+      if (e.out_act) reinterpret_cast<float*>(e.out_act)[(size_t)m * e.a_next_ld + n] = xn;
+      if (e.step == e.vio->vsteps - 1) e.vio->video_out[idx] = xn;
+      break;
+    }
     default:
       break;
   }

@@ -143,13 +143,22 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // Later async-proxy reads of global memory see what this thread has observed.
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
+// Failure-path test hook (wam_test_peer_wait): the last piece of a split tile
+// that is its CTA's final segment waits for g_peer_wait_extra more published
+// partials than exist, with the limit g_peer_wait_limit_ns, so that the
+// bounded wait gives up on a flag nothing sets.  Zero / kWaitLimitNs (the
+// defaults) leave the kernel as it is.
+__device__ int g_peer_wait_extra = 0;
+__device__ unsigned long long g_peer_wait_limit_ns = kWaitLimitNs;
+
 // Bounded wait until *count >= target (a counter other CTAs increment).
-__device__ __forceinline__ bool wait_count(const int* count, int target, unsigned* status, volatile int* abort) {
+__device__ __forceinline__ bool wait_count(const int* count, int target, unsigned* status, volatile int* abort,
+                                           unsigned long long limit_ns = kWaitLimitNs) {
   const volatile int* vc = count;
   const unsigned long long t0 = globaltimer();
   while (*vc < target) {
     if (abort && *abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       atomicOr(status, kStatusTimeoutPeer);
       return false;
     }
@@ -317,6 +326,14 @@ __device__ __forceinline__ void epi_elem(const EpiArgs& e, int m, int n, float y
       const float cs = 0.25f / (s2 + 0.25f), co = sigma * 0.5f / sqrtf(s2 + 0.25f);
       const float xs = e.x_sigma[idx];
       e.vio->video_out[idx] = cs * xs + co * (xs - sigma * y);
+      break;
+    }
+    case kEpiVideoEuler: {
+      const float ds = e.vio->vsched[e.step] - e.vio->vsched[e.step + 1];
+      const float xn = e.out_f32[idx] - ds * y;
+      e.out_f32[idx] = xn;
+      if (e.out_act) reinterpret_cast<__nv_bfloat16*>(e.out_act)[(size_t)m * e.a_next_ld + n] = __float2bfloat16_rn(xn);
+      if (e.step == e.vio->vsteps - 1) e.vio->video_out[idx] = xn;
       break;
     }
     default:
@@ -697,7 +714,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // the last arrival reduces: the others have arrived; wait until they have published
         if (threadIdx.x == 64) {
-          if (!wait_count(g.tickets + 2 * t + 1, npieces - 1, g.status, abort_flag)) {
+          const bool hooked = x == x_end && g_peer_wait_extra > 0;
+          if (!wait_count(g.tickets + 2 * t + 1, npieces - 1 + (hooked ? g_peer_wait_extra : 0), g.status, abort_flag,
+                          hooked ? g_peer_wait_limit_ns : kWaitLimitNs)) {
             *abort_flag = 1;
           } else {
             g.tickets[2 * t] = 0;  // every piece is done with the tickets
@@ -1160,6 +1179,12 @@ cudaError_t prepare_tc_gemm() {
   WAM_PREP(256, false, kClassRes)
 #undef WAM_PREP
   return cudaSuccess;
+}
+
+cudaError_t set_peer_wait_test(int extra, unsigned long long limit_ns) {
+  cudaError_t e = cudaMemcpyToSymbol(g_peer_wait_extra, &extra, sizeof extra);
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_peer_wait_limit_ns, &limit_ns, sizeof limit_ns);
+  return e;
 }
 
 cudaError_t launch_tc_gemm(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {

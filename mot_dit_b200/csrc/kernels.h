@@ -43,6 +43,8 @@ struct VideoIo {
   float t;              // video timestep (noise level) of the chunk
   float u;              // joint variant: unshifted level; shift applied on device
   float shift;          // joint variant: SNR shift s_v (0: use t as is)
+  float vsched[65];     // multi-step video: noise levels s_{N_v} > ... > s_0 of the video Euler steps
+  int vsteps;           // multi-step video: N_v (0: one pass)
 };
 struct ActionIo {
   const float* a_in;    // chunk start [B, L_a, P_a] (noise, or the caller's state)
@@ -62,6 +64,9 @@ enum Epi : int {
   kEpiEuler = 4,     // a[m, n] -= (t_j - t_{j-1}) * (acc + bias[n]); also writes the next in-proj input
   kEpiVideoOut = 5,  // joint variant: video endpoint f^v = c_skip x + c_out (x - sigma v)
   kEpiScaleAct = 6,  // out_act[m, n] = scale * (acc + bias[n]) (act dtype): the LoRA down-projection s x A^T
+  kEpiVideoEuler = 7,  // multi-step video: x[m, n] -= (s_j - s_{j-1}) (acc + bias[n]) into out_f32 (the latents),
+                       // also the next in-projection input out_act (ld a_next_ld) and, after the last step,
+                       // the chunk's video vio->video_out
 };
 
 struct EpiArgs {
@@ -130,6 +135,8 @@ size_t tc_gemm_ws_floats(const TcGemm& g);
 int tc_gemm_ring_partials(int bn, bool swap, bool fused_norm);
 
 cudaError_t launch_tc_gemm(const TcGemm& g, const EpiArgs& e, cudaStream_t s);
+// Failure-path test hook of the split-tile wait (0, kWaitLimitNs: off).
+cudaError_t set_peer_wait_test(int extra, unsigned long long limit_ns);
 // Sets the kernels' shared-memory attributes; call once per device before any
 // launch (and never during stream capture).
 cudaError_t prepare_tc_gemm();
@@ -219,6 +226,84 @@ cudaError_t launch_gen_param(uint64_t seed, uint64_t pid, size_t count, double s
 cudaError_t launch_rope_table(float* cos_t, float* sin_t, int L, int Dh, cudaStream_t s);
 // dst[e] = src[(e / cols) * ld + e % cols] as fp32.
 cudaError_t launch_to_f32(const void* src, bool src_bf16, float* dst, size_t n, int cols, int ld, cudaStream_t s);
+
+// ---- persistent action-expert block (action_block.cu) -------------------
+// One launch = [attention of block i,] then up to five weight GEMM phases
+// (out-projection, FFN up, FFN down, next block's QKV or the output map; or
+// in-projection + QKV of block 0), separated by grid barriers.  Batches of at
+// most 32 action tokens, bf16.
+enum : int { kBTma = 0, kBNorm = 1 };  // B operand: TMA of an activation map / RMSNorm+modulation of x_a
+constexpr int kActionBlockMaps = 11;
+// Tensor maps: 0 w_qkv, 1 w_o, 2 w_f1, 3 w_f2 (3-D, z = block), 4 w_in, 5 w_out,
+// 6 o_a, 7 f_a, 8 a_in (box 64 x 32 rows), 9 q_a and 10 the K/V cache (box 64 x 128 rows).
+struct ActionBlockMaps {
+  CUtensorMap m[kActionBlockMaps];
+};
+// C[token m, feature n] = sum_k X[m, k] W[n, k] over W [n_out, K] (matrix z
+// of map map_w), split into ks k-ranges per 128-row tile; B = X from map
+// map_b (kBTma) or rms(x_a) * (ngain | 1 + nscale) + nshift (kBNorm).
+struct ActionGemmPhase {
+  int map_w, z, n_out, K, ks;
+  int bsrc, map_b;
+  const float* nscale;
+  const float* nshift;
+  const float* ngain;
+  int epi;  // kEpiStoreF32 / kEpiGateRes / kEpiGelu / kEpiQkv / kEpiEuler
+  const float* bias;
+  const float* gate;
+  float* out_f32;
+  __nv_bfloat16* out_act;
+  int ld_out;
+  const float* gq;         // QKV: per-head norm gains [A]
+  const float* gk;
+  __nv_bfloat16* q_out;    // [B, H, L_a, 64]
+  __nv_bfloat16* k_cache;  // block base [B, H, L_tot, 64]
+  __nv_bfloat16* v_cache;
+  int step;                // Euler: step index into the schedule
+  __nv_bfloat16* a_next;   // Euler: next in-projection input (ld a_next_ld)
+  int a_next_ld;
+};
+struct ActionAttnPhase {
+  int zk0, zv0;        // cache-map matrix index of (b = 0, h = 0) of K / V
+  int splits;          // 128-key splits of [0, Lk)
+  __nv_bfloat16* out;  // o_a [B * L_a, ld_out]
+  int ld_out;
+};
+struct ActionBlockArgs {
+  int n_gemm, has_attn;
+  ActionGemmPhase g[5];
+  ActionAttnPhase at;
+  int Ma, La, H, A, da, Lk, cache_len, cache_off, B;
+  const float* x_a;  // fp32 [Ma, da]
+  const float* rope_cos;
+  const float* rope_sin;
+  const ActionIo* aio;
+  float* ws;       // GEMM partial tiles: action_block_ws_floats
+  float* ws_attn;  // attention partials: action_block_attn_ws_floats
+  int* cnt;        // 2 * 64 ints, zero on entry, left zero
+  int* cnt_attn;   // 2 * B * H ints, zero on entry, left zero
+  int* bar;        // grid barrier (count, generation), zero at first use
+  unsigned* status;
+};
+// k-splits of a phase with n_out weight rows and reduction K on nsm SMs
+// (fixed by the shapes, never by the grid size).
+int action_block_ks(int n_out, int K, int nsm);
+// Whether every CTA of a `ctas` grid holds the B k-blocks it needs.
+bool action_block_fits(int n_out, int K, int ks, int ctas);
+size_t action_block_ws_floats(int max_units);
+size_t action_block_attn_ws_floats(int B, int H, int splits);
+int action_block_attn_splits(int Lk);
+cudaError_t prepare_action_block();
+// `ctas` <= the SM count (one CTA per SM: the grid barriers need the whole grid resident).
+cudaError_t launch_action_block(const ActionBlockMaps& m, const ActionBlockArgs& a, int ctas, cudaStream_t s);
+
+// TACD target forward: a_t = (1 - t) a_clean + t eps; and the targets
+// u_TA, v_student, u_CD (any may be null) plus losses[3] = L_TA, L_CD,
+// L_CD + lambda L_TA from the teacher end state, the student and EMA endpoints.
+cudaError_t launch_tacd_noise(const float* a_clean, const float* eps, float t, float* a_t, int n, cudaStream_t s);
+cudaError_t launch_tacd_targets(const float* a_t, const float* a0_teacher, const float* f_student,
+                                const float* f_ema, float t, float lambda, int B, int per_sample, float* u_ta,
+                                float* v_student, float* u_cd, float* losses, cudaStream_t s);
 
 // TMA tensor-map creation (driver entry point resolved at run time).
 bool make_tmap_3d(CUtensorMap* map, const void* base, int K, int rows, int nmat, size_t mat_stride_bytes,

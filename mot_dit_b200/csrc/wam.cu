@@ -15,6 +15,8 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
+#include <initializer_list>
 #include <map>
 #include <memory>
 #include <string>
@@ -88,6 +90,7 @@ struct wam_ctx {
   int* tk_gemm = nullptr;
   float* ws_gemm_v = nullptr;  // video-stream GEMM partial tiles / tickets (the streams overlap)
   int* tk_gemm_v = nullptr;
+  size_t tk_gemm_bytes = 0, tk_gemm_v_bytes = 0;
   float* ws_attn = nullptr;
   int* tk_attn = nullptr;
   unsigned* status = nullptr;
@@ -98,6 +101,10 @@ struct wam_ctx {
   bool vio_valid = false, aio_valid = false;
   float *h_video = nullptr, *h_cond = nullptr, *h_noise = nullptr, *h_out = nullptr;  // host-API staging
   float *j_vout = nullptr, *j_aout = nullptr;
+  // TACD target forward (allocated on first use): a_t, teacher state at s,
+  // teacher end state, student and EMA endpoints; the schedule block of its runs
+  float *td_at = nullptr, *td_as = nullptr, *td_a0 = nullptr, *td_fs = nullptr, *td_fe = nullptr;
+  ActionIo* aio_tacd = nullptr;
 
   // plans
   GemmPlan p_v_qkv, p_v_o, p_v_f1, p_v_f2, p_v_in, p_v_out;
@@ -107,12 +114,22 @@ struct wam_ctx {
   // The action expert's norms run inside the GEMM that consumes them (opt-in;
   // the tokens must fit one 32/64-wide tile and K <= 1024).
   bool fuse_norm_a = false;
+  // Persistent action-block path (action_block.cu): one launch per action
+  // block; grid sizes for launches that may overlap the video expert (CEWP
+  // first step, eager action steps) and for the rest.
+  bool ab_on = false;
+  int ab_ctas = 0, ab_ctas_overlap = 0;
+  int ab_ks_in = 1, ab_ks_qkv = 1, ab_ks_o = 1, ab_ks_f1 = 1, ab_ks_f2 = 1, ab_ks_out = 1, ab_splits = 1;
+  ActionBlockMaps ab_maps;
+  float *ab_ws = nullptr, *ab_ws_attn = nullptr;
+  int *ab_cnt = nullptr, *ab_cnt_attn = nullptr, *ab_bar = nullptr;
 
   // TMA maps
   CUtensorMap m_hv, m_ov, m_fv, m_xvin, m_w_qkv_v, m_w_o_v, m_w_f1_v, m_w_f2_v, m_w_vin, m_w_vout;
   CUtensorMap m_w_in, m_w_qkv_a, m_w_o_a, m_w_f1_a, m_w_f2_a, m_w_out, m_ain, m_ha, m_oa, m_fa;
   CUtensorMap m_la_qkv, m_la_o, m_la_f1, m_la_f2;  // LoRA A factors [r, in] per block
   CUtensorMap m_qv, m_cache;  // video-attention operands
+  CUtensorMap m_qa128, m_cache128;  // action-block attention operands (128-row boxes)
   // video GEMM outputs (TMA stores, 32-row boxes): x_v fp32, f_v bf16, Q, the K/V cache
   CUtensorMap m_xv_out, m_fv_out, m_qv_out, m_cache_out;
 
@@ -138,6 +155,16 @@ struct wam_ctx {
   std::vector<ProfRec> prof;
   std::vector<cudaEvent_t> prof_pool;
   size_t prof_next = 0;
+
+  // wavefront trace (wam_trace_chunk): timing events at block boundaries
+  bool trace_on = false;
+  struct TraceRec {
+    int kind, block, step;
+    cudaEvent_t e;
+  };
+  std::vector<TraceRec> trace;
+  std::vector<cudaEvent_t> trace_pool;
+  int trace_step = 0;
 };
 
 namespace {
@@ -183,6 +210,20 @@ struct ProfScope {
     if (b) cudaEventRecordWithFlags(b, s, cudaEventRecordExternal);
   }
 };
+
+// Records a timing event of `kind` for block i on stream s when the context is
+// tracing (wam_trace_chunk); a no-op otherwise.
+void trace_mark(wam_ctx* c, cudaStream_t s, int kind, int i) {
+  if (!c->trace_on) return;
+  if (c->trace.size() >= c->trace_pool.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return;
+    c->trace_pool.push_back(e);
+  }
+  cudaEvent_t e = c->trace_pool[c->trace.size()];
+  cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  c->trace.push_back({kind, i, c->trace_step, e});
+}
 
 // ------------------------------------------------------------ parameters --
 void add_expert(wam_ctx* c, bool video) {
@@ -542,25 +583,12 @@ wam_status norm_linear(wam_ctx* c, const Lin& L, EpiArgs e, const float* sc, con
 
 // ------------------------------------------------------------- experts ----
 // Video expert: P^v_i -> record(e_i) -> Attn^v_i -> R^v_i for every block.
-wam_status enqueue_video(wam_ctx* c, cudaStream_t s, const VideoIo* io, bool joint, cudaEvent_t* ev_ready,
-                         bool war_waits) {
+// The video expert's N DiT blocks on x_v at the modulation in mod_v:
+// P^v_i -> record(e_i) -> Attn^v_i -> R^v_i.
+wam_status enqueue_video_blocks(wam_ctx* c, cudaStream_t s, cudaEvent_t* ev_ready, bool war_waits) {
   const Dims& d = c->d;
   const ExpertIdx& x = c->ev;
   const bool has_out = c->cfg.video_has_output != 0;
-  c->cur_cls = WAM_PROF_VIDEO_IO;
-  if (joint) {
-    c->launches++;
-    ProfScope ps(c, s);
-    CK(launch_noise_video(io, c->x_sigma, d.bf16 ? c->x_vin : c->x_sigma, d.bf16, d.Mv, d.Pv, d.Pv, s));
-    Lin L{&c->m_w_vin, &c->m_xvin, matp(c, x.inw), c->x_sigma, d.dv, d.Pv, 0, &c->p_v_in};
-    RET(linear(c, true, L, d.Mv, epi_base(kEpiStoreF32, vecp(c, x.inb), c->x_v, nullptr, d.dv), nullptr, s));
-  } else {
-    c->launches++;
-    ProfScope ps(c, s);
-    CK(launch_init_video(io, c->x_v, d.B, d.Lc, d.Lvid, d.dv, s));
-  }
-  c->cur_cls = WAM_PROF_VIDEO_TEMB;
-  RET(temb(c, true, &io->t, s));
   for (int i = 0; i < d.N; ++i) {
     const float* mod = c->mod_v + (size_t)i * 6 * d.dv;
     if (war_waits) CK(cudaStreamWaitEvent(s, c->ev_used[i], 0));
@@ -569,6 +597,9 @@ wam_status enqueue_video(wam_ctx* c, cudaStream_t s, const VideoIo* io, bool joi
     c->cur_cls = WAM_PROF_VIDEO_QKV;
     Lin Lq{&c->m_w_qkv_v, &c->m_hv, matp(c, blk(x, i, kQkvW)), c->h_v, 3 * d.A, d.dv, i, &c->p_v_qkv};
     RET(linear(c, true, Lq, d.Mv, epi_qkv(c, true, i), c->qkv_tmp_v, s));
+    // (the trace mark first: an action-side mark after the wait on e_i then
+    // depends on it, so the recorded order is the schedule's)
+    trace_mark(c, s, WAM_TRACE_VIDEO_KV, i);
     if (ev_ready) CK(cudaEventRecord(ev_ready[i], s));
     if (i == d.N - 1 && !has_out) break;
     c->cur_cls = WAM_PROF_VIDEO_ATTN;
@@ -588,15 +619,57 @@ wam_status enqueue_video(wam_ctx* c, cudaStream_t s, const VideoIo* io, bool joi
     e2.gate = mod + 5 * d.dv;
     Lin L2{&c->m_w_f2_v, &c->m_fv, matp(c, blk(x, i, kF2W)), c->f_v, d.dv, d.Fv, i, &c->p_v_f2};
     RET(linear(c, true, L2, d.Mv, e2, nullptr, s));
+    trace_mark(c, s, WAM_TRACE_VIDEO_END, i);
   }
-  if (joint) {
-    c->cur_cls = WAM_PROF_VIDEO_IO;
-    RET(norm(c, c->x_v, c->h_v, d.Mv, d.dv, nullptr, nullptr, vecp(c, x.fng), s));
-    EpiArgs eo = epi_base(kEpiVideoOut, vecp(c, x.outb), nullptr, nullptr, d.Pv);
-    eo.vio = io;
-    eo.x_sigma = c->x_sigma;
-    Lin Lout{&c->m_w_vout, &c->m_hv, matp(c, x.outw), c->h_v, d.Pv, d.dv, 0, &c->p_v_out};
-    RET(linear(c, true, Lout, d.Mv, eo, nullptr, s));
+  return WAM_OK;
+}
+
+// Video expert: P^v_i -> record(e_i) -> Attn^v_i -> R^v_i for every block.
+// n_video > 0: the multi-step video expert -- the patch latents start at
+// io->video scaled by the level io->t (1: pure noise), then n_video passes,
+// each one forward at level io->vsched[j] followed by the Euler step of the
+// latents; only the last pass publishes e_i (the action expert reads its
+// K/V), only the first waits for the previous chunk's consumption events.
+wam_status enqueue_video(wam_ctx* c, cudaStream_t s, const VideoIo* io, bool joint, cudaEvent_t* ev_ready,
+                         bool war_waits, int n_video = 0) {
+  const Dims& d = c->d;
+  const ExpertIdx& x = c->ev;
+  c->cur_cls = WAM_PROF_VIDEO_IO;
+  if (joint || n_video > 0) {
+    c->launches++;
+    ProfScope ps(c, s);
+    CK(launch_noise_video(io, c->x_sigma, d.bf16 ? c->x_vin : c->x_sigma, d.bf16, d.Mv, d.Pv, d.Pv, s));
+  } else {
+    c->launches++;
+    ProfScope ps(c, s);
+    CK(launch_init_video(io, c->x_v, d.B, d.Lc, d.Lvid, d.dv, s));
+  }
+  const int passes = n_video > 0 ? n_video : 1;
+  for (int j = 0; j < passes; ++j) {
+    if (joint || n_video > 0) {
+      c->cur_cls = WAM_PROF_VIDEO_IO;
+      Lin L{&c->m_w_vin, &c->m_xvin, matp(c, x.inw), c->x_sigma, d.dv, d.Pv, 0, &c->p_v_in};
+      RET(linear(c, true, L, d.Mv, epi_base(kEpiStoreF32, vecp(c, x.inb), c->x_v, nullptr, d.dv), nullptr, s));
+    }
+    c->cur_cls = WAM_PROF_VIDEO_TEMB;
+    RET(temb(c, true, n_video > 0 ? &io->vsched[j] : &io->t, s));
+    RET(enqueue_video_blocks(c, s, j == passes - 1 ? ev_ready : nullptr, war_waits && j == 0));
+    if (joint || n_video > 0) {
+      c->cur_cls = WAM_PROF_VIDEO_IO;
+      RET(norm(c, c->x_v, c->h_v, d.Mv, d.dv, nullptr, nullptr, vecp(c, x.fng), s));
+      EpiArgs eo;
+      if (n_video > 0) {
+        eo = epi_base(kEpiVideoEuler, vecp(c, x.outb), c->x_sigma, d.bf16 ? c->x_vin : nullptr, d.Pv);
+        eo.step = j;
+        eo.a_next_ld = d.Pv;
+      } else {
+        eo = epi_base(kEpiVideoOut, vecp(c, x.outb), nullptr, nullptr, d.Pv);
+        eo.x_sigma = c->x_sigma;
+      }
+      eo.vio = io;
+      Lin Lout{&c->m_w_vout, &c->m_hv, matp(c, x.outw), c->h_v, d.Pv, d.dv, 0, &c->p_v_out};
+      RET(linear(c, true, Lout, d.Mv, eo, nullptr, s));
+    }
   }
   return WAM_OK;
 }
@@ -609,9 +682,139 @@ void lora(wam_ctx* c, Lin& L, int i, int local, const CUtensorMap* map, const Ge
   L.plan_u = plan;
 }
 
+// ---- persistent action-block path
+ActionBlockArgs ab_base(wam_ctx* c, const ActionIo* io) {
+  const Dims& d = c->d;
+  ActionBlockArgs a{};
+  a.Ma = d.Ma;
+  a.La = d.La;
+  a.H = d.H;
+  a.A = d.A;
+  a.da = d.da;
+  a.Lk = d.Lv + d.La;
+  a.cache_len = d.Ltot;
+  a.cache_off = d.Lv;
+  a.B = d.B;
+  a.x_a = c->x_a;
+  a.rope_cos = c->rope_cos;
+  a.rope_sin = c->rope_sin;
+  a.aio = io;
+  a.ws = c->ab_ws;
+  a.ws_attn = c->ab_ws_attn;
+  a.cnt = c->ab_cnt;
+  a.cnt_attn = c->ab_cnt_attn;
+  a.bar = c->ab_bar;
+  a.status = c->status;
+  return a;
+}
+
+ActionGemmPhase ab_gemm(int map_w, int z, int n_out, int K, int ks, int bsrc, int map_b, int epi, const float* bias) {
+  ActionGemmPhase g{};
+  g.map_w = map_w;
+  g.z = z;
+  g.n_out = n_out;
+  g.K = K;
+  g.ks = ks;
+  g.bsrc = bsrc;
+  g.map_b = map_b;
+  g.epi = epi;
+  g.bias = bias;
+  return g;
+}
+
+// P^a_i: norm1 (AdaLN of block i) + merged QKV + QK-norm + RoPE + K/V publish.
+ActionGemmPhase ab_qkv(wam_ctx* c, int i) {
+  const Dims& d = c->d;
+  const ExpertIdx& x = c->ea;
+  const float* mod = c->mod_a + (size_t)i * 6 * d.da;
+  ActionGemmPhase g = ab_gemm(0, i, 3 * d.A, d.da, c->ab_ks_qkv, kBNorm, 0, kEpiQkv, vecp(c, blk(x, i, kQkvB)));
+  g.nscale = mod + d.da;
+  g.nshift = mod;
+  g.gq = vecp(c, blk(x, i, kQnG));
+  g.gk = vecp(c, blk(x, i, kKnG));
+  g.q_out = reinterpret_cast<__nv_bfloat16*>(c->q_a);
+  g.k_cache = reinterpret_cast<__nv_bfloat16*>(kcache(c, i));
+  g.v_cache = reinterpret_cast<__nv_bfloat16*>(vcache(c, i));
+  return g;
+}
+
+wam_status ab_launch(wam_ctx* c, const ActionBlockArgs& a, int ctas, cudaStream_t s) {
+  c->launches++;
+  c->cur_cls = WAM_PROF_ACTION_BLOCK;
+  ProfScope ps(c, s);
+  CK(launch_action_block(c->ab_maps, a, ctas, s));
+  return WAM_OK;
+}
+
+// One Euler step on the persistent path: [in-proj, P^a_0], then for every
+// block i: wait(e_i) -> [Attn^a_i, R^a_i, P^a_{i+1} | output map + Euler].
+wam_status enqueue_action_step_blocks(wam_ctx* c, cudaStream_t s, const ActionIo* io, int j,
+                                      const cudaEvent_t* ev_wait, bool record_used) {
+  const Dims& d = c->d;
+  const ExpertIdx& x = c->ea;
+  c->cur_cls = WAM_PROF_ACTION_TEMB;
+  RET(temb(c, false, &io->sched[j], s));
+  // launches that may run beside the video expert take the SMs it leaves free
+  const int ctas = ev_wait ? c->ab_ctas_overlap : c->ab_ctas;
+  {
+    ActionBlockArgs a = ab_base(c, io);
+    ActionGemmPhase in = ab_gemm(4, 0, d.da, d.Kin, c->ab_ks_in, kBTma, 8, kEpiStoreF32, vecp(c, x.inb));
+    in.out_f32 = c->x_a;
+    in.ld_out = d.da;
+    a.g[a.n_gemm++] = in;
+    a.g[a.n_gemm++] = ab_qkv(c, 0);
+    RET(ab_launch(c, a, ctas, s));
+  }
+  for (int i = 0; i < d.N; ++i) {
+    const float* mod = c->mod_a + (size_t)i * 6 * d.da;
+    if (ev_wait) CK(cudaStreamWaitEvent(s, ev_wait[i], 0));
+    trace_mark(c, s, WAM_TRACE_ACTION_ATTN, i);
+    ActionBlockArgs a = ab_base(c, io);
+    a.has_attn = 1;
+    a.at.zk0 = (2 * i) * d.B * d.H;
+    a.at.zv0 = (2 * i + 1) * d.B * d.H;
+    a.at.splits = c->ab_splits;
+    a.at.out = reinterpret_cast<__nv_bfloat16*>(c->o_a);
+    a.at.ld_out = d.lo;
+    ActionGemmPhase o = ab_gemm(1, i, d.da, d.A, c->ab_ks_o, kBTma, 6, kEpiGateRes, vecp(c, blk(x, i, kOB)));
+    o.gate = mod + 2 * d.da;
+    o.out_f32 = c->x_a;
+    o.ld_out = d.da;
+    a.g[a.n_gemm++] = o;
+    ActionGemmPhase f1 = ab_gemm(2, i, d.Fa, d.da, c->ab_ks_f1, kBNorm, 0, kEpiGelu, vecp(c, blk(x, i, kF1B)));
+    f1.nscale = mod + 4 * d.da;
+    f1.nshift = mod + 3 * d.da;
+    f1.out_act = reinterpret_cast<__nv_bfloat16*>(c->f_a);
+    f1.ld_out = d.lf;
+    a.g[a.n_gemm++] = f1;
+    ActionGemmPhase f2 = ab_gemm(3, i, d.da, d.Fa, c->ab_ks_f2, kBTma, 7, kEpiGateRes, vecp(c, blk(x, i, kF2B)));
+    f2.gate = mod + 5 * d.da;
+    f2.out_f32 = c->x_a;
+    f2.ld_out = d.da;
+    a.g[a.n_gemm++] = f2;
+    if (i + 1 < d.N) {
+      a.g[a.n_gemm++] = ab_qkv(c, i + 1);
+    } else {
+      ActionGemmPhase out = ab_gemm(5, 0, d.Pa, d.da, c->ab_ks_out, kBNorm, 0, kEpiEuler, vecp(c, x.outb));
+      out.ngain = vecp(c, x.fng);
+      out.out_f32 = c->a_state;
+      out.ld_out = d.Pa;
+      out.step = j;
+      out.a_next = reinterpret_cast<__nv_bfloat16*>(c->a_in);
+      out.a_next_ld = d.Kin;
+      a.g[a.n_gemm++] = out;
+    }
+    RET(ab_launch(c, a, ctas, s));
+    trace_mark(c, s, WAM_TRACE_ACTION_END, i);
+    if (record_used) CK(cudaEventRecord(c->ev_used[i], s));
+  }
+  return WAM_OK;
+}
+
 // One Euler step j of the action expert: P^a_i -> wait(e_i) -> Attn^a_i -> R^a_i.
 wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, int j, const cudaEvent_t* ev_wait,
                                bool record_used) {
+  if (c->ab_on) return enqueue_action_step_blocks(c, s, io, j, ev_wait, record_used);
   const Dims& d = c->d;
   const ExpertIdx& x = c->ea;
   c->cur_cls = WAM_PROF_ACTION_TEMB;
@@ -627,6 +830,7 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
     lora(c, Lq, i, kQkvLa, &c->m_la_qkv, &c->p_u_qkv);
     RET(norm_linear(c, Lq, epi_qkv(c, false, i), mod + d.da, mod, nullptr, WAM_PROF_ACTION_QKV, s));
     if (ev_wait) CK(cudaStreamWaitEvent(s, ev_wait[i], 0));
+    trace_mark(c, s, WAM_TRACE_ACTION_ATTN, i);
     c->cur_cls = WAM_PROF_ACTION_ATTN;
     RET(attention(c, false, i, s));
     if (record_used) CK(cudaEventRecord(c->ev_used[i], s));
@@ -646,6 +850,7 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
     Lin L2{&c->m_w_f2_a, &c->m_fa, matp(c, blk(x, i, kF2W)), c->f_a, d.da, d.Fa, i, &c->p_a_f2, d.lf};
     lora(c, L2, i, kF2La, &c->m_la_f2, &c->p_u_f2);
     RET(linear(c, false, L2, d.Ma, e2, nullptr, s));
+    trace_mark(c, s, WAM_TRACE_ACTION_END, i);
   }
   EpiArgs ee = epi_base(kEpiEuler, vecp(c, x.outb), c->a_state, nullptr, d.Pa);
   ee.aio = io;
@@ -659,7 +864,7 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
 
 // A whole chunk: video once, then `steps` Euler steps (or the joint one-step).
 wam_status enqueue_chunk(wam_ctx* c, int steps, int mode, bool joint, cudaStream_t sv, cudaStream_t sa,
-                         cudaEvent_t* ev_kv) {
+                         cudaEvent_t* ev_kv, int n_video = 0) {
   const Dims& d = c->d;
   const bool cewp = mode == WAM_SCHED_CEWP;
   cudaStream_t s_act = cewp ? sa : sv;
@@ -680,12 +885,19 @@ wam_status enqueue_chunk(wam_ctx* c, int steps, int mode, bool joint, cudaStream
   if (cewp) {
     // The experts need not be enqueued interleaved block by block: the two
     // streams run concurrently, and the per-block events order Attn^a_i after P^v_i.
-    RET(enqueue_video(c, sv, c->vio_chunk, joint, ev_kv, false));
-    for (int j = 0; j < steps; ++j) RET(enqueue_action_step(c, sa, c->aio_chunk, j, j == 0 ? ev_kv : nullptr, false));
+    RET(enqueue_video(c, sv, c->vio_chunk, joint, ev_kv, false, n_video));
+    for (int j = 0; j < steps; ++j) {
+      c->trace_step = j;
+      RET(enqueue_action_step(c, sa, c->aio_chunk, j, j == 0 ? ev_kv : nullptr, false));
+    }
   } else {
-    RET(enqueue_video(c, sv, c->vio_chunk, joint, nullptr, false));
-    for (int j = 0; j < steps; ++j) RET(enqueue_action_step(c, sv, c->aio_chunk, j, nullptr, false));
+    RET(enqueue_video(c, sv, c->vio_chunk, joint, nullptr, false, n_video));
+    for (int j = 0; j < steps; ++j) {
+      c->trace_step = j;
+      RET(enqueue_action_step(c, sv, c->aio_chunk, j, nullptr, false));
+    }
   }
+  c->trace_step = 0;
   c->launches++;
   {
     c->cur_cls = WAM_PROF_ACTION_IO;
@@ -713,11 +925,17 @@ wam_status set_chunk_io(wam_ctx* c, const VideoIo& v, const ActionIo& a, cudaStr
   return WAM_OK;
 }
 
-wam_status run_chunk(wam_ctx* c, int steps, int mode, int use_graph, bool joint, cudaStream_t sv, cudaStream_t sa) {
-  const long long key = ((long long)steps << 8) | (mode << 1) | (joint ? 1 : 0);
+// Graph key of a chunk: Euler steps, video passes, schedule, joint variant.
+long long chunk_key(int steps, int n_video, int mode, bool joint) {
+  return ((long long)steps << 24) | ((long long)n_video << 16) | (mode << 1) | (joint ? 1 : 0);
+}
+
+wam_status run_chunk(wam_ctx* c, int steps, int mode, int use_graph, bool joint, cudaStream_t sv, cudaStream_t sa,
+                     int n_video = 0) {
+  const long long key = chunk_key(steps, n_video, mode, joint);
   if (!use_graph) {
     c->launches = 0;
-    RET(enqueue_chunk(c, steps, mode, joint, sv, mode == WAM_SCHED_CEWP ? sa : sv, c->ev_kv.data()));
+    RET(enqueue_chunk(c, steps, mode, joint, sv, mode == WAM_SCHED_CEWP ? sa : sv, c->ev_kv.data(), n_video));
     c->launch_counts[key] = c->launches;
   } else {
     auto it = c->graphs.find(key);
@@ -725,7 +943,7 @@ wam_status run_chunk(wam_ctx* c, int steps, int mode, int use_graph, bool joint,
       cudaGraph_t graph = nullptr;
       c->launches = 0;
       CK(cudaStreamBeginCapture(c->cap_v, cudaStreamCaptureModeThreadLocal));
-      wam_status st = enqueue_chunk(c, steps, mode, joint, c->cap_v, c->cap_a, c->ev_kv_cap.data());
+      wam_status st = enqueue_chunk(c, steps, mode, joint, c->cap_v, c->cap_a, c->ev_kv_cap.data(), n_video);
       cudaError_t ce = cudaStreamEndCapture(c->cap_v, &graph);
       if (st != WAM_OK) {
         if (graph) cudaGraphDestroy(graph);
@@ -872,13 +1090,16 @@ void wam_destroy(wam_ctx* c) {
   for (auto e : {c->ev_fork, c->ev_join, c->ev_pre, c->ev_post})
     if (e) cudaEventDestroy(e);
   for (auto e : c->prof_pool) cudaEventDestroy(e);
+  for (auto e : c->trace_pool) cudaEventDestroy(e);
   if (c->cap_v) cudaStreamDestroy(c->cap_v);
   if (c->cap_a) cudaStreamDestroy(c->cap_a);
   void* bufs[] = {c->wmat, c->wvec, c->x_v, c->x_a, c->a_state, c->x_sigma, c->h_v, c->q_v, c->o_v, c->f_v,
                   c->x_vin, c->h_a, c->q_a, c->o_a, c->f_a, c->a_in, c->qkv_tmp_v, c->qkv_tmp_a, c->kv,
                   c->mod_v, c->mod_a, c->temb_v, c->temb_a, c->rope_cos, c->rope_sin, c->ws_gemm, c->tk_gemm, c->ws_gemm_v, c->tk_gemm_v, c->zero_r,
                   c->ws_attn, c->tk_attn, c->status, c->vio_chunk, c->vio_eager, c->aio_chunk, c->aio_eager,
-                  c->h_video, c->h_cond, c->h_noise, c->h_out, c->j_vout, c->j_aout};
+                  c->h_video, c->h_cond, c->h_noise, c->h_out, c->j_vout, c->j_aout, c->ab_ws, c->ab_ws_attn,
+                  c->ab_cnt, c->ab_cnt_attn, c->ab_bar, c->td_at, c->td_as, c->td_a0, c->td_fs, c->td_fe,
+                  c->aio_tacd};
   for (void* p : bufs)
     if (p) cudaFree(p);
   delete c;
@@ -992,10 +1213,18 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
       return (k <= 2 && tiles % k == 0) ? tiles / k : vctas;
     };
     const int bn_res = ((d.Mv + 127) / 128) * (d.dv / 256) >= 2 * vctas ? 256 : 128;
+    // WAM_VIDEO_OPROJ_BN / WAM_VIDEO_FFN2_BN (128 or 256) override the tile
+    // width of the two gate-residual GEMMs
+    auto bn_env = [&](const char* name, int dflt) {
+      const char* v = getenv(name);
+      const int n = v ? atoi(v) : 0;
+      return (n == 128 || n == 256) && d.dv % n == 0 ? n : dflt;
+    };
+    const int bn_o = bn_env("WAM_VIDEO_OPROJ_BN", bn_res), bn_f2 = bn_env("WAM_VIDEO_FFN2_BN", bn_res);
     c->p_v_qkv = {256, 1, grid(3 * d.A, 256)};
-    c->p_v_o = {bn_res, 1, grid(d.dv, bn_res)};
+    c->p_v_o = {bn_o, 1, grid(d.dv, bn_o)};
     c->p_v_f1 = {256, 1, grid(d.Fv, 256)};
-    c->p_v_f2 = {bn_res, 1, grid(d.dv, bn_res)};
+    c->p_v_f2 = {bn_f2, 1, grid(d.dv, bn_f2)};
     c->p_v_in = {128, 1, grid(d.dv, 128)};
     c->p_v_out = {64, 1, grid(d.Pv > 0 ? d.Pv : 64, 64)};
     const int bn_a = d.Ma <= 32 ? 32 : (d.Ma <= 64 ? 64 : (d.Ma <= 128 ? 128 : 256));
@@ -1059,8 +1288,10 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   }
   RET(dalloc(c, &c->ws_gemm, ws * 4));
   RET(dalloc(c, &c->tk_gemm, (size_t)tiles * 2 * 4));
+  c->tk_gemm_bytes = (size_t)tiles * 2 * 4;
   RET(dalloc(c, &c->ws_gemm_v, ws_v * 4));
   RET(dalloc(c, &c->tk_gemm_v, (size_t)tiles_v * 2 * 4));
+  c->tk_gemm_v_bytes = (size_t)tiles_v * 2 * 4;
   RET(dalloc(c, &c->ws_attn, attention_ws_floats(d.B, d.H, d.Dh, d.La, c->attn_splits) * 4));
   RET(dalloc(c, &c->tk_attn, (size_t)d.B * d.H * 4));
 
@@ -1110,6 +1341,61 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     ok = ok && make_tmap_sw128(&c->m_cache_out, c->kv, 2, d.Dh, d.Ltot, 2 * d.N * d.B * d.H,
                                (size_t)d.Ltot * d.Dh * 2, 64, 32);
     if (!ok) return fail(c, WAM_ERR_CUDA, "tensor map creation failed");
+
+    // Persistent action-block path: bf16 without LoRA, at most 32 action
+    // tokens per chunk, action width a multiple of 64 up to 768 (the block's
+    // B operand and one attention unit share a 48 KB region).  WAM_ACTION_BLOCKS=0
+    // keeps the per-operation kernels.
+    const char* abv = getenv("WAM_ACTION_BLOCKS");
+    const bool ab_want = !(abv && abv[0] == '0');
+    if (ab_want && d.r == 0 && d.Ma <= 32 && d.da % 64 == 0 && d.da <= 768 && d.Fa % 64 == 0 && d.A % 64 == 0 &&
+        d.Fa <= 4096 && d.A <= 4096) {
+      int nsm = 148;
+      CK(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, c->device));
+      c->ab_ctas = nsm;
+      int vctas_used = std::max(1, nsm * 73 / 100);
+      if (const char* v = getenv("WAM_VIDEO_GEMM_CTAS")) {
+        const int n = atoi(v);
+        if (n > 0) vctas_used = std::min(n, nsm);
+      }
+      c->ab_ctas_overlap = std::max(8, nsm - vctas_used);
+      if (const char* v = getenv("WAM_ACTION_BLOCK_CTAS")) {
+        const int n = atoi(v);
+        if (n > 0) c->ab_ctas_overlap = std::min(n, nsm);
+      }
+      c->ab_ks_in = action_block_ks(d.da, d.Kin, nsm);
+      c->ab_ks_qkv = action_block_ks(3 * d.A, d.da, nsm);
+      c->ab_ks_o = action_block_ks(d.da, d.A, nsm);
+      c->ab_ks_f1 = action_block_ks(d.Fa, d.da, nsm);
+      c->ab_ks_f2 = action_block_ks(d.da, d.Fa, nsm);
+      c->ab_ks_out = action_block_ks(d.Pa, d.da, nsm);
+      c->ab_splits = action_block_attn_splits(d.Lv + d.La);
+      bool fits = (3 * d.A + 127) / 128 <= 64 && (d.Fa + 127) / 128 <= 64;
+      for (int g : {c->ab_ctas, c->ab_ctas_overlap}) {
+        fits = fits && action_block_fits(d.da, d.Kin, c->ab_ks_in, g) && action_block_fits(3 * d.A, d.da, c->ab_ks_qkv, g) &&
+               action_block_fits(d.da, d.A, c->ab_ks_o, g) && action_block_fits(d.Fa, d.da, c->ab_ks_f1, g) &&
+               action_block_fits(d.da, d.Fa, c->ab_ks_f2, g) && action_block_fits(d.Pa, d.da, c->ab_ks_out, g);
+      }
+      if (fits) {
+        auto units = [&](int n_out, int ks) { return ((n_out + 127) / 128) * ks; };
+        int mu = std::max({units(d.da, c->ab_ks_in), units(3 * d.A, c->ab_ks_qkv), units(d.da, c->ab_ks_o),
+                           units(d.Fa, c->ab_ks_f1), units(d.da, c->ab_ks_f2), units(d.Pa, c->ab_ks_out)});
+        CK(prepare_action_block());
+        RET(dalloc(c, &c->ab_ws, action_block_ws_floats(mu) * 4));
+        RET(dalloc(c, &c->ab_ws_attn, action_block_attn_ws_floats(d.B, d.H, c->ab_splits) * 4));
+        RET(dalloc(c, &c->ab_cnt, 2 * 64 * 4));
+        RET(dalloc(c, &c->ab_cnt_attn, (size_t)2 * d.B * d.H * 4));
+        RET(dalloc(c, &c->ab_bar, 2 * 4));
+        bool mok = make_tmap_3d(&c->m_qa128, c->q_a, d.Dh, d.La, d.B * d.H, (size_t)d.La * d.Dh * 2, 128) &&
+                   make_tmap_3d(&c->m_cache128, c->kv, d.Dh, d.Ltot, 2 * d.N * d.B * d.H, (size_t)d.Ltot * d.Dh * 2, 128);
+        if (!mok) return fail(c, WAM_ERR_CUDA, "tensor map creation failed");
+        const CUtensorMap* mm[kActionBlockMaps] = {&c->m_w_qkv_a, &c->m_w_o_a, &c->m_w_f1_a, &c->m_w_f2_a,
+                                                   &c->m_w_in,    &c->m_w_out, &c->m_oa,    &c->m_fa,
+                                                   &c->m_ain,     &c->m_qa128, &c->m_cache128};
+        for (int k = 0; k < kActionBlockMaps; ++k) c->ab_maps.m[k] = *mm[k];
+        c->ab_on = true;
+      }
+    }
   }
 
   c->ev_kv.resize(d.N);
@@ -1241,6 +1527,114 @@ wam_status wam_joint_one_step(wam_ctx* c, const float* vclean, const float* veps
   return run_chunk(c, 1, mode, use_graph, true, sv, sa);
 }
 
+namespace {
+// S eager Euler steps of the action expert of `c` along sched[0..S] from
+// dev_in into dev_out, on `s`, with the block K/V already in c's cache.
+wam_status run_action_steps(wam_ctx* c, cudaStream_t s, const float* dev_in, float* dev_out, const float* sched,
+                            int S) {
+  const Dims& d = c->d;
+  ActionIo a{};
+  a.a_in = dev_in;
+  a.a_out = dev_out;
+  for (int j = 0; j <= S; ++j) a.sched[j] = sched[j];
+  a.steps = S;
+  CK(launch_set_action_io(c->aio_tacd, a, s));
+  CK(launch_init_action(c->aio_tacd, c->a_state, d.bf16 ? c->a_in : nullptr, d.bf16, d.Ma, d.Pa, d.Kin, s));
+  for (int j = 0; j < S; ++j) RET(enqueue_action_step(c, s, c->aio_tacd, j, nullptr, false));
+  CK(launch_copy_out(c->aio_tacd, c->a_state, d.Ma * d.Pa, s));
+  return WAM_OK;
+}
+}  // namespace
+
+wam_status wam_tacd_targets(wam_ctx* c, wam_ctx* ema, const float* video, const float* cond, const float* a_clean,
+                            const float* eps, float t, int K, float lambda, float* u_ta, float* v_student,
+                            float* u_cd, float* losses, float* a_t_out, float* a0_teacher_out, void* stream) {
+  if (!c || !ema) return WAM_ERR_INVALID_ARG;
+  const Dims& d = c->d;
+  if (!video || !a_clean || !eps || !losses || (d.Lc > 0 && !cond) || d.Pv > 0 || !(t > 0.f && t <= 1.f) || K < 1 ||
+      K > kMaxSteps)
+    return fail(c, WAM_ERR_INVALID_ARG, "wam_tacd_targets: bad arguments");
+  if (d.r <= 0 || memcmp(&c->cfg, &ema->cfg, sizeof c->cfg) != 0 || c->device != ema->device)
+    return fail(c, WAM_ERR_INVALID_ARG, "wam_tacd_targets: student and EMA need the same LoRA model on one device");
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t n = (size_t)d.Ma * d.Pa;
+  for (float** p : {&c->td_at, &c->td_as, &c->td_a0, &c->td_fs, &c->td_fe})
+    if (!*p) RET(dalloc(c, p, n * 4));
+  if (!c->aio_tacd) RET(dalloc(c, &c->aio_tacd, sizeof(ActionIo)));
+  if (ema != c && !ema->aio_tacd) RET(dalloc(ema, &ema->aio_tacd, sizeof(ActionIo)));
+  // teacher grid t_k = t k / K (k = K .. 0); s = t (K - 1) / K is its first point
+  float grid[kMaxSteps + 1];
+  for (int k = 0; k <= K; ++k) grid[k] = (float)((double)t * (double)(K - k) / (double)K);
+  const float s_pt = grid[1];
+  // a_t, and the frozen video expert once (t_v = 0) into the student's cache
+  CK(launch_tacd_noise(a_clean, eps, t, c->td_at, (int)n, s));
+  VideoIo v{};
+  v.video = video;
+  v.cond = cond;
+  CK(launch_set_video_io(c->vio_eager, v, s));
+  RET(enqueue_video(c, s, c->vio_eager, false, nullptr, false));
+  // teacher: the base weights (LoRA scale 0 adds exact zeros), K Euler steps
+  // from (a_t, t) to 0; the first state is a~_s
+  const float scale = c->cfg.lora_scale;
+  c->cfg.lora_scale = 0.f;
+  wam_status st = run_action_steps(c, s, c->td_at, c->td_as, grid, 1);
+  if (st == WAM_OK) st = K > 1 ? run_action_steps(c, s, c->td_as, c->td_a0, grid + 1, K - 1) : WAM_OK;
+  c->cfg.lora_scale = scale;
+  RET(st);
+  const float* a0T = K > 1 ? c->td_a0 : c->td_as;
+  // student endpoint f(a_t, t) = a_t - t v (one step t -> 0)
+  const float sched_st[2] = {t, 0.f};
+  RET(run_action_steps(c, s, c->td_at, c->td_fs, sched_st, 1));
+  // EMA endpoint f^-(a~_s, s) over the same K/V (s = 0: the endpoint map is the identity)
+  const float* fe = c->td_as;
+  if (s_pt > 0.f) {
+    if (ema != c) {
+      const size_t kv_bytes = (size_t)2 * d.N * d.B * d.H * d.Ltot * d.Dh * c->esz;
+      CK(cudaMemcpyAsync(ema->kv, c->kv, kv_bytes, cudaMemcpyDeviceToDevice, s));
+    }
+    const float sched_ema[2] = {s_pt, 0.f};
+    RET(run_action_steps(ema, s, c->td_as, c->td_fe, sched_ema, 1));
+    fe = c->td_fe;
+  }
+  if (a_t_out) CK(cudaMemcpyAsync(a_t_out, c->td_at, n * 4, cudaMemcpyDeviceToDevice, s));
+  if (a0_teacher_out) CK(cudaMemcpyAsync(a0_teacher_out, a0T, n * 4, cudaMemcpyDeviceToDevice, s));
+  CK(launch_tacd_targets(c->td_at, a0T, c->td_fs, fe, t, lambda, d.B, d.La * d.Pa, u_ta, v_student, u_cd, losses, s));
+  return WAM_OK;
+}
+
+wam_status wam_infer_chunk_multistep(wam_ctx* c, const float* video_eps, const float* noise, float* video_out,
+                                     float* actions_out, int n_video, const float* sched_v, int S,
+                                     const float* t_sched, int mode, int use_graph, void* stream_video,
+                                     void* stream_action) {
+  if (!c) return WAM_ERR_INVALID_ARG;
+  if (c->d.Pv <= 0 || !c->cfg.video_has_output)
+    return fail(c, WAM_ERR_UNSUPPORTED, "wam_infer_chunk_multistep needs a patch-input model with a video output");
+  if (!video_eps || !noise || !video_out || !actions_out || n_video < 1 || n_video > kMaxSteps || S < 1 ||
+      S > kMaxSteps || (mode != WAM_SCHED_SEQUENTIAL && mode != WAM_SCHED_CEWP))
+    return fail(c, WAM_ERR_INVALID_ARG, "wam_infer_chunk_multistep: bad arguments");
+  cudaStream_t sv = (cudaStream_t)stream_video, sa = (cudaStream_t)stream_action;
+  if (mode == WAM_SCHED_CEWP && sa == sv) return fail(c, WAM_ERR_INVALID_ARG, "CEWP needs two distinct streams");
+  VideoIo v{};
+  for (int j = 0; j <= n_video; ++j) v.vsched[j] = sched_v ? sched_v[j] : (float)(n_video - j) / (float)n_video;
+  if (!valid_schedule(v.vsched, n_video) || v.vsched[0] != 1.f)
+    return fail(c, WAM_ERR_INVALID_ARG, "wam_infer_chunk_multistep: video schedule must fall from 1 within [0,1]");
+  v.vsteps = n_video;
+  v.video = video_eps;  // the latents at level 1 are the noise itself: (1 - 1) x + 1 eps
+  v.eps = video_eps;
+  v.t = 1.f;
+  v.video_out = video_out;
+  ActionIo a{};
+  for (int j = 0; j <= S; ++j) a.sched[j] = t_sched ? t_sched[j] : (float)(S - j) / (float)S;
+  if (!valid_schedule(a.sched, S)) return fail(c, WAM_ERR_INVALID_ARG, "wam_infer_chunk_multistep: bad schedule");
+  a.steps = S;
+  a.a_in = noise;
+  a.a_out = actions_out;
+  CK(cudaEventRecord(c->ev_pre, sa));
+  CK(cudaStreamWaitEvent(sv, c->ev_pre, 0));
+  RET(set_chunk_io(c, v, a, sv));
+  return run_chunk(c, S, mode, use_graph, false, sv, sa, n_video);
+}
+
 wam_status wam_profile_chunk(wam_ctx* c, const float* video, const float* cond, const float* noise, float* out, int S,
                              void* stream, float* host_ms, int* host_counts) {
   if (!c || !host_ms || !host_counts) return WAM_ERR_INVALID_ARG;
@@ -1291,6 +1685,67 @@ wam_status wam_profile_chunk(wam_ctx* c, const float* video, const float* cond, 
     CK(cudaEventElapsedTime(&ms, r.a, r.b));
     host_ms[r.cls] += ms;
     host_counts[r.cls] += 1;
+  }
+  return WAM_OK;
+}
+
+wam_status wam_trace_chunk(wam_ctx* c, const float* video, const float* cond, const float* noise, float* out, int S,
+                           int mode, void* stream_video, void* stream_action, float* host_ms, int capacity,
+                           int* count) {
+  if (!c || !host_ms || !count || capacity < 0) return WAM_ERR_INVALID_ARG;
+  if (!video || !noise || !out || (c->d.Lc > 0 && !cond) || c->d.Pv > 0 || S < 1 || S > kMaxSteps ||
+      (mode != WAM_SCHED_SEQUENTIAL && mode != WAM_SCHED_CEWP))
+    return fail(c, WAM_ERR_INVALID_ARG, "wam_trace_chunk: bad arguments");
+  cudaStream_t sv = (cudaStream_t)stream_video, sa = (cudaStream_t)stream_action;
+  if (mode == WAM_SCHED_CEWP && sa == sv) return fail(c, WAM_ERR_INVALID_ARG, "CEWP needs two distinct streams");
+  ActionIo a{};
+  for (int j = 0; j <= S; ++j) a.sched[j] = (float)(S - j) / (float)S;
+  a.steps = S;
+  a.a_in = noise;
+  a.a_out = out;
+  VideoIo v{};
+  v.video = video;
+  v.cond = cond;
+  CK(cudaEventRecord(c->ev_pre, sa));
+  CK(cudaStreamWaitEvent(sv, c->ev_pre, 0));
+  RET(set_chunk_io(c, v, a, sv));
+  CK(cudaStreamSynchronize(sv));
+  // capture the chunk with timing events at the block boundaries, replay once
+  c->trace.clear();
+  c->trace_on = true;
+  cudaGraph_t graph = nullptr;
+  CK(cudaStreamBeginCapture(c->cap_v, cudaStreamCaptureModeThreadLocal));
+  trace_mark(c, c->cap_v, WAM_TRACE_START, 0);
+  wam_status st = enqueue_chunk(c, S, mode, false, c->cap_v, mode == WAM_SCHED_CEWP ? c->cap_a : c->cap_v,
+                                c->ev_kv_cap.data());
+  if (st == WAM_OK) trace_mark(c, c->cap_v, WAM_TRACE_END, 0);
+  c->trace_on = false;
+  cudaError_t ce = cudaStreamEndCapture(c->cap_v, &graph);
+  if (st != WAM_OK) {
+    if (graph) cudaGraphDestroy(graph);
+    return st;
+  }
+  CK(ce);
+  cudaGraphExec_t exec = nullptr;
+  ce = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  CK(ce);
+  // one warm replay, then the timed one
+  for (int r = 0; r < 2 && ce == cudaSuccess; ++r) {
+    ce = cudaGraphLaunch(exec, sv);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(sv);
+  }
+  cudaGraphExecDestroy(exec);
+  CK(ce);
+  // records: (kind, block, step, ms since the start mark)
+  *count = (int)c->trace.size();
+  for (size_t k = 0; k < c->trace.size() && (int)k < capacity; ++k) {
+    float ms = 0.f;
+    CK(cudaEventElapsedTime(&ms, c->trace[0].e, c->trace[k].e));
+    host_ms[4 * k + 0] = (float)c->trace[k].kind;
+    host_ms[4 * k + 1] = (float)c->trace[k].block;
+    host_ms[4 * k + 2] = (float)c->trace[k].step;
+    host_ms[4 * k + 3] = ms;
   }
   return WAM_OK;
 }
@@ -1393,16 +1848,31 @@ wam_status wam_check_device_status(wam_ctx* c) {
   unsigned st = 0;
   CK(cudaMemcpy(&st, c->status, 4, cudaMemcpyDeviceToHost));
   if (st) {
+    // A kernel that gave up may have left its tickets, counters or grid
+    // barrier mid-way: clear them so that the next call starts clean.
     CK(cudaMemset(c->status, 0, 4));
+    if (c->tk_gemm) CK(cudaMemset(c->tk_gemm, 0, c->tk_gemm_bytes));
+    if (c->tk_gemm_v) CK(cudaMemset(c->tk_gemm_v, 0, c->tk_gemm_v_bytes));
+    if (c->ab_cnt) CK(cudaMemset(c->ab_cnt, 0, 2 * 64 * 4));
+    if (c->ab_cnt_attn) CK(cudaMemset(c->ab_cnt_attn, 0, (size_t)2 * c->d.B * c->d.H * 4));
+    if (c->ab_bar) CK(cudaMemset(c->ab_bar, 0, 2 * 4));
+    if (c->tk_attn) CK(cudaMemset(c->tk_attn, 0, (size_t)c->d.B * c->d.H * 4));
+    CK(cudaDeviceSynchronize());
     return fail(c, WAM_ERR_TIMEOUT, "device bounded wait gave up (status bits 0x%x)", st);
   }
   return WAM_OK;
 }
 
+wam_status wam_test_peer_wait(int extra, unsigned long long limit_ns) {
+  if (extra < 0 || (extra > 0 && limit_ns == 0)) return WAM_ERR_INVALID_ARG;
+  if (extra == 0) limit_ns = 2000000000ull;  // the kernels' normal limit (2 s)
+  return set_peer_wait_test(extra, limit_ns) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
+}
+
 int wam_chunk_kernel_count(wam_ctx* c, int S) {
   if (!c) return -1;
   for (auto& kv : c->launch_counts)
-    if ((kv.first >> 8) == S) return kv.second;
+    if ((kv.first >> 24) == S) return kv.second;
   return -1;
 }
 

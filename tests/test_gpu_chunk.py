@@ -252,3 +252,33 @@ def test_device_memory_limit_reports_oom(monkeypatch):
     a0 = run_chunk(wam, inp, S=1)
     assert np.isfinite(a0).all()
     wam.close()
+
+
+def test_bounded_wait_timeout_is_reported_and_the_next_call_is_clean():
+    """Failure detection without a GPU fault: the test hook makes the last
+    piece of every split GEMM tile wait for one partial tile more than exists
+    (a count nothing raises) with a 20 ms limit.  The kernels give up, wind
+    down and return; wam_check_device_status reports WAM_ERR_TIMEOUT and
+    resets the tickets; with the hook off the next chunk equals the reference
+    bitwise and the status is clean."""
+    c = _mid()
+    wam = W.Wam(c, seed=9)
+    inp = inputs(c, 9)
+    ref = run_chunk(wam, inp, S=1)
+    assert W.lib().wam_test_peer_wait(1, 20_000_000) == 0
+    try:
+        dev = torch.device("cuda", 0)
+        video, cond, noise = (torch.from_numpy(inp[k]).to(dev) for k in ("video", "cond", "noise"))
+        out = torch.empty_like(noise)
+        sv, sa = torch.cuda.Stream(), torch.cuda.Stream()
+        wam.infer_chunk(video, cond, noise, out, S=1, mode=W.CEWP, use_graph=False, stream_video=sv,
+                        stream_action=sa)
+        sv.synchronize()
+        with pytest.raises(W.WamError) as e:
+            wam.check_device_status()
+        assert e.value.status == 5
+    finally:
+        assert W.lib().wam_test_peer_wait(0, 0) == 0
+    again = run_chunk(wam, inp, S=1)   # run_chunk checks the status itself
+    assert np.array_equal(again, ref)
+    wam.close()

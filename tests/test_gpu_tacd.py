@@ -86,3 +86,63 @@ def test_tacd_targets_through_the_chunk_entry_point(dtype):
         assert e <= tol, f"{k}: rel L2 {e:.3e} (tol {tol})"
     l_ta = T.chunk_mean_sq(got["v_student"] - got["u_ta"])
     assert abs(l_ta - ref["l_ta"]) <= 5 * tol * ref["l_ta"], (l_ta, ref["l_ta"])
+
+
+def _ema_params(c, seed, P_student):
+    """The EMA target's parameters: the student's, with LoRA factors drawn
+    from another seed (an EMA that has drifted from the student)."""
+    other = PR.generate_params(ocfg(c), seed + 1)
+    return {k: (other[k] if k.endswith((".la", ".lb")) else v) for k, v in P_student.items()}
+
+
+@pytest.mark.parametrize("dtype,K", [("fp32", 10), ("fp32", 1), ("bf16", 10)])
+def test_tacd_targets_entry_point(dtype, K):
+    """wam_tacd_targets: video once, the teacher (base weights) K steps over
+    [t, 0], the student and a distinct EMA LoRA over the shared K/V, device-side
+    noising, targets and the deterministic loss reduction -- against the
+    oracle's tacd_targets (rel. L2 1e-4 fp32 / 1e-2 bf16 on u_TA, v_student,
+    u_CD; the losses within 5x that, relative)."""
+    if dtype == "fp32":
+        c = W.preset(1).replace(lora_rank=64, lora_scale=0.5)
+    else:
+        c = W.WamConfig(**MID_BF16).replace(lora_rank=128, lora_scale=1.0, n_blocks=2)
+    seed, t = 31, 0.625
+    inp = synthetic.make_inputs(seed, batch=c.batch, l_cond=c.l_cond, l_video=c.l_video, video_width=c.d_video,
+                                l_action=c.l_action, action_dim=c.action_dim, action_clean=True)
+    for k in ("action_clean", "noise"):   # a_t exact in fp32 on this grid (see above)
+        inp[k] = (np.round(inp[k] * 4096) / 4096).astype(np.float32)
+    oc = ocfg(c)
+    P_student = PR.generate_params(oc, seed)
+    P_ema = _ema_params(c, seed, P_student)
+    ref = T.tacd_targets(oc, T.without_lora(P_student), P_student, P_ema, inp, t=t, K=K)
+
+    student = W.Wam(c, seed=seed)
+    ema = W.Wam(c, seed=seed)
+    names = [n for n, _, _ in PR.param_specs(oc)]
+    ema.import_params(np.concatenate([np.asarray(P_ema[n], np.float32).ravel() for n in names]))
+    dev = torch.device("cuda", 0)
+    d = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to(dev) for k in ("video", "action_clean", "noise")}
+    cond = torch.from_numpy(inp["cond"]).to(dev) if c.l_cond else None
+    outs = {k: torch.full_like(d["noise"], float("nan")) for k in ("u_ta", "v_student", "u_cd", "a_t", "a0_T")}
+    losses = torch.full((3,), float("nan"), device=dev)
+    s = torch.cuda.Stream()
+    student.tacd_targets(ema, d["video"], cond, d["action_clean"], d["noise"], t, K, 0.2, outs["u_ta"],
+                         outs["v_student"], outs["u_cd"], losses, a_t=outs["a_t"], a0_teacher=outs["a0_T"], stream=s)
+    s.synchronize()
+    student.check_device_status()
+    got = {k: v.cpu().numpy().astype(np.float64) for k, v in outs.items()}
+    l = losses.cpu().numpy().astype(np.float64)
+    student.close()
+    ema.close()
+    assert np.array_equal(got["a_t"], ref["a_t"])
+    tol = TOL[c.dtype]
+    for k, want in (("u_ta", ref["u_ta"]), ("v_student", ref["v_student"]), ("u_cd", ref["u_cd"])):
+        assert np.isfinite(got[k]).all(), k
+        e = rel_l2(got[k], want)
+        assert e <= tol, f"{k}: rel L2 {e:.3e} (tol {tol})"
+    assert rel_l2(got["a0_T"], ref["a0_T"]) <= tol
+    for i, key in enumerate(("l_ta", "l_cd")):
+        assert abs(l[i] - ref[key]) <= 5 * tol * ref[key], (key, l[i], ref[key])
+    assert abs(l[2] - (l[1] + 0.2 * l[0])) <= 1e-6 * l[2]
+    if K == 1:   # s = 0: the EMA endpoint is the teacher's one-step state, so u_CD = u_TA
+        np.testing.assert_array_equal(got["u_cd"], got["u_ta"])
