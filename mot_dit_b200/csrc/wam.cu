@@ -1207,10 +1207,13 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     // in the short tail (QKV at 1088 tokens: 162 tiles on 81 CTAs instead of
     // 1.5 tiles on each of 108; chunk 4.33 -> 4.15 ms).  With more tiles per
     // CTA the split overhead is small and all vctas CTAs are kept.
+    // WAM_VIDEO_SPLIT_FREE=0 turns the rule off (always vctas CTAs, stream-K).
+    const char* sfv = getenv("WAM_VIDEO_SPLIT_FREE");
+    const bool split_free = !(sfv && sfv[0] == '0');
     auto grid = [&](int n_out, int bn) {
       const int tiles = ((d.Mv + 127) / 128) * ((n_out + bn - 1) / bn);
       const int k = (tiles + vctas - 1) / vctas;  // tiles per CTA
-      return (k <= 2 && tiles % k == 0) ? tiles / k : vctas;
+      return (split_free && k <= 2 && tiles % k == 0) ? tiles / k : vctas;
     };
     const int bn_res = ((d.Mv + 127) / 128) * (d.dv / 256) >= 2 * vctas ? 256 : 128;
     // WAM_VIDEO_OPROJ_BN / WAM_VIDEO_FFN2_BN (128 or 256) override the tile
@@ -1342,12 +1345,14 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
                                (size_t)d.Ltot * d.Dh * 2, 64, 32);
     if (!ok) return fail(c, WAM_ERR_CUDA, "tensor map creation failed");
 
-    // Persistent action-block path: bf16 without LoRA, at most 32 action
-    // tokens per chunk, action width a multiple of 64 up to 768 (the block's
-    // B operand and one attention unit share a 48 KB region).  WAM_ACTION_BLOCKS=0
-    // keeps the per-operation kernels.
+    // Persistent action-block path (opt-in, WAM_ACTION_BLOCKS=1): bf16
+    // without LoRA, at most 32 action tokens per chunk, action width a
+    // multiple of 64 up to 768 (the block's B operand and one attention unit
+    // share a 48 KB region).  Off by default: on the config-2 / config-3
+    // chunks its launches (about 80 us per block, latency of the phase
+    // chain) are slower than the per-operation kernels.
     const char* abv = getenv("WAM_ACTION_BLOCKS");
-    const bool ab_want = !(abv && abv[0] == '0');
+    const bool ab_want = abv && abv[0] == '1';
     if (ab_want && d.r == 0 && d.Ma <= 32 && d.da % 64 == 0 && d.da <= 768 && d.Fa % 64 == 0 && d.A % 64 == 0 &&
         d.Fa <= 4096 && d.A <= 4096) {
       int nsm = 148;

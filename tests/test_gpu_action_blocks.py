@@ -27,7 +27,7 @@ SMALL = dict(n_blocks=3, d_video=256, d_action=128, n_heads=4, head_dim=64, ffn_
 
 
 def _wam(monkeypatch, seed, ctas=None, blocks=True, **kw):
-    monkeypatch.setenv("WAM_ACTION_BLOCKS", "1" if blocks else "0")
+    monkeypatch.setenv("WAM_ACTION_BLOCKS", "1" if blocks else "0")   # (the path is opt-in)
     if ctas is not None:
         monkeypatch.setenv("WAM_ACTION_BLOCK_CTAS", str(ctas))
     else:

@@ -14,8 +14,9 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("batch", [1, 2])
-def test_trace_records_the_wavefront(batch):
+@pytest.mark.parametrize("batch,blocks", [(1, "0"), (1, "1"), (2, "0")])
+def test_trace_records_the_wavefront(monkeypatch, batch, blocks):
+    monkeypatch.setenv("WAM_ACTION_BLOCKS", blocks)   # per-operation kernels / persistent action blocks
     c = W.WamConfig(**MID_BF16).replace(batch=batch)
     wam = W.Wam(c, seed=3)
     inp = inputs(c, 3)
