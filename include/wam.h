@@ -226,6 +226,18 @@ wam_status wam_read_kv(wam_ctx* ctx, int block, int which, float* host_buf, size
  * bounded waits (WAM_ERR_TIMEOUT, then clears the flag) or CUDA errors. */
 wam_status wam_check_device_status(wam_ctx* ctx);
 
+/* Pixel front-end of the patch-input (joint) model: the Flash-WAM setting
+ * cuts 128 x 128 RGB frames into 16 x 16 patches of 3 x 8 x 8 = 192 values
+ * (Flash-WAM close reading, 数据与训练流程).  inverse = 0: dev_frames
+ * [B, F, C, H, W] (channel-first) -> dev_patches [B, F (H/p)(W/p), C p p];
+ * token f (H/p)(W/p) + py (W/p) + px, feature c p^2 + iy p + ix holds pixel
+ * (f, c, py p + iy, px p + ix).  inverse = 1: the other way (dev_patches read,
+ * dev_frames written), e.g. for the video endpoint.  H and W multiples of p.
+ * Enqueued on `stream`.  (The pages name a VAE encoder in the end-to-end
+ * latency but give no architecture or weights: none is built.) */
+wam_status wam_patchify(const float* dev_frames, float* dev_patches, int B, int F, int C, int H, int W, int p,
+                        int inverse, void* stream);
+
 /* Failure-path test hook (tests only; every context of the process on the
  * current device).  With extra > 0, the last piece of a split GEMM tile that
  * is its CTA's final segment waits for `extra` more partial tiles than exist,

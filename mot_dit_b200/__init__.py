@@ -13,6 +13,7 @@ from ._binding import (  # noqa: F401
     FP32,
     PROF_CLASSES,
     SEQUENTIAL,
+    TRACE_KINDS,
     Wam,
     WamConfig,
     WamError,
@@ -22,5 +23,6 @@ from ._binding import (  # noqa: F401
     op_attention_noalloc,
     op_linear,
     op_norm_mod,
+    patchify,
     preset,
 )

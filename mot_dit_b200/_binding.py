@@ -80,6 +80,7 @@ def lib():
         "wam_profile_chunk": (C.c_int, [_P, _P, _P, _P, _P, C.c_int, _P, _P, _P]),
         "wam_trace_chunk": (C.c_int, [_P, _P, _P, _P, _P, C.c_int, C.c_int, _P, _P, _P, C.c_int, _P]),
         "wam_test_peer_wait": (C.c_int, [C.c_int, C.c_uint64]),
+        "wam_patchify": (C.c_int, [_P, _P] + [C.c_int] * 7 + [_P]),
         "wam_status_str": (C.c_char_p, [C.c_int]),
         "wam_last_error": (C.c_char_p, [_P]),
         "wam_op_linear": (C.c_int, [C.c_int, _P, _P, _P, _P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _P]),
@@ -329,6 +330,13 @@ def op_attention(dtype, q, k, v, out, B, H, Dh, Lq, Lk, Lcache, splits=1, stream
                                 _stream(stream))
     if st:
         raise WamError(st, "wam_op_attention")
+
+
+def patchify(frames, patches, B, F, C, H, W, p, inverse=False, stream=None):
+    """Frames [B, F, C, H, W] <-> patch tokens [B, F (H/p)(W/p), C p p] (wam_patchify)."""
+    st = lib().wam_patchify(_ptr(frames), _ptr(patches), B, F, C, H, W, p, int(inverse), _stream(stream))
+    if st:
+        raise WamError(st, "wam_patchify")
 
 
 def op_attention_noalloc(q, k, v, out, B, H, Lq, Lk, Lcache, splits, stream=None):

@@ -297,6 +297,11 @@ cudaError_t prepare_action_block();
 // `ctas` <= the SM count (one CTA per SM: the grid barriers need the whole grid resident).
 cudaError_t launch_action_block(const ActionBlockMaps& m, const ActionBlockArgs& a, int ctas, cudaStream_t s);
 
+// Pixel front-end: frames [B, F, C, H, W] -> patch tokens [B, F (H/p)(W/p), C p p]
+// (inverse: the other way).
+cudaError_t launch_patchify(const float* src, float* dst, int B, int F, int C, int H, int W, int p, bool inverse,
+                            cudaStream_t s);
+
 // TACD target forward: a_t = (1 - t) a_clean + t eps; and the targets
 // u_TA, v_student, u_CD (any may be null) plus losses[3] = L_TA, L_CD,
 // L_CD + lambda L_TA from the teacher end state, the student and EMA endpoints.

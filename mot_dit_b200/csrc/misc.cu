@@ -222,6 +222,33 @@ __global__ void copy_out_kernel(const ActionIo* __restrict__ io, const float* __
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) out[i] = a[i];
 }
 
+// ------------------------------------------------------ pixel front-end -----
+// Patchify / unpatchify of channel-first frames [B, F, C, H, W] <-> patch
+// tokens [B, F (H/p)(W/p), C p p] (token = frame-major raster order of the
+// patches, feature = (channel, row, column) within the patch).  One thread
+// per patch-token element; the patch side is written (patchify) or read
+// (unpatchify) contiguously.
+__global__ void patchify_kernel(const float* __restrict__ src, float* __restrict__ dst, int F, int C, int H, int W,
+                                int p, size_t n, int inverse) {
+  pdl_trigger();
+  pdl_wait();
+  const int Hp = H / p, Wp = W / p, cpp = C * p * p;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t tok = i / cpp;
+    const int feat = (int)(i - tok * cpp);
+    const int per_sample = F * Hp * Wp;
+    const size_t b = tok / per_sample;
+    const int t = (int)(tok - b * per_sample);
+    const int f = t / (Hp * Wp), py = (t / Wp) % Hp, px = t % Wp;
+    const int c = feat / (p * p), iy = (feat / p) % p, ix = feat % p;
+    const size_t pix = ((((b * F + f) * C + c) * (size_t)H + (py * p + iy)) * W) + px * p + ix;
+    if (inverse)
+      dst[pix] = src[i];
+    else
+      dst[i] = src[pix];
+  }
+}
+
 // -------------------------------------------------- seeded parameters ------
 __device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
   uint64_t z = x + 0x9E3779B97F4A7C15ull;
@@ -332,6 +359,13 @@ cudaError_t launch_noise_video(const VideoIo* io, float* x_sigma, void* x_act, b
                                int ld_act, cudaStream_t s) {
   return launch_k(noise_video_kernel, dim3(grid_for((size_t)n_rows * P, 256)), dim3(256), 0, s, io, x_sigma, x_act,
                   (int)act_bf16, n_rows, P, ld_act);
+}
+
+cudaError_t launch_patchify(const float* src, float* dst, int B, int F, int C, int H, int W, int p, bool inverse,
+                            cudaStream_t s) {
+  const size_t n = (size_t)B * F * C * H * W;
+  return launch_k(patchify_kernel, dim3(grid_for(n, 256)), dim3(256), 0, s, src, dst, F, C, H, W, p, n,
+                  inverse ? 1 : 0);
 }
 
 cudaError_t launch_copy_out(const ActionIo* io, const float* a_state, int n, cudaStream_t s) {

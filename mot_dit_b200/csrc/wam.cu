@@ -1868,6 +1868,16 @@ wam_status wam_check_device_status(wam_ctx* c) {
   return WAM_OK;
 }
 
+wam_status wam_patchify(const float* frames, float* patches, int B, int F, int C, int H, int W, int p, int inverse,
+                        void* stream) {
+  if (!frames || !patches || B < 1 || F < 1 || C < 1 || p < 1 || H < p || W < p || H % p || W % p)
+    return WAM_ERR_INVALID_ARG;
+  return launch_patchify(inverse ? patches : frames, inverse ? const_cast<float*>(frames) : patches, B, F, C, H, W,
+                         p, inverse != 0, (cudaStream_t)stream) == cudaSuccess
+             ? WAM_OK
+             : WAM_ERR_CUDA;
+}
+
 wam_status wam_test_peer_wait(int extra, unsigned long long limit_ns) {
   if (extra < 0 || (extra > 0 && limit_ns == 0)) return WAM_ERR_INVALID_ARG;
   if (extra == 0) limit_ns = 2000000000ull;  // the kernels' normal limit (2 s)
