@@ -230,21 +230,35 @@ cudaError_t launch_to_f32(const void* src, bool src_bf16, float* dst, size_t n, 
 // ---- persistent action-expert block (action_block.cu) -------------------
 // One launch = [attention of block i,] then up to five weight GEMM phases
 // (out-projection, FFN up, FFN down, next block's QKV or the output map; or
-// in-projection + QKV of block 0), separated by grid barriers.  Batches of at
-// most 32 action tokens, bf16.
-enum : int { kBTma = 0, kBNorm = 1 };  // B operand: TMA of an activation map / RMSNorm+modulation of x_a
+// in-projection + QKV of block 0).  A phase's work units wait only on what
+// they read (per-tile and per-head completion counters), never on a grid-wide
+// barrier.  Batches of at most 32 action tokens, bf16.
+enum : int { kBTma = 0, kBNorm = 1, kBAttn = 2 };  // B operand: TMA of an activation map / RMSNorm+modulation
+                                                     // of x_a / the attention output combined from its splits
+enum : int { kDepNone = 0, kDepAll = 1, kDepKRange = 2, kDepHeads = 3 };
 constexpr int kActionBlockMaps = 11;
+constexpr int kActionBlockPhases = 5;
+constexpr int kActionBlockMaxTiles = 64;  // weight tiles of one phase (n_out <= 8192)
+constexpr int kActionBlockMaxKeys = 192;  // keys per attention unit
 // Tensor maps: 0 w_qkv, 1 w_o, 2 w_f1, 3 w_f2 (3-D, z = block), 4 w_in, 5 w_out,
-// 6 o_a, 7 f_a, 8 a_in (box 64 x 32 rows), 9 q_a and 10 the K/V cache (box 64 x 128 rows).
+// 6 (unused), 7 f_a, 8 a_in (box 64 x 32 rows), 9 q_a (box 64 x 128 rows),
+// 10 the K/V cache (box 64 x keys-per-split rows).
 struct ActionBlockMaps {
   CUtensorMap m[kActionBlockMaps];
 };
 // C[token m, feature n] = sum_k X[m, k] W[n, k] over W [n_out, K] (matrix z
-// of map map_w), split into ks k-ranges per 128-row tile; B = X from map
-// map_b (kBTma) or rms(x_a) * (ngain | 1 + nscale) + nshift (kBNorm).
+// of map map_w), split into ks k-ranges per 128-row tile.  B = X from map
+// map_b (kBTma), rms(x_a) * (ngain | 1 + nscale) + nshift with the row sums of
+// squares from ss buffer ss_in (kBNorm), or the attention output (kBAttn).
+// dep: what the phase's units wait for -- every tile of the previous phase
+// (kDepAll), the previous phase's tiles that cover the unit's k-range
+// (kDepKRange), the attention heads of the unit's k-range (kDepHeads).
+// Epilogues writing x_a also write its per-tile row sums of squares into ss
+// buffer ss_out (-1: none) and, when war_phase >= 0, first wait until every
+// CTA has built that earlier phase's operand (it read x_a).
 struct ActionGemmPhase {
   int map_w, z, n_out, K, ks;
-  int bsrc, map_b;
+  int bsrc, map_b, dep, ss_in, ss_out, war_phase;
   const float* nscale;
   const float* nshift;
   const float* ngain;
@@ -264,25 +278,25 @@ struct ActionGemmPhase {
   int a_next_ld;
 };
 struct ActionAttnPhase {
-  int zk0, zv0;        // cache-map matrix index of (b = 0, h = 0) of K / V
-  int splits;          // 128-key splits of [0, Lk)
-  __nv_bfloat16* out;  // o_a [B * L_a, ld_out]
-  int ld_out;
+  int zk0, zv0;  // cache-map matrix index of (b = 0, h = 0) of K / V
+  int splits;    // key splits of [0, Lk)
+  int keys;      // keys per split (a multiple of 64, <= kActionBlockMaxKeys)
 };
 struct ActionBlockArgs {
   int n_gemm, has_attn;
-  ActionGemmPhase g[5];
+  ActionGemmPhase g[kActionBlockPhases];
   ActionAttnPhase at;
   int Ma, La, H, A, da, Lk, cache_len, cache_off, B;
   const float* x_a;  // fp32 [Ma, da]
+  float* ss;         // row sums of squares of x_a: [2][da / 128][Ma]
   const float* rope_cos;
   const float* rope_sin;
   const ActionIo* aio;
-  float* ws;       // GEMM partial tiles: action_block_ws_floats
+  float* ws;       // GEMM partial tiles: action_block_ws_floats (two halves, by phase parity)
+  size_t ws_half;  // floats per half
   float* ws_attn;  // attention partials: action_block_attn_ws_floats
-  int* cnt;        // 2 * 64 ints, zero on entry, left zero
-  int* cnt_attn;   // 2 * B * H ints, zero on entry, left zero
-  int* bar;        // grid barrier (count, generation), zero at first use
+  int* cnt;        // action_block_cnt_ints: zero at first use, left zero by every launch
+  int* cnt_attn;   // B * H ints, likewise
   unsigned* status;
 };
 // k-splits of a phase with n_out weight rows and reduction K on nsm SMs
@@ -292,9 +306,11 @@ int action_block_ks(int n_out, int K, int nsm);
 bool action_block_fits(int n_out, int K, int ks, int ctas);
 size_t action_block_ws_floats(int max_units);
 size_t action_block_attn_ws_floats(int B, int H, int splits);
-int action_block_attn_splits(int Lk);
+int action_block_cnt_ints();
+// Key splits and keys per split of the attention over Lk keys for B * H heads on nsm SMs.
+void action_block_attn_plan(int Lk, int bh, int nsm, int* splits, int* keys);
 cudaError_t prepare_action_block();
-// `ctas` <= the SM count (one CTA per SM: the grid barriers need the whole grid resident).
+// `ctas` <= the SM count (one CTA per SM: units wait on one another, so the whole grid must be resident).
 cudaError_t launch_action_block(const ActionBlockMaps& m, const ActionBlockArgs& a, int ctas, cudaStream_t s);
 
 // Pixel front-end: frames [B, F, C, H, W] -> patch tokens [B, F (H/p)(W/p), C p p]

@@ -119,17 +119,18 @@ struct wam_ctx {
   // first step, eager action steps) and for the rest.
   bool ab_on = false;
   int ab_ctas = 0, ab_ctas_overlap = 0;
-  int ab_ks_in = 1, ab_ks_qkv = 1, ab_ks_o = 1, ab_ks_f1 = 1, ab_ks_f2 = 1, ab_ks_out = 1, ab_splits = 1;
+  int ab_ks_in = 1, ab_ks_qkv = 1, ab_ks_o = 1, ab_ks_f1 = 1, ab_ks_f2 = 1, ab_ks_out = 1, ab_splits = 1, ab_keys = 64;
   ActionBlockMaps ab_maps;
-  float *ab_ws = nullptr, *ab_ws_attn = nullptr;
-  int *ab_cnt = nullptr, *ab_cnt_attn = nullptr, *ab_bar = nullptr;
+  float *ab_ws = nullptr, *ab_ws_attn = nullptr, *ab_ss = nullptr;
+  size_t ab_ws_half = 0;
+  int *ab_cnt = nullptr, *ab_cnt_attn = nullptr;
 
   // TMA maps
   CUtensorMap m_hv, m_ov, m_fv, m_xvin, m_w_qkv_v, m_w_o_v, m_w_f1_v, m_w_f2_v, m_w_vin, m_w_vout;
   CUtensorMap m_w_in, m_w_qkv_a, m_w_o_a, m_w_f1_a, m_w_f2_a, m_w_out, m_ain, m_ha, m_oa, m_fa;
   CUtensorMap m_la_qkv, m_la_o, m_la_f1, m_la_f2;  // LoRA A factors [r, in] per block
   CUtensorMap m_qv, m_cache;  // video-attention operands
-  CUtensorMap m_qa128, m_cache128;  // action-block attention operands (128-row boxes)
+  CUtensorMap m_qa128, m_cache_ab;  // action-block attention operands (Q: 128-row box; K/V: keys per split)
   // video GEMM outputs (TMA stores, 32-row boxes): x_v fp32, f_v bf16, Q, the K/V cache
   CUtensorMap m_xv_out, m_fv_out, m_qv_out, m_cache_out;
 
@@ -696,19 +697,23 @@ ActionBlockArgs ab_base(wam_ctx* c, const ActionIo* io) {
   a.cache_off = d.Lv;
   a.B = d.B;
   a.x_a = c->x_a;
+  a.ss = c->ab_ss;
   a.rope_cos = c->rope_cos;
   a.rope_sin = c->rope_sin;
   a.aio = io;
   a.ws = c->ab_ws;
+  a.ws_half = c->ab_ws_half;
   a.ws_attn = c->ab_ws_attn;
   a.cnt = c->ab_cnt;
   a.cnt_attn = c->ab_cnt_attn;
-  a.bar = c->ab_bar;
   a.status = c->status;
+  a.at.splits = c->ab_splits;
+  a.at.keys = c->ab_keys;
   return a;
 }
 
-ActionGemmPhase ab_gemm(int map_w, int z, int n_out, int K, int ks, int bsrc, int map_b, int epi, const float* bias) {
+ActionGemmPhase ab_gemm(int map_w, int z, int n_out, int K, int ks, int bsrc, int map_b, int epi, const float* bias,
+                        int dep) {
   ActionGemmPhase g{};
   g.map_w = map_w;
   g.z = z;
@@ -719,6 +724,10 @@ ActionGemmPhase ab_gemm(int map_w, int z, int n_out, int K, int ks, int bsrc, in
   g.map_b = map_b;
   g.epi = epi;
   g.bias = bias;
+  g.dep = dep;
+  g.ss_in = -1;
+  g.ss_out = -1;
+  g.war_phase = -1;
   return g;
 }
 
@@ -727,7 +736,8 @@ ActionGemmPhase ab_qkv(wam_ctx* c, int i) {
   const Dims& d = c->d;
   const ExpertIdx& x = c->ea;
   const float* mod = c->mod_a + (size_t)i * 6 * d.da;
-  ActionGemmPhase g = ab_gemm(0, i, 3 * d.A, d.da, c->ab_ks_qkv, kBNorm, 0, kEpiQkv, vecp(c, blk(x, i, kQkvB)));
+  ActionGemmPhase g = ab_gemm(0, i, 3 * d.A, d.da, c->ab_ks_qkv, kBNorm, 0, kEpiQkv, vecp(c, blk(x, i, kQkvB)), kDepAll);
+  g.ss_in = 1;  // x_a's row sums from the FFN-down (or in-projection) tiles
   g.nscale = mod + d.da;
   g.nshift = mod;
   g.gq = vecp(c, blk(x, i, kQnG));
@@ -758,9 +768,10 @@ wam_status enqueue_action_step_blocks(wam_ctx* c, cudaStream_t s, const ActionIo
   const int ctas = ev_wait ? c->ab_ctas_overlap : c->ab_ctas;
   {
     ActionBlockArgs a = ab_base(c, io);
-    ActionGemmPhase in = ab_gemm(4, 0, d.da, d.Kin, c->ab_ks_in, kBTma, 8, kEpiStoreF32, vecp(c, x.inb));
+    ActionGemmPhase in = ab_gemm(4, 0, d.da, d.Kin, c->ab_ks_in, kBTma, 8, kEpiStoreF32, vecp(c, x.inb), kDepNone);
     in.out_f32 = c->x_a;
     in.ld_out = d.da;
+    in.ss_out = 1;
     a.g[a.n_gemm++] = in;
     a.g[a.n_gemm++] = ab_qkv(c, 0);
     RET(ab_launch(c, a, ctas, s));
@@ -773,29 +784,33 @@ wam_status enqueue_action_step_blocks(wam_ctx* c, cudaStream_t s, const ActionIo
     a.has_attn = 1;
     a.at.zk0 = (2 * i) * d.B * d.H;
     a.at.zv0 = (2 * i + 1) * d.B * d.H;
-    a.at.splits = c->ab_splits;
-    a.at.out = reinterpret_cast<__nv_bfloat16*>(c->o_a);
-    a.at.ld_out = d.lo;
-    ActionGemmPhase o = ab_gemm(1, i, d.da, d.A, c->ab_ks_o, kBTma, 6, kEpiGateRes, vecp(c, blk(x, i, kOB)));
+    // out-projection: B = the attention output, combined from its splits
+    ActionGemmPhase o = ab_gemm(1, i, d.da, d.A, c->ab_ks_o, kBAttn, 0, kEpiGateRes, vecp(c, blk(x, i, kOB)), kDepHeads);
     o.gate = mod + 2 * d.da;
     o.out_f32 = c->x_a;
     o.ld_out = d.da;
+    o.ss_out = 0;
     a.g[a.n_gemm++] = o;
-    ActionGemmPhase f1 = ab_gemm(2, i, d.Fa, d.da, c->ab_ks_f1, kBNorm, 0, kEpiGelu, vecp(c, blk(x, i, kF1B)));
+    ActionGemmPhase f1 = ab_gemm(2, i, d.Fa, d.da, c->ab_ks_f1, kBNorm, 0, kEpiGelu, vecp(c, blk(x, i, kF1B)), kDepAll);
+    f1.ss_in = 0;
     f1.nscale = mod + 4 * d.da;
     f1.nshift = mod + 3 * d.da;
     f1.out_act = reinterpret_cast<__nv_bfloat16*>(c->f_a);
     f1.ld_out = d.lf;
     a.g[a.n_gemm++] = f1;
-    ActionGemmPhase f2 = ab_gemm(3, i, d.da, d.Fa, c->ab_ks_f2, kBTma, 7, kEpiGateRes, vecp(c, blk(x, i, kF2B)));
+    ActionGemmPhase f2 = ab_gemm(3, i, d.da, d.Fa, c->ab_ks_f2, kBTma, 7, kEpiGateRes, vecp(c, blk(x, i, kF2B)),
+                                 kDepKRange);
     f2.gate = mod + 5 * d.da;
     f2.out_f32 = c->x_a;
     f2.ld_out = d.da;
+    f2.ss_out = 1;
+    f2.war_phase = 1;  // FFN-up's operand reads x_a: every CTA has built it before x_a changes
     a.g[a.n_gemm++] = f2;
     if (i + 1 < d.N) {
       a.g[a.n_gemm++] = ab_qkv(c, i + 1);
     } else {
-      ActionGemmPhase out = ab_gemm(5, 0, d.Pa, d.da, c->ab_ks_out, kBNorm, 0, kEpiEuler, vecp(c, x.outb));
+      ActionGemmPhase out = ab_gemm(5, 0, d.Pa, d.da, c->ab_ks_out, kBNorm, 0, kEpiEuler, vecp(c, x.outb), kDepAll);
+      out.ss_in = 1;
       out.ngain = vecp(c, x.fng);
       out.out_f32 = c->a_state;
       out.ld_out = d.Pa;
@@ -1098,7 +1113,7 @@ void wam_destroy(wam_ctx* c) {
                   c->mod_v, c->mod_a, c->temb_v, c->temb_a, c->rope_cos, c->rope_sin, c->ws_gemm, c->tk_gemm, c->ws_gemm_v, c->tk_gemm_v, c->zero_r,
                   c->ws_attn, c->tk_attn, c->status, c->vio_chunk, c->vio_eager, c->aio_chunk, c->aio_eager,
                   c->h_video, c->h_cond, c->h_noise, c->h_out, c->j_vout, c->j_aout, c->ab_ws, c->ab_ws_attn,
-                  c->ab_cnt, c->ab_cnt_attn, c->ab_bar, c->td_at, c->td_as, c->td_a0, c->td_fs, c->td_fe,
+                  c->ab_ss, c->ab_cnt, c->ab_cnt_attn, c->td_at, c->td_as, c->td_a0, c->td_fs, c->td_fe,
                   c->aio_tacd};
   for (void* p : bufs)
     if (p) cudaFree(p);
@@ -1374,8 +1389,8 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
       c->ab_ks_f1 = action_block_ks(d.Fa, d.da, nsm);
       c->ab_ks_f2 = action_block_ks(d.da, d.Fa, nsm);
       c->ab_ks_out = action_block_ks(d.Pa, d.da, nsm);
-      c->ab_splits = action_block_attn_splits(d.Lv + d.La);
-      bool fits = (3 * d.A + 127) / 128 <= 64 && (d.Fa + 127) / 128 <= 64;
+      action_block_attn_plan(d.Lv + d.La, d.B * d.H, nsm, &c->ab_splits, &c->ab_keys);
+      bool fits = (3 * d.A + 127) / 128 <= 64 && (d.Fa + 127) / 128 <= 64 && d.da % 128 == 0 && d.Dh == 64;
       for (int g : {c->ab_ctas, c->ab_ctas_overlap}) {
         fits = fits && action_block_fits(d.da, d.Kin, c->ab_ks_in, g) && action_block_fits(3 * d.A, d.da, c->ab_ks_qkv, g) &&
                action_block_fits(d.da, d.A, c->ab_ks_o, g) && action_block_fits(d.Fa, d.da, c->ab_ks_f1, g) &&
@@ -1386,17 +1401,19 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
         int mu = std::max({units(d.da, c->ab_ks_in), units(3 * d.A, c->ab_ks_qkv), units(d.da, c->ab_ks_o),
                            units(d.Fa, c->ab_ks_f1), units(d.da, c->ab_ks_f2), units(d.Pa, c->ab_ks_out)});
         CK(prepare_action_block());
+        c->ab_ws_half = action_block_ws_floats(mu) / 2;
         RET(dalloc(c, &c->ab_ws, action_block_ws_floats(mu) * 4));
         RET(dalloc(c, &c->ab_ws_attn, action_block_attn_ws_floats(d.B, d.H, c->ab_splits) * 4));
-        RET(dalloc(c, &c->ab_cnt, 2 * 64 * 4));
-        RET(dalloc(c, &c->ab_cnt_attn, (size_t)2 * d.B * d.H * 4));
-        RET(dalloc(c, &c->ab_bar, 2 * 4));
+        RET(dalloc(c, &c->ab_ss, (size_t)2 * (d.da / 128) * d.Ma * 4));
+        RET(dalloc(c, &c->ab_cnt, (size_t)action_block_cnt_ints() * 4));
+        RET(dalloc(c, &c->ab_cnt_attn, (size_t)d.B * d.H * 4));
         bool mok = make_tmap_3d(&c->m_qa128, c->q_a, d.Dh, d.La, d.B * d.H, (size_t)d.La * d.Dh * 2, 128) &&
-                   make_tmap_3d(&c->m_cache128, c->kv, d.Dh, d.Ltot, 2 * d.N * d.B * d.H, (size_t)d.Ltot * d.Dh * 2, 128);
+                   make_tmap_3d(&c->m_cache_ab, c->kv, d.Dh, d.Ltot, 2 * d.N * d.B * d.H, (size_t)d.Ltot * d.Dh * 2,
+                                c->ab_keys);
         if (!mok) return fail(c, WAM_ERR_CUDA, "tensor map creation failed");
         const CUtensorMap* mm[kActionBlockMaps] = {&c->m_w_qkv_a, &c->m_w_o_a, &c->m_w_f1_a, &c->m_w_f2_a,
                                                    &c->m_w_in,    &c->m_w_out, &c->m_oa,    &c->m_fa,
-                                                   &c->m_ain,     &c->m_qa128, &c->m_cache128};
+                                                   &c->m_ain,     &c->m_qa128, &c->m_cache_ab};
         for (int k = 0; k < kActionBlockMaps; ++k) c->ab_maps.m[k] = *mm[k];
         c->ab_on = true;
       }
@@ -1858,9 +1875,8 @@ wam_status wam_check_device_status(wam_ctx* c) {
     CK(cudaMemset(c->status, 0, 4));
     if (c->tk_gemm) CK(cudaMemset(c->tk_gemm, 0, c->tk_gemm_bytes));
     if (c->tk_gemm_v) CK(cudaMemset(c->tk_gemm_v, 0, c->tk_gemm_v_bytes));
-    if (c->ab_cnt) CK(cudaMemset(c->ab_cnt, 0, 2 * 64 * 4));
-    if (c->ab_cnt_attn) CK(cudaMemset(c->ab_cnt_attn, 0, (size_t)2 * c->d.B * c->d.H * 4));
-    if (c->ab_bar) CK(cudaMemset(c->ab_bar, 0, 2 * 4));
+    if (c->ab_cnt) CK(cudaMemset(c->ab_cnt, 0, (size_t)action_block_cnt_ints() * 4));
+    if (c->ab_cnt_attn) CK(cudaMemset(c->ab_cnt_attn, 0, (size_t)c->d.B * c->d.H * 4));
     if (c->tk_attn) CK(cudaMemset(c->tk_attn, 0, (size_t)c->d.B * c->d.H * 4));
     CK(cudaDeviceSynchronize());
     return fail(c, WAM_ERR_TIMEOUT, "device bounded wait gave up (status bits 0x%x)", st);
