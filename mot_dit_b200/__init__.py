@@ -22,6 +22,7 @@ from ._binding import (  # noqa: F401
     op_attention,
     op_attention_noalloc,
     op_linear,
+    op_linear_tiled,
     op_norm_mod,
     patchify,
     preset,

@@ -84,6 +84,7 @@ def lib():
         "wam_status_str": (C.c_char_p, [C.c_int]),
         "wam_last_error": (C.c_char_p, [_P]),
         "wam_op_linear": (C.c_int, [C.c_int, _P, _P, _P, _P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _P]),
+        "wam_op_linear_tiled": (C.c_int, [_P, _P, _P, _P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _P]),
         "wam_op_attention": (C.c_int, [C.c_int, _P, _P, _P, _P] + [C.c_int] * 7 + [_P]),
         "wam_op_attention_noalloc": (C.c_int, [_P, _P, _P, _P] + [C.c_int] * 6 + [_P]),
         "wam_op_norm_mod": (C.c_int, [C.c_int, _P, _P, C.c_int, C.c_int, _P, _P, _P, _P]),
@@ -317,6 +318,13 @@ def op_linear(dtype, x, w, bias, out, M, N, K, swap=False, splits=1, stream=None
                              _stream(stream))
     if st:
         raise WamError(st, "wam_op_linear")
+
+
+def op_linear_tiled(x, w, bias, out, M, N, K, bn=256, pair=True, ctas=0, stream=None):
+    st = lib().wam_op_linear_tiled(_ptr(x), _ptr(w), _ptr(bias), _ptr(out), M, N, K, bn, int(pair), ctas,
+                                   _stream(stream))
+    if st:
+        raise WamError(st, "wam_op_linear_tiled")
 
 
 def op_norm_mod(dtype, x, h, M, d, scale=None, shift=None, gain=None, stream=None):

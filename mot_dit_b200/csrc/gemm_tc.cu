@@ -64,12 +64,18 @@ enum : int {
 // Largest reduction length of the fused-norm B operand (held whole in shared memory).
 constexpr int kNormKMax = 1024;
 
-template <int BN, bool SWAP, int EPI>
+// PAIR: the CTA is one of a pair sharing an M = 256 MMA (normal orientation):
+// it loads its own 128 A rows and half of the tile's BN B rows, and its
+// output tile is still 128 x BN.
+template <int BN, bool SWAP, int EPI, bool PAIR = false>
 struct TileCfg {
   static constexpr bool kNB = EPI == kClassNormB;
   static_assert(!kNB || (SWAP && BN <= 64), "fused-norm B operand: swapped orientation, <= 64 tokens");
+  static_assert(!PAIR || (!SWAP && BN == 256 && (EPI == kClassStore || EPI == kClassRes || EPI == kClassQkv)),
+                "CTA pairs: normal orientation, 256-wide tiles, TMA-store epilogues");
   static constexpr int kABytes = BM * BK * 2;
-  static constexpr int kBBytes = kNB ? 0 : BN * BK * 2;  // per stage
+  static constexpr int kBRows = PAIR ? BN / 2 : BN;      // B rows this CTA loads
+  static constexpr int kBBytes = kNB ? 0 : kBRows * BK * 2;  // per stage
   static constexpr int kStageBytes = kABytes + kBBytes;
   // fused-norm B operand, resident: [k-block][BN rows][128 B], 128-byte swizzle
   static constexpr int kResB = kNB ? (kNormKMax / BK) * BN * 128 : 0;
@@ -142,6 +148,78 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 }
 // Later async-proxy reads of global memory see what this thread has observed.
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// ---- CTA pairs (2-SM MMA): two CTAs of a cluster of two share one M = 256
+// tensor-core tile.  Rank 0 issues the MMAs; each CTA holds its 128 A rows
+// and half of the B rows at the same shared-memory offsets, and its 128 rows
+// of the accumulator in its own TMEM.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of both CTAs; orders every earlier memory operation (remote
+// mbarrier arrivals included) before anything after it in the other CTA.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address, in the cluster's shared window, of the same object in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+// TMEM allocation of a pair: the same warp of both CTAs, same slot offset.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// 3-D tiled load into this CTA's shared memory whose bytes complete on the
+// barrier at cluster address `bar` -- a barrier of either CTA of the pair
+// (the 2-SM form of the load; no multicast).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+// D (both CTAs' TMEM) (+)= A (both CTAs' rows) * B (both CTAs' halves)^T.
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the barrier at cluster address `addr` (this CTA's or the peer's)
+// once every pair MMA issued so far by this thread completes.
+__device__ __forceinline__ void tc_commit_pair(uint32_t addr) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(addr)
+               : "memory");
+}
+
+#ifdef WAM_GEMM_TIMELINE
+// Diagnostic build only: per CTA of the last launch, %smid and %globaltimer
+// at start, first MMA issue (rank 0 / single CTA), last MMA issue and end.
+__device__ unsigned long long g_gemm_tl[1024][10];
+#define WAM_TL(slot, v) \
+  if (blockIdx.x < 1024) g_gemm_tl[blockIdx.x][slot] = (v)
+#else
+#define WAM_TL(slot, v)
+#endif
 
 // Failure-path test hook (wam_test_peer_wait): the last piece of a split tile
 // that is its CTA's final segment waits for g_peer_wait_extra more published
@@ -355,12 +433,12 @@ __device__ __forceinline__ Seg seg_at(const GemmK& g, long long x, long long x_e
   return s;
 }
 
-template <int BN, bool SWAP, int EPI>
+template <int BN, bool SWAP, int EPI, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                    const __grid_constant__ CUtensorMap map_o, const __grid_constant__ CUtensorMap map_o2,
                    const GemmK g, const EpiArgs e) {
-  using C = TileCfg<BN, SWAP, EPI>;
+  using C = TileCfg<BN, SWAP, EPI, PAIR>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The 128-byte swizzle is a function of the address bits: every tile must
   // start on a 1024-byte boundary.
@@ -368,6 +446,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) atomicOr(g.status, kStatusTimeoutDrain);
     return;
   }
+#ifdef WAM_GEMM_TIMELINE
+  if (threadIdx.x == 0) {
+    unsigned sm;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    WAM_TL(0, sm);
+    WAM_TL(1, globaltimer());
+  }
+#endif
   uint8_t* smem = smem_raw;
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kStages * C::kABytes;
@@ -385,16 +471,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long x_begin = kbound(g, blockIdx.x), x_end = kbound(g, blockIdx.x + 1);
+  // Stream-K unit: the CTA, or the CTA pair (both CTAs of a pair run the same
+  // segments; rank 1 takes the odd 128-row tile of each 256-row pair tile).
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const long long x_begin = kbound(g, unit), x_end = kbound(g, unit + 1);
 
   if (threadIdx.x == 0) {
+    // rank 0 of a pair: an accumulator is drained once both CTAs'
+    // epilogues are done (the peer's stage bytes complete on rank 0's full
+    // barriers, which expect both CTAs' bytes)
+    const bool lead = PAIR && rank == 0;
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accf[b], 1);
-      mbar_init(&acce[b], 4);
+      mbar_init(&acce[b], lead ? 8 : 4);
     }
     mbar_init(redb, 1);
     mbar_init(bready, 1);
@@ -409,19 +503,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!SWAP && EPI == kClassQkv) prefetch_tensormap(&map_o2);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the peer's barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_trigger();  // the next kernel may start its own set-up now
+
+  // first rows of this CTA's A and B loads for tile (ta, tb)
+  auto arow = [&](int ta) { return SWAP ? ta * BM : (PAIR ? 2 * ta + (int)rank : ta) * BM; };
+  auto brow = [&](int tb) { return SWAP ? tb * BN : tb * BN + (PAIR ? (int)rank * C::kBRows : 0); };
 
   if (warp == 0) {
     if (lane == 0) {
       int it = 0, issued = 0;
       bool ok = true;
+      // Stage st's loads.  A pair's stage is one barrier, rank 0's: rank 0
+      // arms it for both CTAs' bytes and the peer's loads complete on it.
+      const bool peer = PAIR && rank == 1;
+      auto arm = [&](int st) {
+        if (!peer) mbar_arrive_expect_tx(&full[st], (PAIR ? 2 : 1) * C::kStageBytes);
+      };
+      auto load = [&](const CUtensorMap* map, uint8_t* dst, int st, int kb, int y, int z) {
+        if (peer)
+          tma_load_3d_pair(dst, map, cluster_addr(&full[st], 0), kb * BK, y, z);
+        else
+          tma_load_3d(dst, map, &full[st], kb * BK, y, z);
+      };
       // The weights never change during a chunk: the first segment's weight
       // tiles are requested before waiting for the previous kernel.
       int pre = 0;
@@ -430,19 +546,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ta = sg.t % g.tiles_a, tb = sg.t / g.tiles_a;
         pre = min(C::kStages, sg.kb1 - sg.kb0);
         for (int i = 0; i < pre; ++i) {
-          mbar_arrive_expect_tx(&full[i], C::kStageBytes);
+          arm(i);
           if (SWAP)
-            tma_load_3d(sA + i * C::kABytes, &map_a, &full[i], (sg.kb0 + i) * BK, ta * BM, g.z_a);
+            load(&map_a, sA + i * C::kABytes, i, sg.kb0 + i, arow(ta), g.z_a);
           else
-            tma_load_3d(sB + i * C::kBBytes, &map_b, &full[i], (sg.kb0 + i) * BK, tb * BN, g.z_b);
+            load(&map_b, sB + i * C::kBBytes, i, sg.kb0 + i, brow(tb), g.z_b);
         }
         // with the fused norm the producer reads weights only: no wait for the previous kernel
         if (!C::kNB) pdl_wait();
         for (int i = 0; i < pre && !C::kNB; ++i) {
           if (SWAP)
-            tma_load_3d(sB + i * C::kBBytes, &map_b, &full[i], (sg.kb0 + i) * BK, tb * BN, g.z_b);
+            load(&map_b, sB + i * C::kBBytes, i, sg.kb0 + i, brow(tb), g.z_b);
           else
-            tma_load_3d(sA + i * C::kABytes, &map_a, &full[i], (sg.kb0 + i) * BK, ta * BM, g.z_a);
+            load(&map_a, sA + i * C::kABytes, i, sg.kb0 + i, arow(ta), g.z_a);
         }
         issued = pre;
       } else if (!C::kNB) {
@@ -460,19 +576,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-          tma_load_3d(sA + s * C::kABytes, &map_a, &full[s], kb * BK, ta * BM, g.z_a);
-          if (!C::kNB) tma_load_3d(sB + s * C::kBBytes, &map_b, &full[s], kb * BK, tb * BN, g.z_b);
+          arm(s);
+          load(&map_a, sA + s * C::kABytes, s, kb, arow(ta), g.z_a);
+          if (!C::kNB) load(&map_b, sB + s * C::kBBytes, s, kb, brow(tb), g.z_b);
           issued = it + 1;
         }
       }
-      // Drain: never leave the CTA with copies into its shared memory in flight.
-      for (int i = max(0, issued - C::kStages); i < issued; ++i)
-        mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1, g.status, kStatusTimeoutDrain, nullptr);
+      // Drain: never leave the CTA with copies into its shared memory in
+      // flight (a pair's rank 0 waits for both CTAs' bytes; the peer's
+      // arrive there) ...
+      if (!peer)
+        for (int i = max(0, issued - C::kStages); i < issued; ++i)
+          mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1, g.status, kStatusTimeoutDrain, nullptr);
+      if constexpr (PAIR) {
+        // ... nor with the pair's MMAs still reading it: the commits of the
+        // last stages have arrived (every issued stage is consumed first;
+        // one shared limit for all of them)
+        volatile int gave_up = 0;
+        for (int i = max(0, issued - C::kStages); i < issued; ++i)
+          mbar_wait(&empty[i % C::kStages], (i / C::kStages) & 1, g.status, kStatusTimeoutDrain, &gave_up);
+      }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+    if (PAIR && rank == 1) {
+      // the peer's MMA warp has nothing to issue: rank 0 runs the pair's MMAs
+    } else if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * BM : BM, BN);
       int it = 0, lt = 0;
       bool ok = true;
       if (C::kNB && x_begin < x_end) {  // the B operand is computed by the epilogue warps
@@ -483,7 +612,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Seg sg = seg_at(g, x, x_end);
         x += sg.kb1 - sg.kb0;
         const int buf = lt & 1;
-        if (lt >= 2 && !mbar_wait(&acce[buf], ((lt >> 1) - 1) & 1, g.status, kStatusTimeoutAccum, abort_flag)) {
+        if (lt >= 2 &&
+            !mbar_wait(&acce[buf], ((lt >> 1) - 1) & 1, g.status, kStatusTimeoutAccum, abort_flag)) {
           ok = false;
           break;
         }
@@ -496,15 +626,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
+          if (it == 0) WAM_TL(2, globaltimer());
+          WAM_TL(3, globaltimer());
           const uint32_t a0 = smem_u32(sA + s * C::kABytes);
           const uint32_t b0 = C::kNB ? smem_u32(sBres + kb * (BN * 128)) : smem_u32(sB + s * C::kBBytes);
+          if constexpr (PAIR) {
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            tc_mma_bf16(d_tmem, smem_desc_k128(a0 + k * 32), smem_desc_k128(b0 + k * 32), idesc,
-                        (kb > sg.kb0 || k > 0) ? 1u : 0u);
-          tc_commit(&empty[s]);
+            for (int k = 0; k < BK / 16; ++k)
+              tc_mma_bf16_pair(d_tmem, smem_desc_k128(a0 + k * 32), smem_desc_k128(b0 + k * 32), idesc,
+                               (kb > sg.kb0 || k > 0) ? 1u : 0u);
+            tc_commit_pair(smem_u32(&empty[s]));  // both CTAs may refill the stage
+            tc_commit_pair(cluster_addr(&empty[s], 1));
+          } else {
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              tc_mma_bf16(d_tmem, smem_desc_k128(a0 + k * 32), smem_desc_k128(b0 + k * 32), idesc,
+                          (kb > sg.kb0 || k > 0) ? 1u : 0u);
+            tc_commit(&empty[s]);
+          }
         }
-        tc_commit(&accf[buf]);
+        if constexpr (PAIR) {
+          tc_commit_pair(smem_u32(&accf[buf]));  // both CTAs' accumulator halves are ready
+          tc_commit_pair(cluster_addr(&accf[buf], 1));
+        } else {
+          tc_commit(&accf[buf]);
+        }
       }
     }
     __syncwarp();
@@ -604,7 +750,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int c_first = kowner(g, t0);
       const int npieces = kowner(g, t0 + g.KB - 1) - c_first + 1;
       const int buf = lt & 1;
-      const int m0w = ta * BM + quad * 32;  // normal orientation: this warp's first row
+      const int m0w = arow(ta) + quad * 32;  // normal orientation: this warp's first row
+      const int tk = PAIR ? 2 * t + (int)rank : t;  // the tickets of this CTA's 128-row tile
       const int nb = tb * BN;
 
       // ---- prefetch while the MMA of this segment runs
@@ -683,15 +830,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto release = [&]() {  // this warp's TMEM reads of the buffer are done
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acce[buf]);
+        if (lane == 0) {
+          if (PAIR && rank == 1)
+            mbar_arrive_cluster(cluster_addr(&acce[buf], 0));  // the MMAs are issued by rank 0
+          else
+            mbar_arrive(&acce[buf]);
+        }
       };
 
+      if (threadIdx.x == 64 && x == x_end) WAM_TL(5, globaltimer());  // last segment's accumulator ready
       // ---- a tile shared with other CTAs (see "Split tiles" above)
-      const int mine = (int)blockIdx.x - c_first;  // this CTA's piece of tile t
+      const int mine = unit - c_first;  // this CTA's piece of tile t
+      // CTA holding piece p's partial (the same rank of the piece's pair)
+      auto piece_cta = [&](int p) { return PAIR ? 2 * (c_first + p) + (int)rank : c_first + p; };
       bool from_smem = false;
       if (npieces > 1) {
         if (threadIdx.x == 64) {
-          const int prev = atomicAdd(g.tickets + 2 * t, 1);
+          const int prev = atomicAdd(g.tickets + 2 * tk, 1);
           *last_flag = (prev == npieces - 1) ? 1 : 0;
         }
         epi_bar();
@@ -709,18 +864,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __threadfence();
           epi_bar();
-          if (threadIdx.x == 64) atomicAdd(g.tickets + 2 * t + 1, 1);
+          if (threadIdx.x == 64) atomicAdd(g.tickets + 2 * tk + 1, 1);
+          if (threadIdx.x == 64 && x == x_end) WAM_TL(9, globaltimer());  // published (not the reducer)
           continue;
         }
         // the last arrival reduces: the others have arrived; wait until they have published
         if (threadIdx.x == 64) {
           const bool hooked = x == x_end && g_peer_wait_extra > 0;
-          if (!wait_count(g.tickets + 2 * t + 1, npieces - 1 + (hooked ? g_peer_wait_extra : 0), g.status, abort_flag,
+          if (!wait_count(g.tickets + 2 * tk + 1, npieces - 1 + (hooked ? g_peer_wait_extra : 0), g.status, abort_flag,
                           hooked ? g_peer_wait_limit_ns : kWaitLimitNs)) {
             *abort_flag = 1;
           } else {
-            g.tickets[2 * t] = 0;  // every piece is done with the tickets
-            g.tickets[2 * t + 1] = 0;
+            g.tickets[2 * tk] = 0;  // every piece is done with the tickets
+            g.tickets[2 * tk + 1] = 0;
             __threadfence();
             constexpr uint32_t kPart = BM * BN * 4;
             if (x == x_end && (uint32_t)(npieces - 1) * kPart <= (uint32_t)(C::kStages * C::kStageBytes)) {
@@ -732,7 +888,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (p == mine) continue;
                 const int cp = c_first + p;
                 const int slot = (p == 0 && t0 != kbound(g, cp)) ? 1 : 0;
-                const uint8_t* src = reinterpret_cast<const uint8_t*>(g.ws + ((size_t)cp * 2 + slot) * (BM * BN));
+                const uint8_t* src =
+                    reinterpret_cast<const uint8_t*>(g.ws + ((size_t)piece_cta(p) * 2 + slot) * (BM * BN));
                 for (uint32_t o = 0; o < kPart; o += 32768)
                   bulk_load(smem + k * kPart + o, src + o, min(32768u, kPart - o), redb);
                 ++k;
@@ -743,6 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         epi_bar();
         if (*abort_flag) break;
+        if (threadIdx.x == 64 && x == x_end) WAM_TL(6, globaltimer());  // partners published (reducer)
         from_smem = *last_flag == 2;
         if (from_smem) {
           // at most one bulk reduction per CTA (its last segment): phase 0
@@ -782,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             const int cp = c_first + p;
             const int slot = (p == 0 && t0 != kbound(g, cp)) ? 1 : 0;
-            const float* src = g.ws + ((size_t)cp * 2 + slot) * (BM * BN) + off;
+            const float* src = g.ws + ((size_t)piece_cta(p) * 2 + slot) * (BM * BN) + off;
 #pragma unroll
             for (int j = 0; j < 8; ++j) t4[j] = __ldcg(reinterpret_cast<const float4*>(src + (size_t)j * BM * 4));
           }
@@ -1034,8 +1192,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if (threadIdx.x == 64) WAM_TL(7, globaltimer());  // epilogue loop done
     // the warp's bulk stores are complete before the CTA's shared memory goes away
     if (!SWAP && EPI != kClassScalar && lane == 0) bulk_wait_all();
+    if (threadIdx.x == 64) WAM_TL(8, globaltimer());
     __syncwarp();
   }
 
@@ -1054,24 +1214,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&accf[l & 1], (l >> 1) & 1, g.status, kStatusTimeoutDrain, nullptr);
     }
     __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
   }
+  // A pair stays until both CTAs are done: rank 0's MMAs read the peer's
+  // shared memory, and each CTA arrives on the other's barriers.
+  if constexpr (PAIR) cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem, C::kTmemCols);
+    else
+      tmem_dealloc(tmem, C::kTmemCols);
+  }
+  if (threadIdx.x == 0) WAM_TL(4, globaltimer());
 }
 
-template <int BN, bool SWAP, int EPI>
+template <int BN, bool SWAP, int EPI, bool PAIR = false>
 cudaError_t prepare_one() {
-  return cudaFuncSetAttribute(tc_gemm_kernel<BN, SWAP, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TileCfg<BN, SWAP, EPI>::kSmem);
+  return cudaFuncSetAttribute(tc_gemm_kernel<BN, SWAP, EPI, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TileCfg<BN, SWAP, EPI, PAIR>::kSmem);
 }
 
 int g_num_sms = 0;
+int g_max_pairs = 0;  // clusters of two 227 KB CTAs the device holds at once
 
-// Persistent grid size: swapped -- tiles x splits; normal -- max_ctas or one
-// per SM; never more CTAs than k-blocks.
-int ctas_of(const TcGemm& t) {
+// Launch as clusters of two CTAs (pairs of SMs), with programmatic dependent
+// launch like launch_k.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pairs(void (*kernel)(KArgs...), int pairs, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Output rows of one tile row (the stream-K tile): 128, or 256 for a pair.
+int tile_rows(const TcGemm& t) { return t.pair ? 2 * BM : BM; }
+
+// Stream-K units of a launch (CTAs, or CTA pairs): swapped -- tiles x splits;
+// normal -- max_ctas (or one CTA per SM), halved for pairs; never more units
+// than k-blocks.
+int units_of(const TcGemm& t) {
   const int kb = (t.K + BK - 1) / BK;
-  const long long tiles = (long long)((t.rows_a + BM - 1) / BM) * ((t.rows_b + t.bn - 1) / t.bn);
+  const long long tiles = (long long)((t.rows_a + tile_rows(t) - 1) / tile_rows(t)) * ((t.rows_b + t.bn - 1) / t.bn);
   long long want;
   if (t.swap) {
     int splits = t.splits < 1 ? 1 : t.splits;
@@ -1079,57 +1274,73 @@ int ctas_of(const TcGemm& t) {
     want = tiles * splits;
   } else {
     want = t.max_ctas > 0 ? t.max_ctas : g_num_sms;
+    if (t.pair) {
+      want /= 2;
+      if (g_max_pairs > 0 && want > g_max_pairs) want = g_max_pairs;
+    }
   }
   const long long W = tiles * kb;
   if (want > W) want = W;
   if (want < 1) want = 1;
   return (int)want;
 }
+int ctas_of(const TcGemm& t) { return units_of(t) * (t.pair ? 2 : 1); }
 
-template <int BN, bool SWAP, int EPI>
+template <int BN, bool SWAP, int EPI, bool PAIR = false>
 cudaError_t launch_one(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
-  using C = TileCfg<BN, SWAP, EPI>;
+  using C = TileCfg<BN, SWAP, EPI, PAIR>;
   GemmK g;
   g.rows_a = t.rows_a;
   g.rows_b = t.rows_b;
   g.K = t.K;
   g.z_a = t.z_a;
   g.z_b = t.z_b;
-  g.tiles_a = (t.rows_a + BM - 1) / BM;
+  g.tiles_a = (t.rows_a + tile_rows(t) - 1) / tile_rows(t);
   g.KB = (t.K + BK - 1) / BK;
   g.W = (long long)g.tiles_a * ((t.rows_b + BN - 1) / BN) * g.KB;
-  g.G = ctas_of(t);
+  g.G = units_of(t);
   g.ws = t.ws;
   g.tickets = t.tickets;
   g.status = t.status;
   // unused output maps are passed as copies of the A map
   const CUtensorMap& mo = e.map_o ? *e.map_o : *t.map_a;
   const CUtensorMap& mo2 = e.map_o2 ? *e.map_o2 : *t.map_a;
-  return launch_k(tc_gemm_kernel<BN, SWAP, EPI>, dim3(g.G), dim3(kThreads), C::kSmem, s, *t.map_a, *t.map_b, mo, mo2,
-                  g, e);
+  if constexpr (PAIR)
+    return launch_pairs(tc_gemm_kernel<BN, SWAP, EPI, true>, g.G, C::kSmem, s, *t.map_a, *t.map_b, mo, mo2, g, e);
+  else
+    return launch_k(tc_gemm_kernel<BN, SWAP, EPI, false>, dim3(g.G), dim3(kThreads), C::kSmem, s, *t.map_a, *t.map_b,
+                    mo, mo2, g, e);
 }
 
-template <int BN>
+template <int BN, bool PAIR = false>
 cudaError_t launch_normal(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
   switch (e.kind) {
     case kEpiStoreF32:
     case kEpiGelu:
       if (!e.map_o) return cudaErrorInvalidValue;
-      return launch_one<BN, false, kClassStore>(t, e, s);
+      return launch_one<BN, false, kClassStore, PAIR>(t, e, s);
     case kEpiGateRes:
       if (!e.map_o) return cudaErrorInvalidValue;
-      return launch_one<BN, false, kClassRes>(t, e, s);
+      return launch_one<BN, false, kClassRes, PAIR>(t, e, s);
     case kEpiQkv:
       if (!e.map_o || !e.map_o2) return cudaErrorInvalidValue;
-      return launch_one<BN, false, kClassQkv>(t, e, s);
+      return launch_one<BN, false, kClassQkv, PAIR>(t, e, s);
     default:
-      return launch_one<BN, false, kClassScalar>(t, e, s);
+      if constexpr (PAIR)
+        return cudaErrorInvalidValue;  // per-element epilogues run on single CTAs
+      else
+        return launch_one<BN, false, kClassScalar>(t, e, s);
   }
 }
 
 }  // namespace
 
 size_t tc_gemm_ws_floats(const TcGemm& t) { return (size_t)ctas_of(t) * 2 * BM * t.bn; }
+
+size_t tc_gemm_tickets(const TcGemm& t) {
+  const int row_tiles = ((t.rows_a + tile_rows(t) - 1) / tile_rows(t)) * (t.pair ? 2 : 1);
+  return (size_t)2 * row_tiles * ((t.rows_b + t.bn - 1) / t.bn);
+}
 
 namespace {
 template <int BN, bool SWAP, int EPI>
@@ -1178,8 +1389,43 @@ cudaError_t prepare_tc_gemm() {
   WAM_PREP(256, false, kClassQkv)
   WAM_PREP(256, false, kClassRes)
 #undef WAM_PREP
+  if ((e = prepare_one<256, false, kClassStore, true>()) != cudaSuccess) return e;
+  if ((e = prepare_one<256, false, kClassRes, true>()) != cudaSuccess) return e;
+  if ((e = prepare_one<256, false, kClassQkv, true>()) != cudaSuccess) return e;
+  {
+    // how many pairs fit at once (SMs pair up within a GPC; some may be left over)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = TileCfg<256, false, kClassRes, true>::kSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, tc_gemm_kernel<256, false, kClassRes, true>, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = g_num_sms / 2;
+    }
+    g_max_pairs = n;
+  }
   return cudaSuccess;
 }
+
+int tc_gemm_max_pairs() { return g_max_pairs; }
+
+#ifdef WAM_GEMM_TIMELINE
+extern "C" int wam_debug_gemm_timeline(unsigned long long* host, int n) {
+  if (n > 1024) n = 1024;
+  const int r = cudaMemcpyFromSymbol(host, g_gemm_tl, sizeof(unsigned long long) * 10 * n) == cudaSuccess ? g_max_pairs : -1;
+  static unsigned long long zero[1024][10];
+  cudaMemcpyToSymbol(g_gemm_tl, zero, sizeof zero);
+  return r;
+}
+#endif
 
 cudaError_t set_peer_wait_test(int extra, unsigned long long limit_ns) {
   cudaError_t e = cudaMemcpyToSymbol(g_peer_wait_extra, &extra, sizeof extra);
@@ -1198,6 +1444,10 @@ cudaError_t launch_tc_gemm(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
       case 64: return launch_one<64, true, kClassNormB>(t, e, s);
     }
     return cudaErrorInvalidValue;
+  }
+  if (t.pair) {  // CTA pairs: normal orientation, 256-wide tiles
+    if (t.swap || t.bn != 256 || t.rows_b % 32 != 0) return cudaErrorInvalidValue;
+    return launch_normal<256, true>(t, e, s);
   }
   if (t.swap) {
     switch (t.bn) {

@@ -121,6 +121,8 @@ struct TcGemm {
   int splits;                // swapped: CTAs = tiles * splits (each tile's K split evenly)
   bool swap;
   int max_ctas;              // normal: persistent grid size (0: one CTA per SM)
+  bool pair;                 // normal, bn 256: CTA pairs share M = 256 MMAs (2-SM tensor-core tiles);
+                             // the B map's box is then bn / 2 rows (each CTA loads half)
   float* ws;                 // partial tiles: 2 * CTAs * 128 * bn floats (tc_gemm_ws_floats)
   int* tickets;              // two per output tile, zero on entry, left zero
   unsigned* status;
@@ -128,6 +130,10 @@ struct TcGemm {
 
 // Workspace floats the launch needs for K-split partial tiles.
 size_t tc_gemm_ws_floats(const TcGemm& g);
+// Ticket ints the launch needs (two per 128-row output tile).
+size_t tc_gemm_tickets(const TcGemm& g);
+// CTA pairs the device holds at once (0 before prepare_tc_gemm).
+int tc_gemm_max_pairs();
 // Partial tiles the last piece of a split tile can bring into its operand
 // ring at once (the fast reduction path); tiles split into more pieces are
 // summed from global memory instead.  Normal orientation: the smallest ring

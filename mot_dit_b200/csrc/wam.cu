@@ -62,6 +62,7 @@ struct Dims {
 
 struct GemmPlan {
   int bn = 128, splits = 1, max_ctas = 0;
+  bool pair = false;  // normal orientation, bn 256: CTA pairs (2-SM MMA)
 };
 
 }  // namespace
@@ -385,6 +386,7 @@ wam_status run_tc(wam_ctx* c, const CUtensorMap& A, const CUtensorMap& Bm, int r
   g.splits = p.splits;
   g.swap = swap;
   g.max_ctas = p.max_ctas;
+  g.pair = p.pair;
   g.ws = video ? c->ws_gemm_v : c->ws_gemm;
   g.tickets = video ? c->tk_gemm_v : c->tk_gemm;
   g.status = c->status;
@@ -1225,10 +1227,21 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     // WAM_VIDEO_SPLIT_FREE=0 turns the rule off (always vctas CTAs, stream-K).
     const char* sfv = getenv("WAM_VIDEO_SPLIT_FREE");
     const bool split_free = !(sfv && sfv[0] == '0');
-    auto grid = [&](int n_out, int bn) {
-      const int tiles = ((d.Mv + 127) / 128) * ((n_out + bn - 1) / bn);
-      const int k = (tiles + vctas - 1) / vctas;  // tiles per CTA
-      return (split_free && k <= 2 && tiles % k == 0) ? tiles / k : vctas;
+    // CTA pairs (2-SM MMA, M = 256 over two SMs; WAM_VIDEO_PAIR=1): each SM
+    // stages its own 128 token rows and half of the 256 weight rows of a
+    // tile, half the operand bytes per flop of a 1-SM 128 x 256 tile.  Off by
+    // default: the 1-SM 256-wide main loop already runs at the tensor-core
+    // rate (0.38 us per 64-deep k-block at 1088 tokens, both forms), and the
+    // pairs' longer split-tile tails made them slower (FFN-down 41 vs 30 us).
+    const char* pv = getenv("WAM_VIDEO_PAIR");
+    const bool pair = pv && pv[0] == '1' && d.dv % 256 == 0 && (3 * d.A) % 256 == 0 && d.Fv % 256 == 0;
+    auto grid = [&](int n_out, int bn, bool pr) {
+      const int unit_rows = pr ? 256 : 128, units = pr ? vctas / 2 : vctas;
+      const int tiles = ((d.Mv + unit_rows - 1) / unit_rows) * ((n_out + bn - 1) / bn);
+      const int k = (tiles + units - 1) / units;  // tiles per unit
+      // whole tiles per unit, unless that leaves a quarter of the units idle
+      const bool whole = split_free && k <= 2 && tiles % k == 0 && 4 * (tiles / k) >= 3 * units;
+      return (whole ? tiles / k : units) * (pr ? 2 : 1);
     };
     const int bn_res = ((d.Mv + 127) / 128) * (d.dv / 256) >= 2 * vctas ? 256 : 128;
     // WAM_VIDEO_OPROJ_BN / WAM_VIDEO_FFN2_BN (128 or 256) override the tile
@@ -1239,12 +1252,19 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
       return (n == 128 || n == 256) && d.dv % n == 0 ? n : dflt;
     };
     const int bn_o = bn_env("WAM_VIDEO_OPROJ_BN", bn_res), bn_f2 = bn_env("WAM_VIDEO_FFN2_BN", bn_res);
-    c->p_v_qkv = {256, 1, grid(3 * d.A, 256)};
-    c->p_v_o = {bn_o, 1, grid(d.dv, bn_o)};
-    c->p_v_f1 = {256, 1, grid(d.Fv, 256)};
-    c->p_v_f2 = {bn_f2, 1, grid(d.dv, bn_f2)};
-    c->p_v_in = {128, 1, grid(d.dv, 128)};
-    c->p_v_out = {64, 1, grid(d.Pv > 0 ? d.Pv : 64, 64)};
+    if (pair) {
+      c->p_v_qkv = {256, 1, grid(3 * d.A, 256, true), true};
+      c->p_v_o = {256, 1, grid(d.dv, 256, true), true};
+      c->p_v_f1 = {256, 1, grid(d.Fv, 256, true), true};
+      c->p_v_f2 = {256, 1, grid(d.dv, 256, true), true};
+    } else {
+      c->p_v_qkv = {256, 1, grid(3 * d.A, 256, false)};
+      c->p_v_o = {bn_o, 1, grid(d.dv, bn_o, false)};
+      c->p_v_f1 = {256, 1, grid(d.Fv, 256, false)};
+      c->p_v_f2 = {bn_f2, 1, grid(d.dv, bn_f2, false)};
+    }
+    c->p_v_in = {128, 1, grid(d.dv, 128, false)};
+    c->p_v_out = {64, 1, grid(d.Pv > 0 ? d.Pv : 64, 64, false)};
     const int bn_a = d.Ma <= 32 ? 32 : (d.Ma <= 64 ? 64 : (d.Ma <= 128 ? 128 : 256));
     // Opt-in (WAM_FUSE_NORM=1): every CTA of the fused GEMM re-reads all of
     // x_a for the row norms, and on the config-2/3 chunks that measured slower
@@ -1281,8 +1301,9 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
       g.splits = p.splits;
       g.swap = swap;
       g.max_ctas = p.max_ctas;
+      g.pair = p.pair;
       *w = std::max(*w, tc_gemm_ws_floats(g));
-      *t = std::max(*t, ((rows_a + 127) / 128) * ((rows_b + p.bn - 1) / p.bn));
+      *t = std::max(*t, (int)(tc_gemm_tickets(g) / 2));
     };
     need(c->p_a_in, d.da, d.Ma, d.Kin, true, &ws, &tiles);
     need(c->p_a_qkv, 3 * d.A, d.Ma, d.da + d.r, true, &ws, &tiles);
@@ -1321,7 +1342,9 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     auto amap = [&](CUtensorMap* m, const void* p, int rows, int K, int box) {
       ok = ok && make_tmap_3d(m, p, K, rows, 1, 0, box);
     };
-    const int bnv_qkv = c->p_v_qkv.bn, bnv_o = c->p_v_o.bn, bnv_f1 = c->p_v_f1.bn, bnv_f2 = c->p_v_f2.bn;
+    // weight boxes: the tile's rows, or half of them for CTA pairs
+    auto wbox = [](const GemmPlan& p) { return p.pair ? p.bn / 2 : p.bn; };
+    const int bnv_qkv = wbox(c->p_v_qkv), bnv_o = wbox(c->p_v_o), bnv_f1 = wbox(c->p_v_f1), bnv_f2 = wbox(c->p_v_f2);
     const int bna = c->p_a_qkv.bn;
     amap(&c->m_hv, c->h_v, d.Mv, d.dv, 128);
     amap(&c->m_ov, c->o_v, d.Mv, d.A, 128);
@@ -1908,36 +1931,39 @@ int wam_chunk_kernel_count(wam_ctx* c, int S) {
 }
 
 // ------------------------------------------------- single-op entry points --
-wam_status wam_op_linear(int dtype, const void* x, const void* w, const float* bias, float* out, int M, int N, int K,
-                         int swap, int splits, void* stream) {
-  if (!x || !w || !bias || !out || M < 1 || N < 1 || K < 1) return WAM_ERR_INVALID_ARG;
-  cudaStream_t s = (cudaStream_t)stream;
-  EpiArgs e;
-  e.kind = kEpiStoreF32;
-  e.bias = bias;
-  e.out_f32 = out;
-  e.ld_out = N;
-  if (dtype == WAM_FP32) return launch_f32_gemm((const float*)x, K, (const float*)w, M, N, K, e, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
-  if (dtype != WAM_BF16 || K % 64) return WAM_ERR_INVALID_ARG;
-  const int bn = swap ? (M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256) : 128;
+namespace {
+// One GEMM with bias into fp32 out[M, N] through the tcgen05 kernel (private
+// workspace grown on demand).  Normal orientation: bn 128 or 256, `ctas`
+// persistent CTAs (0: all SMs), pair = CTA pairs; swapped: `ctas` = CTAs per
+// output tile.
+wam_status op_linear_bf16(const void* x, const void* w, const float* bias, float* out, int M, int N, int K, bool swap,
+                          int ctas, int bn_normal, bool pair, cudaStream_t s) {
+  if (K % 64) return WAM_ERR_INVALID_ARG;
+  const int bn = swap ? (M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256) : bn_normal;
   if (swap && M > 256) return WAM_ERR_INVALID_ARG;
-  if (!swap && N % 32) return WAM_ERR_INVALID_ARG;
+  if (!swap && (N % 32 || (bn != 128 && bn != 256) || (pair && bn != 256))) return WAM_ERR_INVALID_ARG;
   static thread_local unsigned* status = nullptr;
   if (!status) {
     if (prepare_tc_gemm() != cudaSuccess) return WAM_ERR_CUDA;
     if (cudaMalloc(&status, 4) != cudaSuccess) return WAM_ERR_OOM;
     cudaMemset(status, 0, 4);
   }
+  EpiArgs e;
+  e.kind = kEpiStoreF32;
+  e.bias = bias;
+  e.out_f32 = out;
+  e.ld_out = N;
   TcGemm g{};
   g.rows_a = swap ? N : M;
   g.rows_b = swap ? M : N;
   g.K = K;
   g.z_a = g.z_b = 0;
   g.bn = bn;
-  g.splits = swap ? std::max(1, splits) : 1;
-  g.swap = swap != 0;
-  g.max_ctas = swap ? 0 : std::max(0, splits);  // normal orientation: `splits` = persistent CTAs (0: all SMs)
-  const int tiles = 2 * ((g.rows_a + 127) / 128) * ((g.rows_b + bn - 1) / bn);  // two tickets per tile
+  g.splits = swap ? std::max(1, ctas) : 1;
+  g.swap = swap;
+  g.max_ctas = swap ? 0 : std::max(0, ctas);
+  g.pair = pair;
+  const size_t tickets = tc_gemm_tickets(g);
   static thread_local float* ws = nullptr;
   static thread_local int* tk = nullptr;
   static thread_local size_t ws_cap = 0, tk_cap = 0;
@@ -1949,16 +1975,17 @@ wam_status wam_op_linear(int dtype, const void* x, const void* w, const float* b
     if (cudaMalloc(&ws, need * 4) != cudaSuccess) return WAM_ERR_OOM;
     ws_cap = need;
   }
-  if ((size_t)tiles > tk_cap) {
+  if (tickets > tk_cap) {
     if (tk) cudaFree(tk);
     tk = nullptr;
     tk_cap = 0;
-    if (cudaMalloc(&tk, tiles * 4) != cudaSuccess) return WAM_ERR_OOM;
-    if (cudaMemset(tk, 0, tiles * 4) != cudaSuccess) return WAM_ERR_CUDA;
-    tk_cap = tiles;
+    if (cudaMalloc(&tk, tickets * 4) != cudaSuccess) return WAM_ERR_OOM;
+    if (cudaMemset(tk, 0, tickets * 4) != cudaSuccess) return WAM_ERR_CUDA;
+    tk_cap = tickets;
   }
   CUtensorMap mx, mw, mo;
-  if (!make_tmap_3d(&mx, x, K, M, 1, 0, swap ? bn : 128) || !make_tmap_3d(&mw, w, K, N, 1, 0, swap ? 128 : bn))
+  const int wbox = swap ? 128 : (pair ? bn / 2 : bn);
+  if (!make_tmap_3d(&mx, x, K, M, 1, 0, swap ? bn : 128) || !make_tmap_3d(&mw, w, K, N, 1, 0, wbox))
     return WAM_ERR_INVALID_ARG;
   if (!swap) {
     if (!make_tmap_sw128(&mo, out, 4, N, M, 1, 0, 32, 32)) return WAM_ERR_INVALID_ARG;
@@ -1970,6 +1997,29 @@ wam_status wam_op_linear(int dtype, const void* x, const void* w, const float* b
   g.tickets = tk;
   g.status = status;
   return launch_tc_gemm(g, e, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
+}
+}  // namespace
+
+wam_status wam_op_linear(int dtype, const void* x, const void* w, const float* bias, float* out, int M, int N, int K,
+                         int swap, int splits, void* stream) {
+  if (!x || !w || !bias || !out || M < 1 || N < 1 || K < 1) return WAM_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (dtype == WAM_FP32) {
+    EpiArgs e;
+    e.kind = kEpiStoreF32;
+    e.bias = bias;
+    e.out_f32 = out;
+    e.ld_out = N;
+    return launch_f32_gemm((const float*)x, K, (const float*)w, M, N, K, e, s) == cudaSuccess ? WAM_OK : WAM_ERR_CUDA;
+  }
+  if (dtype != WAM_BF16) return WAM_ERR_INVALID_ARG;
+  return op_linear_bf16(x, w, bias, out, M, N, K, swap != 0, splits, 128, false, s);
+}
+
+wam_status wam_op_linear_tiled(const void* x, const void* w, const float* bias, float* out, int M, int N, int K, int bn,
+                               int pair, int ctas, void* stream) {
+  if (!x || !w || !bias || !out || M < 1 || N < 1 || K < 1 || ctas < 0) return WAM_ERR_INVALID_ARG;
+  return op_linear_bf16(x, w, bias, out, M, N, K, false, ctas, bn, pair != 0, (cudaStream_t)stream);
 }
 
 wam_status wam_op_norm_mod(int dtype, const float* x, void* h, int M, int d, const float* scale, const float* shift,

@@ -72,6 +72,23 @@ def test_fused_action_norm(monkeypatch, batch):
     wam.close()
 
 
+@pytest.mark.parametrize("batch", [1, 2])
+def test_video_cta_pairs(monkeypatch, batch):
+    """Opt-in CTA-pair video GEMMs (WAM_VIDEO_PAIR=1: 2-SM MMAs, M = 256 over
+    two SMs): parity with the oracle, CEWP == sequential and graph == eager
+    bitwise."""
+    monkeypatch.setenv("WAM_VIDEO_PAIR", "1")
+    c = _mid().replace(batch=batch)
+    wam = W.Wam(c, seed=17)
+    inp = inputs(c, 17)
+    a0 = run_chunk(wam, inp, S=2, mode=W.CEWP, use_graph=True)
+    for mode, graph in ((W.SEQUENTIAL, True), (W.CEWP, False)):
+        assert np.array_equal(a0, run_chunk(wam, inp, S=2, mode=mode, use_graph=graph))
+    ref_a0, ref_veff = oracle_chunk(c, 17, inp, S=2)
+    check_parity(a0, inp, ref_a0, ref_veff, c.dtype)
+    wam.close()
+
+
 def test_mid_bf16_parity_and_kv_publish():
     c = _mid()
     wam = W.Wam(c, seed=11)
