@@ -227,6 +227,63 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ------------------------------------------------- norm + modulation -------
+// One row, one warp: h = rms(x) * (gain ? gain[n] : 1 + scale[n]) + (shift ?
+// shift[n] : 0), rms(x) = x / sqrt(mean(x^2) + 1e-6).  A lane holds up to
+// kRowNormV float4 of the row in registers so every load of the row is in
+// flight at once (d a multiple of 4, d <= 32 * 4 * kRowNormV).  Every place
+// that normalises a row calls this, so all of them round alike.
+constexpr int kRowNormV = 12;
+
+template <bool BF16>
+__device__ __forceinline__ void norm_mod_row(const float* __restrict__ x, void* __restrict__ h, int d,
+                                             const float* __restrict__ scale, const float* __restrict__ shift,
+                                             const float* __restrict__ gain, int lane) {
+  const float4* xr = reinterpret_cast<const float4*>(x);
+  const int n4 = d >> 2;
+  float4 v[kRowNormV];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < kRowNormV; ++k) {
+    const int i = lane + 32 * k;
+    v[k] = i < n4 ? xr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int k = 0; k < kRowNormV; ++k) ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float r = 1.0f / sqrtf(ss / (float)d + 1e-6f);
+#pragma unroll
+  for (int k = 0; k < kRowNormV; ++k) {
+    const int i = lane + 32 * k;
+    if (i >= n4) break;
+    float y[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+    float4 mul4, add4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (gain) {
+      mul4 = __ldg(reinterpret_cast<const float4*>(gain) + i);
+    } else {
+      mul4 = __ldg(reinterpret_cast<const float4*>(scale) + i);
+      mul4.x += 1.f;
+      mul4.y += 1.f;
+      mul4.z += 1.f;
+      mul4.w += 1.f;
+    }
+    if (shift) add4 = __ldg(reinterpret_cast<const float4*>(shift) + i);
+    y[0] = y[0] * r * mul4.x + add4.x;
+    y[1] = y[1] * r * mul4.y + add4.y;
+    y[2] = y[2] * r * mul4.z + add4.z;
+    y[3] = y[3] * r * mul4.w + add4.w;
+    if (BF16) {
+      uint2 p;
+      p.x = pack_bf16(y[0], y[1]);
+      p.y = pack_bf16(y[2], y[3]);
+      reinterpret_cast<uint2*>(h)[i] = p;
+    } else {
+      reinterpret_cast<float4*>(h)[i] = make_float4(y[0], y[1], y[2], y[3]);
+    }
+  }
+}
+
 // GELU, tanh form: 0.5 x (1 + tanh(z)), z = sqrt(2/pi) (x + 0.044715 x^3),
 // evaluated through the identity 0.5 (1 + tanh(z)) = 1 / (1 + exp(-2 z)).
 __device__ __forceinline__ float gelu_tanh(float x) {

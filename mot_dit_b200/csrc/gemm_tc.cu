@@ -45,6 +45,7 @@
 #include "kernels.h"
 
 namespace wam {
+static_assert(kRowNormMax == 32 * 4 * kRowNormV, "norm row width limit");
 namespace {
 
 constexpr int BM = 128;
@@ -214,7 +215,7 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t addr) {
 #ifdef WAM_GEMM_TIMELINE
 // Diagnostic build only: per CTA of the last launch, %smid and %globaltimer
 // at start, first MMA issue (rank 0 / single CTA), last MMA issue and end.
-__device__ unsigned long long g_gemm_tl[1024][10];
+__device__ unsigned long long g_gemm_tl[1024][16];
 #define WAM_TL(slot, v) \
   if (blockIdx.x < 1024) g_gemm_tl[blockIdx.x][slot] = (v)
 #else
@@ -554,6 +555,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // with the fused norm the producer reads weights only: no wait for the previous kernel
         if (!C::kNB) pdl_wait();
+        if (!SWAP && e.na_x) {
+          // the A operand is written by this launch (norm prologue): every row done
+          if (!wait_count(e.na_cnt + 1, g.rows_a, g.status, abort_flag)) *abort_flag = 1;
+          __threadfence();
+          fence_proxy_async_global();  // (the loads are issued either way, so every stage completes)
+        }
         for (int i = 0; i < pre && !C::kNB; ++i) {
           if (SWAP)
             load(&map_b, sB + i * C::kBBytes, i, sg.kb0 + i, brow(tb), g.z_b);
@@ -657,6 +664,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     pdl_wait();  // outputs / residual rows belong to the previous kernel until it is done
+    if (!SWAP && e.na_x) {
+      // Norm prologue: token rows of the A operand, one per warp at a time,
+      // from the launch's shared row counter (no CTA waits for another to
+      // start: the running CTAs take every row between them).
+      int n = 0;
+      while (true) {
+        int r = 0;
+        if (lane == 0) r = atomicAdd(e.na_cnt, 1);
+        r = __shfl_sync(0xffffffffu, r, 0);
+        if (r >= g.rows_a) break;
+        norm_mod_row<true>(e.na_x + (size_t)r * g.K, reinterpret_cast<__nv_bfloat16*>(e.na_h) + (size_t)r * g.K, g.K,
+                           e.na_scale, e.na_shift, nullptr, lane);
+        ++n;
+      }
+      if (n > 0) {
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(e.na_cnt + 1, n);
+      }
+    }
     const int quad = warp & 3;
     const int row = quad * 32 + lane;  // TMEM lane = tile row
     const EpiRegs R = hoist(e);
@@ -855,12 +882,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           float* my = g.ws + ((size_t)blockIdx.x * 2 + (first_seg ? 0 : 1)) * (BM * BN);
           for (int c = 0; c < BN; c += 32) {
             float v[32];
+            if (threadIdx.x == 64 && c < 64 && x == x_end) WAM_TL(10 + 3 * (c >> 5), globaltimer());
             tmem_ld32(t_row + c, v);
+            if (threadIdx.x == 64 && c < 64 && x == x_end) WAM_TL(11 + 3 * (c >> 5), globaltimer());
             if (c + 32 >= BN) release();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               __stcg(reinterpret_cast<float4*>(my + ((size_t)((c >> 5) * 8 + j) * BM + row) * 4),
                      make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+            if (threadIdx.x == 64 && c < 64 && x == x_end) WAM_TL(12 + 3 * (c >> 5), globaltimer());
           }
           __threadfence();
           epi_bar();
@@ -1226,6 +1256,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_dealloc(tmem, C::kTmemCols);
   }
   if (threadIdx.x == 0) WAM_TL(4, globaltimer());
+  if (!SWAP && e.na_x && threadIdx.x == 0) {
+    // every CTA is past its rows and its wait once all have counted out here
+    __threadfence();
+    if (atomicAdd(e.na_cnt + 2, 1) == (int)gridDim.x - 1) {
+      e.na_cnt[0] = 0;
+      e.na_cnt[1] = 0;
+      e.na_cnt[2] = 0;
+      __threadfence();
+    }
+  }
 }
 
 template <int BN, bool SWAP, int EPI, bool PAIR = false>
@@ -1420,8 +1460,8 @@ int tc_gemm_max_pairs() { return g_max_pairs; }
 #ifdef WAM_GEMM_TIMELINE
 extern "C" int wam_debug_gemm_timeline(unsigned long long* host, int n) {
   if (n > 1024) n = 1024;
-  const int r = cudaMemcpyFromSymbol(host, g_gemm_tl, sizeof(unsigned long long) * 10 * n) == cudaSuccess ? g_max_pairs : -1;
-  static unsigned long long zero[1024][10];
+  const int r = cudaMemcpyFromSymbol(host, g_gemm_tl, sizeof(unsigned long long) * 16 * n) == cudaSuccess ? g_max_pairs : -1;
+  static unsigned long long zero[1024][16];
   cudaMemcpyToSymbol(g_gemm_tl, zero, sizeof zero);
   return r;
 }
@@ -1436,6 +1476,9 @@ cudaError_t set_peer_wait_test(int extra, unsigned long long limit_ns) {
 cudaError_t launch_tc_gemm(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
   if (g_num_sms == 0) return cudaErrorNotReady;
   if (!t.ws || !t.tickets) return cudaErrorInvalidValue;
+  // norm prologue: normal orientation, rows of at most 32 * 4 * kRowNormV values
+  if (e.na_x && (t.swap || !e.na_h || !e.na_cnt || !e.na_scale || t.K % 4 || t.K > 32 * 4 * kRowNormV))
+    return cudaErrorInvalidValue;
   if (e.nb_x) {  // fused norm of the token rows: swapped, one token tile, K <= kNormKMax
     if (!t.swap || t.rows_b > t.bn || t.K > kNormKMax || t.K % BK)
       return cudaErrorInvalidValue;

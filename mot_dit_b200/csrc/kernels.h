@@ -30,6 +30,9 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Widest row the RMSNorm / modulation kernels and the GEMM norm prologue take.
+constexpr int kRowNormMax = 1536;
+
 constexpr int kMaxSteps = 64;  // Euler steps per chunk held in the device schedule
 
 // Per-call inputs read by the first/last kernels of a chunk.  They live in
@@ -107,6 +110,18 @@ struct EpiArgs {
   const float* nb_scale = nullptr;
   const float* nb_shift = nullptr;
   const float* nb_gain = nullptr;
+  // Normal orientation only: the launch first writes its own A operand,
+  // na_h[r] = rms(na_x[r]) * (1 + na_scale) + na_shift as bf16 for every
+  // token row r (fp32 rows, ld = K; na_h is the memory map_a reads).  Rows
+  // are taken one at a time from na_cnt[0] by whichever CTAs run, counted
+  // done in na_cnt[1]; A tiles are loaded once all rows are done; the last
+  // CTA out (na_cnt[2]) sets the three counters back to zero.  The counters
+  // are private to one stream's launches.
+  const float* na_x = nullptr;
+  const float* na_scale = nullptr;
+  const float* na_shift = nullptr;
+  void* na_h = nullptr;
+  int* na_cnt = nullptr;
 };
 
 // C[m, n] = sum_k X[m, k] W[n, k] (+ epilogue), bf16 operands via TMA into

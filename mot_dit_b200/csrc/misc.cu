@@ -17,12 +17,7 @@ namespace {
 constexpr int kNormWarps = 16;  // rows per CTA (config-2 chunk 4.09 -> 4.02 ms against 8)
 
 // ------------------------------------------------- norm + modulation -------
-// h = rms(x) * (gain ? gain[n] : 1 + scale[n]) + (shift ? shift[n] : 0);
-// rms(x) = x / sqrt(mean(x^2) + 1e-6).  One warp per row; a lane holds up to
-// kNormV float4 of the row in registers so every load of the row is in flight
-// at once (d <= 32 * 4 * kNormV).
-constexpr int kNormV = 12;
-
+// One warp per row (norm_mod_row, shared with the fused-norm GEMM prologue).
 template <bool BF16>
 __global__ void __launch_bounds__(32 * kNormWarps)
     norm_mod_kernel(const float* __restrict__ x, void* __restrict__ h, int M, int d, const float* __restrict__ scale,
@@ -30,51 +25,10 @@ __global__ void __launch_bounds__(32 * kNormWarps)
   pdl_trigger();
   pdl_wait();
   const int row = blockIdx.x * kNormWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
   if (row >= M) return;
-  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * d);
-  const int n4 = d >> 2;
-  float4 v[kNormV];
-  float ss = 0.f;
-#pragma unroll
-  for (int k = 0; k < kNormV; ++k) {
-    const int i = lane + 32 * k;
-    v[k] = i < n4 ? xr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-#pragma unroll
-  for (int k = 0; k < kNormV; ++k) ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float r = 1.0f / sqrtf(ss / (float)d + 1e-6f);
-#pragma unroll
-  for (int k = 0; k < kNormV; ++k) {
-    const int i = lane + 32 * k;
-    if (i >= n4) break;
-    float y[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-    float4 mul4, add4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (gain) {
-      mul4 = __ldg(reinterpret_cast<const float4*>(gain) + i);
-    } else {
-      mul4 = __ldg(reinterpret_cast<const float4*>(scale) + i);
-      mul4.x += 1.f;
-      mul4.y += 1.f;
-      mul4.z += 1.f;
-      mul4.w += 1.f;
-    }
-    if (shift) add4 = __ldg(reinterpret_cast<const float4*>(shift) + i);
-    y[0] = y[0] * r * mul4.x + add4.x;
-    y[1] = y[1] * r * mul4.y + add4.y;
-    y[2] = y[2] * r * mul4.z + add4.z;
-    y[3] = y[3] * r * mul4.w + add4.w;
-    if (BF16) {
-      uint2 p;
-      p.x = pack_bf16(y[0], y[1]);
-      p.y = pack_bf16(y[2], y[3]);
-      reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(h) + (size_t)row * ldh)[i] = p;
-    } else {
-      reinterpret_cast<float4*>(reinterpret_cast<float*>(h) + (size_t)row * ldh)[i] = make_float4(y[0], y[1], y[2], y[3]);
-    }
-  }
+  norm_mod_row<BF16>(x + (size_t)row * d, BF16 ? (void*)(reinterpret_cast<__nv_bfloat16*>(h) + (size_t)row * ldh)
+                                                : (void*)(reinterpret_cast<float*>(h) + (size_t)row * ldh),
+                     d, scale, shift, gain, threadIdx.x & 31);
 }
 
 // ------------------------------------------------ timestep conditioning ----
@@ -310,7 +264,7 @@ cudaError_t launch_norm_mod(const float* x, void* h, bool h_bf16, int M, int d, 
                             const float* shift, const float* gain, cudaStream_t s, int ldh) {
   if (ldh == 0) ldh = d;
   if (ldh < d || ldh % 4) return cudaErrorInvalidValue;
-  if (d % 4 != 0 || d > 32 * 4 * kNormV) return cudaErrorInvalidValue;
+  if (d % 4 != 0 || d > 32 * 4 * kRowNormV) return cudaErrorInvalidValue;
   dim3 grid((M + kNormWarps - 1) / kNormWarps);
   if (h_bf16)
     return launch_k(norm_mod_kernel<true>, grid, dim3(32 * kNormWarps), 0, s, x, h, M, d, scale, shift, gain, ldh);

@@ -92,6 +92,8 @@ struct wam_ctx {
   float* ws_gemm_v = nullptr;  // video-stream GEMM partial tiles / tickets (the streams overlap)
   int* tk_gemm_v = nullptr;
   size_t tk_gemm_bytes = 0, tk_gemm_v_bytes = 0;
+  int* na_cnt = nullptr;     // video norm prologue row counters (taken, done, CTAs out)
+  bool fuse_norm_v = false;  // the video QKV / FFN-up GEMMs normalise their own A rows
   float* ws_attn = nullptr;
   int* tk_attn = nullptr;
   unsigned* status = nullptr;
@@ -595,11 +597,25 @@ wam_status enqueue_video_blocks(wam_ctx* c, cudaStream_t s, cudaEvent_t* ev_read
   for (int i = 0; i < d.N; ++i) {
     const float* mod = c->mod_v + (size_t)i * 6 * d.dv;
     if (war_waits) CK(cudaStreamWaitEvent(s, c->ev_used[i], 0));
-    c->cur_cls = WAM_PROF_VIDEO_NORM;
-    RET(norm(c, c->x_v, c->h_v, d.Mv, d.dv, mod + d.dv, mod, nullptr, s));
+    // the A operand h_v = norm(x_v) with the block's modulation: in the GEMM's
+    // own prologue (fused), or by the norm kernel
+    auto norm_a = [&](EpiArgs& e, const float* scale, const float* shift) -> wam_status {
+      if (c->fuse_norm_v) {
+        e.na_x = c->x_v;
+        e.na_scale = scale;
+        e.na_shift = shift;
+        e.na_h = c->h_v;
+        e.na_cnt = c->na_cnt;
+        return WAM_OK;
+      }
+      c->cur_cls = WAM_PROF_VIDEO_NORM;
+      return norm(c, c->x_v, c->h_v, d.Mv, d.dv, scale, shift, nullptr, s);
+    };
+    EpiArgs eq = epi_qkv(c, true, i);
+    RET(norm_a(eq, mod + d.dv, mod));
     c->cur_cls = WAM_PROF_VIDEO_QKV;
     Lin Lq{&c->m_w_qkv_v, &c->m_hv, matp(c, blk(x, i, kQkvW)), c->h_v, 3 * d.A, d.dv, i, &c->p_v_qkv};
-    RET(linear(c, true, Lq, d.Mv, epi_qkv(c, true, i), c->qkv_tmp_v, s));
+    RET(linear(c, true, Lq, d.Mv, eq, c->qkv_tmp_v, s));
     // (the trace mark first: an action-side mark after the wait on e_i then
     // depends on it, so the recorded order is the schedule's)
     trace_mark(c, s, WAM_TRACE_VIDEO_KV, i);
@@ -612,11 +628,11 @@ wam_status enqueue_video_blocks(wam_ctx* c, cudaStream_t s, cudaEvent_t* ev_read
     eo.gate = mod + 2 * d.dv;
     Lin Lo{&c->m_w_o_v, &c->m_ov, matp(c, blk(x, i, kOW)), c->o_v, d.dv, d.A, i, &c->p_v_o};
     RET(linear(c, true, Lo, d.Mv, eo, nullptr, s));
-    c->cur_cls = WAM_PROF_VIDEO_NORM;
-    RET(norm(c, c->x_v, c->h_v, d.Mv, d.dv, mod + 4 * d.dv, mod + 3 * d.dv, nullptr, s));
+    EpiArgs e1 = epi_base(kEpiGelu, vecp(c, blk(x, i, kF1B)), nullptr, c->f_v, d.Fv);
+    RET(norm_a(e1, mod + 4 * d.dv, mod + 3 * d.dv));
     c->cur_cls = WAM_PROF_VIDEO_FFN_UP;
     Lin L1{&c->m_w_f1_v, &c->m_hv, matp(c, blk(x, i, kF1W)), c->h_v, d.Fv, d.dv, i, &c->p_v_f1};
-    RET(linear(c, true, L1, d.Mv, epi_base(kEpiGelu, vecp(c, blk(x, i, kF1B)), nullptr, c->f_v, d.Fv), nullptr, s));
+    RET(linear(c, true, L1, d.Mv, e1, nullptr, s));
     c->cur_cls = WAM_PROF_VIDEO_FFN_DOWN;
     EpiArgs e2 = epi_base(kEpiGateRes, vecp(c, blk(x, i, kF2B)), c->x_v, nullptr, d.dv);
     e2.gate = mod + 5 * d.dv;
@@ -1272,6 +1288,15 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     const char* fv = getenv("WAM_FUSE_NORM");
     c->fuse_norm_a = fv && fv[0] == '1' && bn_a <= 64 && d.da <= 1024 && d.da % 64 == 0 && d.r == 0;
     const bool fn = c->fuse_norm_a;
+    // Opt-in (WAM_VIDEO_FUSED_NORM=1): the video QKV / FFN-up GEMMs compute
+    // their A operand (the block's RMSNorm + AdaLN modulation of x_v) in their
+    // own prologue instead of a separate norm launch.  Off by default: in the
+    // captured chunk the norm kernel starts early (dependent launch) and costs
+    // ~2-3 us on the critical path, while the prologue runs the 1088 rows on
+    // only four warps per CTA before the first MMA (config-2 chunk 4.77 ms
+    // fused against 4.12 ms).
+    const char* fvv = getenv("WAM_VIDEO_FUSED_NORM");
+    c->fuse_norm_v = fvv && fvv[0] == '1' && d.dv % 4 == 0 && d.dv <= kRowNormMax;
     // CTAs per action GEMM (tiles x splits, about): the weight stream spread
     // over this many SMs; WAM_ACTION_CTAS overrides.
     int actas = nsm;
@@ -1330,6 +1355,7 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   c->tk_gemm_bytes = (size_t)tiles * 2 * 4;
   RET(dalloc(c, &c->ws_gemm_v, ws_v * 4));
   RET(dalloc(c, &c->tk_gemm_v, (size_t)tiles_v * 2 * 4));
+  RET(dalloc(c, &c->na_cnt, 3 * 4));
   c->tk_gemm_v_bytes = (size_t)tiles_v * 2 * 4;
   RET(dalloc(c, &c->ws_attn, attention_ws_floats(d.B, d.H, d.Dh, d.La, c->attn_splits) * 4));
   RET(dalloc(c, &c->tk_attn, (size_t)d.B * d.H * 4));
@@ -1898,6 +1924,7 @@ wam_status wam_check_device_status(wam_ctx* c) {
     CK(cudaMemset(c->status, 0, 4));
     if (c->tk_gemm) CK(cudaMemset(c->tk_gemm, 0, c->tk_gemm_bytes));
     if (c->tk_gemm_v) CK(cudaMemset(c->tk_gemm_v, 0, c->tk_gemm_v_bytes));
+    if (c->na_cnt) CK(cudaMemset(c->na_cnt, 0, 3 * 4));
     if (c->ab_cnt) CK(cudaMemset(c->ab_cnt, 0, (size_t)action_block_cnt_ints() * 4));
     if (c->ab_cnt_attn) CK(cudaMemset(c->ab_cnt_attn, 0, (size_t)c->d.B * c->d.H * 4));
     if (c->tk_attn) CK(cudaMemset(c->tk_attn, 0, (size_t)c->d.B * c->d.H * 4));

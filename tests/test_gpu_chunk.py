@@ -89,6 +89,32 @@ def test_video_cta_pairs(monkeypatch, batch):
     wam.close()
 
 
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_video_fused_norm(monkeypatch, pair):
+    """Opt-in fused video norm (WAM_VIDEO_FUSED_NORM=1): the QKV / FFN-up
+    GEMMs write their own A operand from x_v in a prologue (the rows shared out
+    through a counter).  It rounds like the norm kernel, so the chunk is
+    bitwise the unfused one; CEWP == sequential, graph == eager, and fifty
+    replays (the counters reset themselves every launch)."""
+    monkeypatch.setenv("WAM_VIDEO_PAIR", pair)
+    c = _mid().replace(batch=2)
+    inp = inputs(c, 19)
+    monkeypatch.setenv("WAM_VIDEO_FUSED_NORM", "0")
+    wam = W.Wam(c, seed=19)
+    ref = run_chunk(wam, inp, S=2)
+    wam.close()
+    monkeypatch.setenv("WAM_VIDEO_FUSED_NORM", "1")
+    wam = W.Wam(c, seed=19)
+    got = run_chunk(wam, inp, S=2, mode=W.CEWP, use_graph=True)
+    assert np.array_equal(got, ref)
+    for mode, graph in ((W.SEQUENTIAL, True), (W.CEWP, False)):
+        assert np.array_equal(run_chunk(wam, inp, S=2, mode=mode, use_graph=graph), ref)
+    for _ in range(50):
+        assert np.array_equal(run_chunk(wam, inp, S=2), ref)
+    wam.check_device_status()
+    wam.close()
+
+
 def test_mid_bf16_parity_and_kv_publish():
     c = _mid()
     wam = W.Wam(c, seed=11)
