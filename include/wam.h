@@ -327,6 +327,21 @@ wam_status wam_op_linear_tiled(const void* dev_x, const void* dev_w, const float
 wam_status wam_op_attention(int dtype, const void* dev_q, const void* dev_k, const void* dev_v, void* dev_out,
                             int B, int H, int Dh, int Lq, int Lk, int Lcache, int splits, void* stream);
 
+/* The joint action attention of the chunk path: out[B*Lq, H*64] (bf16) =
+ * softmax(q k^T / 8) v per (sample, head) over cache rows [0, Lk), the
+ * action queries against the concatenated [K^v_i; K^a_i] (RealtimeWAM
+ * summary page, 前置知识 "Mixture-of-Transformers" / "KV 缓存").  q bf16
+ * [B, H, Lq, 64] with Lq <= 64; k / v bf16 [B, H, Lcache, 64].  The keys of
+ * each (sample, head) are split over `splits` CTAs of a cluster (1, 2, 4 or
+ * 8 with splits * Lq <= 279; 0 chooses from the SM count) whose partials
+ * are merged in split order,
+ * so the result does not depend on timing.  Cache rows below `ready` are
+ * read before the kernel waits for the previous kernel on the stream, so they
+ * must be complete when the call is enqueued (0: no such assumption).
+ * WAM_ERR_INVALID_ARG for other shapes; enqueued on `stream`. */
+wam_status wam_op_attention_joint(const void* dev_q, const void* dev_k, const void* dev_v, void* dev_out, int B, int H,
+                                  int Lq, int Lk, int Lcache, int ready, int splits, void* stream);
+
 /* h[M, d] = rms(x) * (dev_gain ? gain : 1 + scale) + (dev_shift ? shift : 0)
  * per row, rms(x) = x / sqrt(mean(x^2) + 1e-6): the RMSNorm / AdaLN
  * modulation prologue of every block (and, with a gain, the final norm).

@@ -23,6 +23,7 @@ from ._binding import (  # noqa: F401
     op_attention_noalloc,
     op_linear,
     op_linear_tiled,
+    op_attention_joint,
     op_norm_mod,
     patchify,
     preset,

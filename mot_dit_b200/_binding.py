@@ -85,6 +85,8 @@ def lib():
         "wam_last_error": (C.c_char_p, [_P]),
         "wam_op_linear": (C.c_int, [C.c_int, _P, _P, _P, _P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _P]),
         "wam_op_linear_tiled": (C.c_int, [_P, _P, _P, _P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _P]),
+        "wam_op_attention_joint": (C.c_int, [_P, _P, _P, _P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                            C.c_int, _P]),
         "wam_op_attention": (C.c_int, [C.c_int, _P, _P, _P, _P] + [C.c_int] * 7 + [_P]),
         "wam_op_attention_noalloc": (C.c_int, [_P, _P, _P, _P] + [C.c_int] * 6 + [_P]),
         "wam_op_norm_mod": (C.c_int, [C.c_int, _P, _P, C.c_int, C.c_int, _P, _P, _P, _P]),
@@ -325,6 +327,13 @@ def op_linear_tiled(x, w, bias, out, M, N, K, bn=256, pair=True, ctas=0, stream=
                                    _stream(stream))
     if st:
         raise WamError(st, "wam_op_linear_tiled")
+
+
+def op_attention_joint(q, k, v, out, B, H, Lq, Lk, Lcache, ready=0, splits=0, stream=None):
+    st = lib().wam_op_attention_joint(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Lq, Lk, Lcache, ready, splits,
+                                      _stream(stream))
+    if st:
+        raise WamError(st, "wam_op_attention_joint")
 
 
 def op_norm_mod(dtype, x, h, M, d, scale=None, shift=None, gain=None, stream=None):

@@ -31,6 +31,7 @@ constexpr int kTK = 64;     // keys per tile
 constexpr int kAttnThreads = 128;
 constexpr int kMaxSplits = 32;  // key splits of the action attention
 constexpr int kCombineBytes = 96 * 1024;  // dynamic shared memory for staging partial O rows
+constexpr int kJMaxSplits = 8;  // joint action attention: CTAs per cluster (key splits)
 
 // Row-major [64][64] bf16 tile, 16-byte chunks XOR-swizzled by row.
 __device__ __forceinline__ uint32_t tile_off(int row, int chunk) {
@@ -336,6 +337,280 @@ __global__ void attn_f32_kernel(const float* __restrict__ q, const float* __rest
   }
 }
 
+// ------------------------------------------------ joint action attention --
+// The action queries of one (sample, head) against the joint key list, split
+// over the `splits` CTAs of a cluster (rank = split): each takes keys
+// [split * kps, (split + 1) * kps) in 64-key tiles, brought in by TMA into a
+// kJStages-deep mbarrier ring.  Tiles of cache rows below `ready` (rows the
+// caller guarantees complete at launch) are requested before the
+// dependent-launch wait, while the previous kernel still runs; the chunk
+// passes 0 (a captured cross-stream event edge is programmatic too, so the
+// video rows are complete only after the wait).  Flash loop as above
+// (mma.sync, online softmax in fp32); each CTA then stores its unnormalised
+// partial (O, row max, row sum) into rank 0's shared memory through the
+// cluster's shared window, and rank 0 merges them in split order, so the
+// result does not depend on timing.
+constexpr int kJStages = 4;
+constexpr int kJThreads = 128;
+constexpr int kKVTile = kTK * kD * 2;  // 8 KB: one K or V tile (64 rows x 128 B)
+
+struct AttnJointK {
+  int H, Lq, Lk, splits, kps, ready, ld_out;
+  int zk0, zv0;
+  const __nv_bfloat16* q;
+  __nv_bfloat16* out;
+  unsigned* status;
+};
+
+__device__ __forceinline__ void jt_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t jt_cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_f2(uint32_t addr, float x, float y) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
+}
+
+// The K/V ring and the Q tile; after the flash loop rank 0's copy of this
+// region holds the partials ([split][Lq][64] O, then [split][Lq][2] max / sum).
+constexpr int kJRegion = kJStages * 2 * kKVTile + kTQ * 128;
+constexpr size_t kJSmem = kJRegion + kJStages * 8;
+// A launch that has the GPU to itself asks for more than it needs, so that its
+// CTAs land one per SM (each with the SM's whole L1 / TMA bandwidth): the
+// 10-step chunk ran 19.07 ms this way against 19.77 ms at three per SM.
+constexpr size_t kJSmemSpread = 120 * 1024;
+// Splits whose partials fit the region: splits * Lq * (64 + 2) floats.
+__host__ __device__ constexpr bool joint_fits(int splits, int Lq) { return (size_t)splits * Lq * (kD + 2) * 4 <= kJRegion; }
+
+__global__ void __launch_bounds__(kJThreads, 1)
+    attn_joint_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                      const AttnJointK a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // TMA's 128-byte swizzle is a function of the address bits (tile bases on
+  // 1024-byte boundaries); every CTA of the cluster sees the same layout
+  if (smem_u32(smem_raw) & 1023) {
+    if (threadIdx.x == 0) atomicOr(a.status, kStatusTimeoutDrain);
+    return;
+  }
+  uint8_t* sKV = smem_raw;                                   // [stage][K | V]
+  uint8_t* sQ = sKV + kJStages * 2 * kKVTile;                // [64][128 B]
+  float* sO = reinterpret_cast<float*>(smem_raw);            // rank 0, after the loop: [split][Lq][64] partial O
+  float* sML = sO + a.splits * a.Lq * kD;                    // rank 0, after the loop: [split][Lq][2] max, sum
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + kJRegion);
+  __shared__ int s_abort;
+  __shared__ float s_f[kJMaxSplits * kTQ];  // rank 0: merge weights [split][row]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int split = blockIdx.x % a.splits;  // = the rank in the cluster
+  const int bh = blockIdx.x / a.splits;
+  const int b = bh / a.H, h = bh % a.H;
+  const int k_begin = split * a.kps;
+  const int k_end = min(a.Lk, k_begin + a.kps);
+  const int ntiles = k_end > k_begin ? (k_end - k_begin + kTK - 1) / kTK : 0;
+
+  if (tid == 0) {
+    for (int st = 0; st < kJStages; ++st) mbar_init(&full[st], 1);
+    s_abort = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&map_k);
+    prefetch_tensormap(&map_v);
+  }
+  __syncthreads();
+  pdl_trigger();
+
+  auto issue = [&](int t) {  // tile t into stage t % kJStages
+    const int st = t % kJStages;
+    mbar_arrive_expect_tx(&full[st], 2 * kKVTile);
+    tma_load_3d(sKV + st * 2 * kKVTile, &map_k, &full[st], 0, k_begin + t * kTK, a.zk0 + bh);
+    tma_load_3d(sKV + st * 2 * kKVTile + kKVTile, &map_v, &full[st], 0, k_begin + t * kTK, a.zv0 + bh);
+  };
+  const int first = min(ntiles, kJStages);
+  int issued = 0;
+  if (tid == 0)  // tiles of keys complete before the launch
+    while (issued < first && min(k_end, k_begin + (issued + 1) * kTK) <= a.ready) issue(issued++);
+  pdl_wait();  // the queries and the action rows are the previous kernel's
+  if (tid == 0)
+    while (issued < first) issue(issued++);
+  const __nv_bfloat16* qb = a.q + (size_t)bh * a.Lq * kD;
+  load_tile(smem_u32(sQ), qb, 0, a.Lq, tid);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  const float sl2e = 1.4426950408889634f * rsqrtf((float)kD);
+  float o[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  uint32_t qf[4][4];
+#pragma unroll
+  for (int kt = 0; kt < 4; ++kt) {
+    const int r = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+    const int c = kt * 2 + (lane >> 4);
+    ldsm_x4(smem_u32(sQ) + tile_off(r, c), qf[kt][0], qf[kt][1], qf[kt][2], qf[kt][3]);
+  }
+
+  int consumed = 0;  // (thread 0) tiles whose copies have landed
+  for (int t = 0; t < ntiles; ++t) {
+    const int st = t % kJStages;
+    if (tid == 0) {
+      if (mbar_wait(&full[st], (t / kJStages) & 1, a.status, kStatusTimeoutTmaFull, nullptr))
+        consumed = t + 1;
+      else
+        s_abort = 1;
+    }
+    __syncthreads();
+    if (s_abort) break;  // (uniform: read after the barrier)
+    const uint32_t sK = smem_u32(sKV + st * 2 * kKVTile), sV = sK + kKVTile;
+    float s_[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s_[i][0] = s_[i][1] = s_[i][2] = s_[i][3] = 0.f;
+#pragma unroll
+    for (int kt = 0; kt < 4; ++kt) {
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        const int r = np * 16 + (lane & 7) + 8 * (lane >> 4);
+        const int c = kt * 2 + ((lane >> 3) & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sK + tile_off(r, c), b0, b1, b2, b3);
+        mma_bf16_16816(s_[2 * np], qf[kt][0], qf[kt][1], qf[kt][2], qf[kt][3], b0, b1);
+        mma_bf16_16816(s_[2 * np + 1], qf[kt][0], qf[kt][1], qf[kt][2], qf[kt][3], b2, b3);
+      }
+    }
+    // keys past this split's end (the tile's tail rows belong to the next split or lie past the list)
+    const int kbase = k_begin + t * kTK;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      const int k0 = kbase + nt * 8 + 2 * t4;
+      if (k0 >= k_end) s_[nt][0] = s_[nt][2] = -INFINITY;
+      if (k0 + 1 >= k_end) s_[nt][1] = s_[nt][3] = -INFINITY;
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) mx = fmaxf(mx, fmaxf(s_[nt][2 * r], s_[nt][2 * r + 1]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m_run[r], mx);
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = exp2f((m_run[r] - m_use) * sl2e);
+      float rs = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const float p0 = exp2f((s_[nt][2 * r] - m_use) * sl2e);
+        const float p1 = exp2f((s_[nt][2 * r + 1] - m_use) * sl2e);
+        s_[nt][2 * r] = p0;
+        s_[nt][2 * r + 1] = p1;
+        rs += p0 + p1;
+      }
+      l_run[r] = l_run[r] * alpha + rs;
+      m_run[r] = m_new;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        o[nt][2 * r] *= alpha;
+        o[nt][2 * r + 1] *= alpha;
+      }
+    }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint32_t a0 = pack_bf16(s_[2 * kk][0], s_[2 * kk][1]);
+      const uint32_t a1 = pack_bf16(s_[2 * kk][2], s_[2 * kk][3]);
+      const uint32_t a2 = pack_bf16(s_[2 * kk + 1][0], s_[2 * kk + 1][1]);
+      const uint32_t a3 = pack_bf16(s_[2 * kk + 1][2], s_[2 * kk + 1][3]);
+#pragma unroll
+      for (int dp = 0; dp < 4; ++dp) {
+        const int r = kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int c = dp * 2 + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sV + tile_off(r, c), b0, b1, b2, b3);
+        mma_bf16_16816(o[2 * dp], a0, a1, a2, a3, b0, b1);
+        mma_bf16_16816(o[2 * dp + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+    __syncthreads();  // the stage is read
+    if (tid == 0 && issued < ntiles) issue(issued++);  // tile t + kJStages into the freed stage
+  }
+  // never leave with copies in flight into this CTA's shared memory
+  if (tid == 0)
+    for (int t = consumed; t < issued; ++t)
+      mbar_wait(&full[t % kJStages], (t / kJStages) & 1, a.status, kStatusTimeoutDrain, nullptr);
+
+  float l_tot[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    float l = l_run[r];
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    l_tot[r] = l;
+  }
+  if (a.splits == 1) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int qi = warp * 16 + g + 8 * r;
+      if (qi < a.Lq) {
+        const float inv = 1.0f / l_tot[r];
+        __nv_bfloat16* dst = a.out + (size_t)(b * a.Lq + qi) * a.ld_out + h * kD;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+          *reinterpret_cast<uint32_t*>(dst + nt * 8 + 2 * t4) = pack_bf16(o[nt][2 * r] * inv, o[nt][2 * r + 1] * inv);
+      }
+    }
+    return;
+  }
+  // partial of this split -> rank 0's shared memory, once every CTA of the
+  // cluster is done with its ring (rank 0's is overwritten)
+  jt_cluster_sync();
+  const uint32_t rO = jt_cluster_addr(sO + (size_t)split * a.Lq * kD, 0);
+  const uint32_t rML = jt_cluster_addr(sML + (size_t)split * a.Lq * 2, 0);
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int row = warp * 16 + g + 8 * r;
+    if (row < a.Lq) {
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+        st_cluster_f2(rO + (uint32_t)(row * kD + nt * 8 + 2 * t4) * 4, o[nt][2 * r], o[nt][2 * r + 1]);
+      if (t4 == 0) st_cluster_f2(rML + (uint32_t)row * 8, m_run[r], l_tot[r]);
+    }
+  }
+  jt_cluster_sync();  // every partial is in rank 0's shared memory
+  if (split != 0) return;
+  // merge in split order: M = max_s m_s, f_s = 2^((m_s - M) c) / sum_s 2^((m_s - M) c) l_s
+  if (tid < a.Lq) {
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < a.splits; ++s2) M = fmaxf(M, sML[(s2 * a.Lq + tid) * 2]);
+    float den = 0.f;
+    for (int s2 = 0; s2 < a.splits; ++s2) {
+      const float f = exp2f((sML[(s2 * a.Lq + tid) * 2] - M) * sl2e);
+      s_f[s2 * kTQ + tid] = f;
+      den += f * sML[(s2 * a.Lq + tid) * 2 + 1];
+    }
+    const float inv = 1.0f / den;
+    for (int s2 = 0; s2 < a.splits; ++s2) s_f[s2 * kTQ + tid] *= inv;
+  }
+  __syncthreads();
+  for (int i = tid; i < a.Lq * (kD / 4); i += kJThreads) {
+    const int row = i / (kD / 4), c4 = i % (kD / 4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s2 = 0; s2 < a.splits; ++s2) {
+      const float f = s_f[s2 * kTQ + row];
+      const float4 v4 = reinterpret_cast<const float4*>(sO + ((size_t)s2 * a.Lq + row) * kD)[c4];
+      acc.x += f * v4.x;
+      acc.y += f * v4.y;
+      acc.z += f * v4.z;
+      acc.w += f * v4.w;
+    }
+    uint2 w;
+    w.x = pack_bf16(acc.x, acc.y);
+    w.y = pack_bf16(acc.z, acc.w);
+    *reinterpret_cast<uint2*>(a.out + (size_t)(b * a.Lq + row) * a.ld_out + h * kD + 4 * c4) = w;
+  }
+}
+
 }  // namespace
 
 size_t attention_ws_floats(int B, int H, int Dh, int Lq, int splits) {
@@ -389,6 +664,56 @@ cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t s) {
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+int attention_joint_splits(int BH, int Lq, int Lk, int num_sms) {
+  int sp = 1;
+  while (sp < kJMaxSplits && BH * sp * 2 <= num_sms && Lk >= 2 * sp * kTK && joint_fits(2 * sp, Lq)) sp *= 2;
+  return sp;
+}
+
+cudaError_t prepare_attention_joint() {
+  return cudaFuncSetAttribute(attn_joint_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kJSmemSpread);
+}
+
+cudaError_t launch_attention_joint(const AttnJoint& t, cudaStream_t s) {
+  const int ldo = t.ld_out ? t.ld_out : t.H * kD;
+  if (t.Lq < 1 || t.Lq > kTQ || t.Lk < 1 || t.B < 1 || t.H < 1 || ldo < t.H * kD || ldo % 4) return cudaErrorInvalidValue;
+  if (t.splits != 1 && t.splits != 2 && t.splits != 4 && t.splits != 8) return cudaErrorInvalidValue;
+  if (!joint_fits(t.splits, t.Lq)) return cudaErrorInvalidValue;
+  AttnJointK k;
+  k.H = t.H;
+  k.Lq = t.Lq;
+  k.Lk = t.Lk;
+  k.splits = t.splits;
+  k.kps = (t.Lk + t.splits - 1) / t.splits;
+  k.ready = t.ready;
+  k.ld_out = ldo;
+  k.zk0 = t.zk0;
+  k.zv0 = t.zv0;
+  k.q = reinterpret_cast<const __nv_bfloat16*>(t.q);
+  k.out = reinterpret_cast<__nv_bfloat16*>(t.out);
+  k.status = t.status;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(t.B * t.H * t.splits);
+  cfg.blockDim = dim3(kJThreads);
+  cfg.dynamicSmemBytes = t.spread ? kJSmemSpread : kJSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = t.splits;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = 1;
+  ++na;
+  if (pdl_enabled()) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, attn_joint_kernel, *t.map_k, *t.map_v, k);
 }
 
 }  // namespace wam

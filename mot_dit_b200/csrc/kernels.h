@@ -206,6 +206,32 @@ cudaError_t launch_attention_bf16(const AttnArgs& a, cudaStream_t s);
 // any launch (and never during stream capture).
 cudaError_t prepare_attention_bf16();
 
+// Joint action attention: queries q [B, H, Lq, 64] bf16 (Lq <= 64) over
+// cache rows [0, Lk) of the K / V maps ([z][rows][64] bf16, box 64 x 64
+// rows; (b, h) reads matrix z0 + b*H + h), out bf16 rows ld_out apart (0:
+// H*64).  `splits` (1, 2, 4, 8; splits * Lq <= 279) CTAs per (b, h) form a cluster, each taking a
+// contiguous key range; their partials are merged in split order in the
+// cluster's shared memory.  Cache rows below `ready` must be complete before
+// the launch (they are read before the dependent-launch wait); 0 makes no
+// such assumption.
+struct AttnJoint {
+  const CUtensorMap* map_k;
+  const CUtensorMap* map_v;
+  int zk0, zv0;
+  const void* q;
+  void* out;
+  int B, H, Lq, Lk, ld_out;
+  int ready;
+  int splits;
+  bool spread = false;  // one CTA per SM (more shared memory than it needs): for launches with the GPU to themselves
+  unsigned* status;
+};
+cudaError_t launch_attention_joint(const AttnJoint& a, cudaStream_t s);
+cudaError_t prepare_attention_joint();
+// Splits for B*H (sample, head) pairs of Lq queries over Lk keys on num_sms
+// SMs (the partials of all splits fit one CTA's K/V ring: splits * Lq <= 279).
+int attention_joint_splits(int BH, int Lq, int Lk, int num_sms);
+
 // Tensor-core (tcgen05) attention for video queries: one pass over keys
 // [0, Lk) for 128-query tiles.  Q / K / V are 3-D TMA maps over [z][rows][64]
 // bf16 (Q box 64 x 128 rows, K / V box 64 x 64 rows); (b, h) reads matrix

@@ -114,6 +114,8 @@ struct wam_ctx {
   GemmPlan p_a_in, p_a_qkv, p_a_o, p_a_f1, p_a_f2, p_a_out;
   GemmPlan p_u_qkv, p_u_o, p_u_f1, p_u_f2;  // LoRA down-projections u = s x A^T
   int attn_splits = 1;
+  int attn_joint_splits = 0;  // joint action attention on clusters (0: the split-KV kernel)
+  bool attn_spread = true;    // ... one CTA per SM (no video kernels beside it)
   // The action expert's norms run inside the GEMM that consumes them (opt-in;
   // the tokens must fit one 32/64-wide tile and K <= 1024).
   bool fuse_norm_a = false;
@@ -566,6 +568,31 @@ wam_status attention(wam_ctx* c, bool video, int i, cudaStream_t s) {
     CK(launch_attention_tc(t, s));
     return WAM_OK;
   }
+  if (d.bf16 && c->attn_joint_splits > 0) {
+    // action queries over [K^v_i; K^a_i].  Nothing is read before the
+    // dependent-launch wait: under stream capture the edge from the video
+    // stream's event also arrives as a programmatic dependency, so the video
+    // rows too are complete only after the wait (read earlier, the captured
+    // CEWP chunk differed from the sequential one).
+    AttnJoint t;
+    t.map_k = &c->m_cache;
+    t.map_v = &c->m_cache;
+    t.zk0 = (2 * i) * d.B * d.H;
+    t.zv0 = (2 * i + 1) * d.B * d.H;
+    t.q = c->q_a;
+    t.out = c->o_a;
+    t.B = d.B;
+    t.H = d.H;
+    t.Lq = d.La;
+    t.Lk = d.Lv + d.La;
+    t.ld_out = d.lo;
+    t.ready = 0;
+    t.splits = c->attn_joint_splits;
+    t.spread = c->attn_spread;
+    t.status = c->status;
+    CK(launch_attention_joint(t, s));
+    return WAM_OK;
+  }
   CK(d.bf16 ? launch_attention_bf16(a, s) : launch_attention_f32(a, s));
   return WAM_OK;
 }
@@ -850,6 +877,9 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
   if (c->ab_on) return enqueue_action_step_blocks(c, s, io, j, ev_wait, record_used);
   const Dims& d = c->d;
   const ExpertIdx& x = c->ea;
+  // a step that waits on the video blocks runs beside them: its attention
+  // takes little shared memory per CTA so the video GEMMs keep their SMs
+  c->attn_spread = ev_wait == nullptr;
   c->cur_cls = WAM_PROF_ACTION_TEMB;
   RET(temb(c, false, &io->sched[j], s));
   c->cur_cls = WAM_PROF_ACTION_IO;
@@ -1151,6 +1181,7 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
   CK(prepare_tc_gemm());
   CK(prepare_attention_tc());
   CK(prepare_attention_bf16());
+  CK(prepare_attention_joint());
   Dims& d = c->d;
   d.N = cfg->n_blocks; d.dv = cfg->d_video; d.da = cfg->d_action; d.H = cfg->n_heads; d.Dh = cfg->head_dim;
   d.A = d.H * d.Dh; d.Fv = cfg->ffn_video; d.Fa = cfg->ffn_action; d.Lc = cfg->l_cond; d.Lvid = cfg->l_video;
@@ -1349,6 +1380,11 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     if (d.Pv > 0) need(c->p_v_in, d.Mv, d.dv, d.Pv, false, &ws_v, &tiles_v);
     if (cfg->video_has_output) need(c->p_v_out, d.Mv, d.Pv, d.dv, false, &ws_v, &tiles_v);
     c->attn_splits = std::max(1, (d.Lv + d.La + 127) / 128);
+    // Joint action attention on clusters of key splits (WAM_JOINT_ATTN=0:
+    // the split-KV kernel with a ticket combine)
+    const char* jav = getenv("WAM_JOINT_ATTN");
+    if (!(jav && jav[0] == '0') && d.Dh == 64 && d.La <= 64)
+      c->attn_joint_splits = attention_joint_splits(d.B * d.H, d.La, d.Lv + d.La, nsm);
   }
   RET(dalloc(c, &c->ws_gemm, ws * 4));
   RET(dalloc(c, &c->tk_gemm, (size_t)tiles * 2 * 4));
@@ -2047,6 +2083,44 @@ wam_status wam_op_linear_tiled(const void* x, const void* w, const float* bias, 
                                int pair, int ctas, void* stream) {
   if (!x || !w || !bias || !out || M < 1 || N < 1 || K < 1 || ctas < 0) return WAM_ERR_INVALID_ARG;
   return op_linear_bf16(x, w, bias, out, M, N, K, false, ctas, bn, pair != 0, (cudaStream_t)stream);
+}
+
+wam_status wam_op_attention_joint(const void* q, const void* k, const void* v, void* out, int B, int H, int Lq, int Lk,
+                                  int Lcache, int ready, int splits, void* stream) {
+  if (!q || !k || !v || !out || B < 1 || H < 1 || Lq < 1 || Lq > 64 || Lk < 1 || Lk > Lcache || ready < 0 ||
+      ready > Lcache || splits < 0)
+    return WAM_ERR_INVALID_ARG;
+  static thread_local unsigned* status = nullptr;
+  if (!status) {
+    if (prepare_attention_joint() != cudaSuccess) return WAM_ERR_CUDA;
+    if (cudaMalloc(&status, 4) != cudaSuccess) return WAM_ERR_OOM;
+    if (cudaMemset(status, 0, 4) != cudaSuccess) return WAM_ERR_CUDA;
+  }
+  if (splits == 0) {
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    splits = attention_joint_splits(B * H, Lq, Lk, nsm);
+  }
+  CUtensorMap mk, mv;
+  const size_t mat = (size_t)Lcache * 64 * 2;
+  if (!make_tmap_3d(&mk, k, 64, Lcache, B * H, mat, 64) || !make_tmap_3d(&mv, v, 64, Lcache, B * H, mat, 64))
+    return WAM_ERR_INVALID_ARG;
+  AttnJoint t;
+  t.map_k = &mk;
+  t.map_v = &mv;
+  t.zk0 = t.zv0 = 0;
+  t.q = q;
+  t.out = out;
+  t.B = B;
+  t.H = H;
+  t.Lq = Lq;
+  t.Lk = Lk;
+  t.ld_out = 0;
+  t.ready = ready;
+  t.splits = splits;
+  t.status = status;
+  return launch_attention_joint(t, (cudaStream_t)stream) == cudaSuccess ? WAM_OK : WAM_ERR_INVALID_ARG;
 }
 
 wam_status wam_op_norm_mod(int dtype, const float* x, void* h, int M, int d, const float* scale, const float* shift,

@@ -97,6 +97,34 @@ def test_linear_cta_pairs_repeatable():
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
 
+# Joint action attention: (sample, head) split over a cluster of CTAs.
+@pytest.mark.parametrize("B,H,Lq,Lk,Lc,splits,ready", [
+    (1, 24, 32, 1120, 1120, 0, 1088),  # the Fast-WAM-shaped action attention (4 splits), video rows early
+    (1, 4, 32, 1120, 1120, 8, 0),      # 8 splits of 140 keys (ragged tiles)
+    (2, 3, 16, 300, 310, 2, 256),      # 16 queries, a key list shorter than the cache
+    (1, 2, 64, 200, 256, 4, 0),        # 64 queries, 50-key splits (one partial tile each)
+    (3, 2, 7, 70, 70, 1, 70),          # one CTA per (sample, head): no merge
+])
+def test_attention_joint(B, H, Lq, Lk, Lc, splits, ready):
+    q, k, v = _attn_case(B, H, 64, Lq, Lk, Lc, Lq + Lk + splits)
+    q, k, v = (round_bf16(a) for a in (q, k, v))
+    outs = []
+    for rd in (ready, 0):
+        out = torch.full((B * Lq, H * 64), float("nan"), device=DEV, dtype=torch.bfloat16)
+        W.op_attention_joint(_bf16(q), _bf16(k), _bf16(v), out, B, H, Lq, Lk, Lc, ready=rd, splits=splits)
+        torch.cuda.synchronize()
+        outs.append(out.float().cpu().numpy())
+    # reading the early rows before the wait changes only when they load
+    assert np.array_equal(outs[0], outs[1])
+    got = outs[0]
+    q64, k64, v64 = q.astype(np.float64), k[:, :, :Lk].astype(np.float64), v[:, :, :Lk].astype(np.float64)
+    ref = M.merge_heads(M.attention(q64, k64, v64)).reshape(B * Lq, H * 64)
+    ref_absv = M.merge_heads(M.attention(q64, k64, np.abs(v64))).reshape(B * Lq, H * 64)
+    assert np.isfinite(got).all()
+    assert rel_l2(got, ref) < 1e-2
+    assert_elementwise(got, ref, ref_absv)
+
+
 def test_linear_f32():
     rng = np.random.default_rng(1)
     x = rng.standard_normal((70, 48)).astype(np.float32)
