@@ -446,25 +446,42 @@ __global__ void __launch_bounds__(kJThreads, 1)
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  // Up to 32 queries: warp w takes query rows 16 (w & 1) .. + 15 and the key
+  // tiles of parity w >> 1, so two warp pairs work on two tiles at once and
+  // merge at the end; up to 64 queries: warp w takes rows 16 w .. + 15 and
+  // every tile.
+  const bool halves = a.Lq <= 32;
+  const int tpi = halves ? 2 : 1;  // tiles per iteration
+  const int qrow0 = (halves ? (warp & 1) : warp) * 16;
+  const int kh = halves ? (warp >> 1) : 0;
   uint32_t qf[4][4];
 #pragma unroll
   for (int kt = 0; kt < 4; ++kt) {
-    const int r = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+    const int r = qrow0 + (lane & 7) + 8 * ((lane >> 3) & 1);
     const int c = kt * 2 + (lane >> 4);
     ldsm_x4(smem_u32(sQ) + tile_off(r, c), qf[kt][0], qf[kt][1], qf[kt][2], qf[kt][3]);
   }
 
   int consumed = 0;  // (thread 0) tiles whose copies have landed
-  for (int t = 0; t < ntiles; ++t) {
-    const int st = t % kJStages;
+  for (int t0 = 0; t0 < ntiles; t0 += tpi) {
     if (tid == 0) {
-      if (mbar_wait(&full[st], (t / kJStages) & 1, a.status, kStatusTimeoutTmaFull, nullptr))
-        consumed = t + 1;
-      else
-        s_abort = 1;
+      for (int u = t0; u < min(ntiles, t0 + tpi); ++u) {
+        if (mbar_wait(&full[u % kJStages], (u / kJStages) & 1, a.status, kStatusTimeoutTmaFull, nullptr)) {
+          consumed = u + 1;
+        } else {
+          s_abort = 1;
+          break;
+        }
+      }
     }
     __syncthreads();
     if (s_abort) break;  // (uniform: read after the barrier)
+    const int t = t0 + kh;
+    if (t >= ntiles) {  // (the odd pair past the last tile)
+      __syncthreads();
+      continue;
+    }
+    const int st = t % kJStages;
     const uint32_t sK = smem_u32(sKV + st * 2 * kKVTile), sV = sK + kKVTile;
     float s_[8][4];
 #pragma unroll
@@ -532,8 +549,9 @@ __global__ void __launch_bounds__(kJThreads, 1)
         mma_bf16_16816(o[2 * dp + 1], a0, a1, a2, a3, b2, b3);
       }
     }
-    __syncthreads();  // the stage is read
-    if (tid == 0 && issued < ntiles) issue(issued++);  // tile t + kJStages into the freed stage
+    __syncthreads();  // the stages are read
+    if (tid == 0)  // tiles t0 + kJStages .. into the freed stages
+      while (issued < ntiles && issued < t0 + tpi + kJStages) issue(issued++);
   }
   // never leave with copies in flight into this CTA's shared memory
   if (tid == 0)
@@ -548,10 +566,46 @@ __global__ void __launch_bounds__(kJThreads, 1)
     l += __shfl_xor_sync(0xffffffffu, l, 2);
     l_tot[r] = l;
   }
+  __syncthreads();  // (thread 0's drain above: the ring is idle)
+  if (halves) {
+    // the odd-tile pair hands (O, m, l) over in the idle ring; the even-tile
+    // pair merges them into its own (log-sum-exp weights)
+    float* xo = reinterpret_cast<float*>(sKV);  // [32 rows][64]
+    float* xml = xo + 32 * kD;                  // [32 rows][2]
+    if (kh == 1) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = qrow0 + g + 8 * r;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+          *reinterpret_cast<float2*>(xo + row * kD + nt * 8 + 2 * t4) = make_float2(o[nt][2 * r], o[nt][2 * r + 1]);
+        if (t4 == 0) *reinterpret_cast<float2*>(xml + row * 2) = make_float2(m_run[r], l_tot[r]);
+      }
+    }
+    __syncthreads();
+    if (kh == 0) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = qrow0 + g + 8 * r;
+        const float2 ml1 = *reinterpret_cast<const float2*>(xml + row * 2);
+        const float M = fmaxf(m_run[r], ml1.x);  // m_run[r] is finite: the even pair has tile 0
+        const float f0 = exp2f((m_run[r] - M) * sl2e), f1 = exp2f((ml1.x - M) * sl2e);
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          const float2 o1 = *reinterpret_cast<const float2*>(xo + row * kD + nt * 8 + 2 * t4);
+          o[nt][2 * r] = o[nt][2 * r] * f0 + o1.x * f1;
+          o[nt][2 * r + 1] = o[nt][2 * r + 1] * f0 + o1.y * f1;
+        }
+        l_tot[r] = l_tot[r] * f0 + ml1.y * f1;
+        m_run[r] = M;
+      }
+    }
+  }
+  const bool owner = kh == 0;  // this warp holds merged rows
   if (a.splits == 1) {
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int qi = warp * 16 + g + 8 * r;
+    for (int r = 0; r < 2 && owner; ++r) {
+      const int qi = qrow0 + g + 8 * r;
       if (qi < a.Lq) {
         const float inv = 1.0f / l_tot[r];
         __nv_bfloat16* dst = a.out + (size_t)(b * a.Lq + qi) * a.ld_out + h * kD;
@@ -569,8 +623,8 @@ __global__ void __launch_bounds__(kJThreads, 1)
   const uint32_t rML = jt_cluster_addr(sML + (size_t)split * a.Lq * 2, 0);
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
-    const int row = warp * 16 + g + 8 * r;
-    if (row < a.Lq) {
+    const int row = qrow0 + g + 8 * r;
+    if (owner && row < a.Lq) {
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
         st_cluster_f2(rO + (uint32_t)(row * kD + nt * 8 + 2 * t4) * 4, o[nt][2 * r], o[nt][2 * r + 1]);
