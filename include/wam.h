@@ -312,14 +312,18 @@ wam_status wam_op_linear(int dtype, const void* dev_x, const void* dev_w, const 
                          int M, int N, int K, int swap, int splits, void* stream);
 
 /* The same product through the video expert's tile shapes (bf16 only, normal
- * orientation, fp32 out): bn = 128 or 256 output features per CTA tile, and
- * pair = 1 runs 256-wide tiles on CTA pairs -- two CTAs of a cluster share
- * each M = 256 tensor-core MMA (the 2-SM form), each holding its own 128 rows
- * of X and half of the 256 rows of W.  ctas = persistent CTAs (0: one per
- * SM; rounded down to pairs).  K a multiple of 64, N a multiple of 32.
- * Returns WAM_ERR_INVALID_ARG for other shapes or bn / pair values. */
+ * orientation, fp32 out): bn = 128 or 256 output features per CTA tile.
+ * mode 0: single CTAs.  mode 1 (bn 256): CTA pairs -- two CTAs of a cluster
+ * share each M = 256 tensor-core MMA (the 2-SM form), each holding its own
+ * 128 rows of X and half of the 256 rows of W.  mode 2: single-CTA tiles
+ * launched as clusters of two CTAs; a tile whose k-range the stream-K split
+ * gives to the two CTAs of one cluster is finished in column halves, each
+ * CTA's half-partial of the other's columns crossing in shared memory.
+ * ctas = persistent CTAs (0: one per SM; even for mode 2, rounded down to
+ * pairs for mode 1).  K a multiple of 64, N a multiple of 32.  Returns
+ * WAM_ERR_INVALID_ARG for other shapes or values. */
 wam_status wam_op_linear_tiled(const void* dev_x, const void* dev_w, const float* dev_bias, float* dev_out, int M,
-                               int N, int K, int bn, int pair, int ctas, void* stream);
+                               int N, int K, int bn, int mode, int ctas, void* stream);
 
 /* out[B*Lq, H*Dh] = softmax(q k^T / sqrt(Dh)) v per (sample, head) over
  * cache rows [0, Lk); q [B, H, Lq, Dh], k / v [B, H, Lcache, Dh]; bf16

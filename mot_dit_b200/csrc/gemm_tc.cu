@@ -112,6 +112,7 @@ struct GemmK {
   float* ws;     // [G][2][BM * BN] partial tiles
   int* tickets;  // [tiles][2]: pieces arrived, pieces published
   unsigned* status;
+  int csplit;    // launched as clusters of two CTAs: a tile split between them is finished in halves
 };
 
 // First k-block of CTA c, and the CTA owning k-block x (the largest c with
@@ -172,6 +173,14 @@ __device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+// Bulk copy of `bytes` from this CTA's shared memory to cluster address `dst`
+// (another CTA of the cluster), completing on the barrier at cluster address
+// `bar` in that CTA (no multicast).
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "r"(smem_u32(src)), "r"(bytes), "r"(bar)
+               : "memory");
 }
 // TMEM allocation of a pair: the same warp of both CTAs, same slot offset.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot_smem, uint32_t ncols) {
@@ -467,7 +476,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acce = accf + 2;            // [2] accumulator drained (epilogue -> MMA)
   uint64_t* redb = acce + 2;            // partial tiles copied into the ring
   uint64_t* bready = redb + 1;          // fused-norm B operand written (epilogue warps -> MMA)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bready + 1);
+  uint64_t* peer_idle = bready + 1;     // cluster split: the partner's ring may take my half-partial
+  uint64_t* peer_data = peer_idle + 1;  // cluster split: the partner's half-partial is in my ring
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(peer_data + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -493,6 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(redb, 1);
     mbar_init(bready, 1);
+    mbar_init(peer_idle, 1);
+    mbar_init(peer_data, 1);
     *abort_flag = 0;
     *last_flag = 0;
     fence_barrier_init();
@@ -515,6 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if constexpr (PAIR) cluster_sync();  // the peer's barriers exist before any remote arrival
+  if (!PAIR && g.csplit) cluster_sync();  // (the same for the cluster split; g is uniform)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_trigger();  // the next kernel may start its own set-up now
@@ -777,6 +791,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int c_first = kowner(g, t0);
       const int npieces = kowner(g, t0 + g.KB - 1) - c_first + 1;
       const int buf = lt & 1;
+      // A tile split in two between the CTAs of a cluster that covers exactly
+      // their whole k-ranges (stream-K gave CTAs 2k and 2k + 1 one piece each
+      // and nothing else): each CTA finishes half of the columns, the
+      // partner's half-partial arriving in its idle ring through the
+      // cluster's shared window.  Both CTAs decide this alike from g and t.
+      const bool cs = !SWAP && !PAIR && C::kStages * C::kStageBytes >= BM * BN * 4 && g.csplit && npieces == 2 &&
+                      (c_first & 1) == 0 && kbound(g, c_first) == t0 && kbound(g, c_first + 2) == t0 + g.KB;
+      const int c_lo = cs ? (unit - c_first) * (BN / 2) : 0;
+      const int c_hi = cs ? c_lo + BN / 2 : BN;
       const int m0w = arow(ta) + quad * 32;  // normal orientation: this warp's first row
       const int tk = PAIR ? 2 * t + (int)rank : t;  // the tickets of this CTA's 128-row tile
       const int nb = tb * BN;
@@ -810,11 +833,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) bulk_wait_read<0>();  // earlier stores have left the staging
         __syncwarp();
         if constexpr (C::kResBoxes) {
-          // residual boxes 0 and 1 (columns [0, 64)); later boxes stream in
-          // during the epilogue
+          // residual boxes 0 and 1 (columns [c_lo, c_lo + 64)); later boxes
+          // stream in during the epilogue
           for (int k = lane; k < 32 * 16; k += 32) {
             const int r = k >> 4, q4 = k & 15;
-            const int m = m0w + r, n = nb + 4 * q4;
+            const int m = m0w + r, n = nb + c_lo + 4 * q4;
             const bool v = m < g.rows_a && n < g.rows_b;
             cp_async16(smem_u32(box_chunk(stg + (q4 >> 3) * kBox, r, q4 & 7)),
                        v ? (const void*)(R.out_f32 + (size_t)m * R.ld + n) : (const void*)R.out_f32, v);
@@ -866,12 +889,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
 
       if (threadIdx.x == 64 && x == x_end) WAM_TL(5, globaltimer());  // last segment's accumulator ready
+      if (cs) {
+        // My ring is idle (this segment's MMAs are done, nothing in flight).
+        // Its first half receives the partner's half-partial of my columns,
+        // its second half stages mine of the partner's columns, both as
+        // [32-column chunk][row][32 floats] with the 16-byte chunks of a row
+        // rotated by (row & 7) (conflict-free shared-memory access).
+        constexpr uint32_t kHalf = BM * (BN / 2) * 4;
+        const uint32_t peer = (uint32_t)((unit - c_first) ^ 1);
+        if (threadIdx.x == 64) {
+          mbar_arrive_expect_tx(peer_data, kHalf);  // what the partner will send
+          mbar_arrive_cluster(cluster_addr(peer_idle, peer));  // it may send now
+        }
+        const int o_lo = BN / 2 - c_lo;  // the partner's columns
+        uint8_t* stage = smem + kHalf;
+        for (int c = 0; c < BN / 2; c += 32) {
+          float v[32];
+          tmem_ld32(t_row + o_lo + c, v);
+          uint8_t* d = stage + ((c >> 5) * BM + row) * 128;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(d + ((q ^ (row & 7)) << 4)) =
+                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+        fence_proxy_async_smem();  // generic writes -> the bulk copy
+        epi_bar();
+        if (threadIdx.x == 64) {
+          if (!mbar_wait(peer_idle, 0, g.status, kStatusTimeoutPeer, abort_flag)) {
+            *abort_flag = 1;
+          } else {
+            bulk_copy_to_peer(cluster_addr(smem, peer), stage, kHalf, cluster_addr(peer_data, peer));
+            bulk_commit();
+          }
+        }
+        if (!mbar_wait(peer_data, 0, g.status, kStatusTimeoutPeer, abort_flag)) *abort_flag = 1;
+        if (threadIdx.x == 64) bulk_wait_read<0>();  // my staging has been read out (before it is reused)
+        epi_bar();
+        if (threadIdx.x == 64 && x == x_end) WAM_TL(6, globaltimer());  // exchange done
+        if (*abort_flag) break;
+      }
       // ---- a tile shared with other CTAs (see "Split tiles" above)
       const int mine = unit - c_first;  // this CTA's piece of tile t
       // CTA holding piece p's partial (the same rank of the piece's pair)
       auto piece_cta = [&](int p) { return PAIR ? 2 * (c_first + p) + (int)rank : c_first + p; };
       bool from_smem = false;
-      if (npieces > 1) {
+      if (npieces > 1 && !cs) {
         if (threadIdx.x == 64) {
           const int prev = atomicAdd(g.tickets + 2 * tk, 1);
           *last_flag = (prev == npieces - 1) ? 1 : 0;
@@ -944,6 +1006,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       // columns [c, c + 32) of this thread's row: the accumulator, or the sum of
       // all pieces in k order with this CTA's own piece read from TMEM
       auto get = [&](int c, float* v) {
+        if (cs) {  // my piece from TMEM + the partner's, in my ring (two pieces: the order is immaterial)
+          tmem_ld32(t_row + c, *reinterpret_cast<float(*)[32]>(v));
+          if (c + 32 >= c_hi) release();
+          const uint8_t* rp = smem + ((size_t)((c - c_lo) >> 5) * BM + row) * 128;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 p4 = *reinterpret_cast<const float4*>(rp + ((q ^ (row & 7)) << 4));
+            v[4 * q] += p4.x;
+            v[4 * q + 1] += p4.y;
+            v[4 * q + 2] += p4.z;
+            v[4 * q + 3] += p4.w;
+          }
+          return;
+        }
         if (npieces == 1) {
           tmem_ld32(t_row + c, *reinterpret_cast<float(*)[32]>(v));
           if (c + 32 >= BN) release();
@@ -991,7 +1067,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (EPI == kClassStore) {
           const bool gelu = R.kind == kEpiGelu;
           const int cols = gelu ? 64 : 32;  // one 128-byte box row
-          for (int c = 0; c < BN; c += cols) {
+          for (int c = c_lo; c < c_hi; c += cols) {
             float v[64];
             get(c, v);
             if (gelu) get(c + 32, v + 32);
@@ -1032,21 +1108,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++nbox;
           }
         } else if constexpr (EPI == kClassRes) {
-          const int nvb = min(BN, g.rows_b - nb) / 32;  // boxes with valid columns
+          const int nvb = (min(c_hi, g.rows_b - nb) - c_lo) / 32;  // boxes with valid columns in [c_lo, c_hi)
           // box bi's residual rows into buffer bi & 1 (one cp.async group)
           auto load_box = [&](int bi) {
             uint8_t* dst = stg + (bi & 1) * kBox;
             for (int k = lane; k < 32 * 8; k += 32) {
               const int r = k >> 3, q = k & 7;
-              const int m = m0w + r, n = nb + 32 * bi + 4 * q;
+              const int m = m0w + r, n = nb + c_lo + 32 * bi + 4 * q;
               const bool v = m < g.rows_a;
               cp_async16(smem_u32(box_chunk(dst, r, q)),
                          v ? (const void*)(R.out_f32 + (size_t)m * R.ld + n) : (const void*)R.out_f32, v);
             }
             cp_async_commit();
           };
-          for (int c = 0; c < BN; c += 32) {
-            const int bi = c >> 5;
+          for (int c = c_lo; c < c_hi; c += 32) {
+            const int bi = (c - c_lo) >> 5;  // box index within this CTA's columns
             float v[32];
             get(c, v);
             if (!warp_rows || nb + c >= g.rows_b) continue;
@@ -1059,7 +1135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
               }
             }
-            uint8_t* box = stg + (C::kResBoxes ? (bi & 1) : bi) * kBox;  // the residual of these columns
+            uint8_t* box = stg + (C::kResBoxes ? (bi & 1) : (c >> 5)) * kBox;  // the residual of these columns
             const float4* b4 = reinterpret_cast<const float4*>(sVec + c);
             const float4* g4 = reinterpret_cast<const float4*>(sVec + BN + c);
 #pragma unroll
@@ -1089,7 +1165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if constexpr (EPI == kClassQkv) {
           // all 32 tokens valid and in one sample: one TMA store per head
           const bool whole = m0w + 32 <= g.rows_a && (m0w % R.seq_len) + 32 <= R.seq_len;
-          for (int c = 0; c < BN; c += 64) {
+          for (int c = c_lo; c < c_hi; c += 64) {
             float x[64];
             get(c, x);
             get(c + 32, x + 32);
@@ -1132,7 +1208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           // per-element epilogue (Euler update, video endpoint)
-          for (int c = 0; c < BN; c += 32) {
+          for (int c = c_lo; c < c_hi; c += 32) {
             float v[32];
             get(c, v);
             const int n0 = nb + c;
@@ -1342,11 +1418,14 @@ cudaError_t launch_one(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
   g.ws = t.ws;
   g.tickets = t.tickets;
   g.status = t.status;
+  g.csplit = (!PAIR && !SWAP && t.csplit && g.G % 2 == 0) ? 1 : 0;
   // unused output maps are passed as copies of the A map
   const CUtensorMap& mo = e.map_o ? *e.map_o : *t.map_a;
   const CUtensorMap& mo2 = e.map_o2 ? *e.map_o2 : *t.map_a;
   if constexpr (PAIR)
     return launch_pairs(tc_gemm_kernel<BN, SWAP, EPI, true>, g.G, C::kSmem, s, *t.map_a, *t.map_b, mo, mo2, g, e);
+  else if (g.csplit)  // clusters of two CTAs: grid 2 x (G / 2)
+    return launch_pairs(tc_gemm_kernel<BN, SWAP, EPI, false>, g.G / 2, C::kSmem, s, *t.map_a, *t.map_b, mo, mo2, g, e);
   else
     return launch_k(tc_gemm_kernel<BN, SWAP, EPI, false>, dim3(g.G), dim3(kThreads), C::kSmem, s, *t.map_a, *t.map_b,
                     mo, mo2, g, e);

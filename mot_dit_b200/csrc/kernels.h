@@ -138,6 +138,9 @@ struct TcGemm {
   int max_ctas;              // normal: persistent grid size (0: one CTA per SM)
   bool pair;                 // normal, bn 256: CTA pairs share M = 256 MMAs (2-SM tensor-core tiles);
                              // the B map's box is then bn / 2 rows (each CTA loads half)
+  bool csplit;               // normal, single CTAs: launch as clusters of two (even grid); a tile whose
+                             // k-range stream-K splits between the two CTAs of a cluster is finished
+                             // in column halves, the partials crossing in shared memory
   float* ws;                 // partial tiles: 2 * CTAs * 128 * bn floats (tc_gemm_ws_floats)
   int* tickets;              // two per output tile, zero on entry, left zero
   unsigned* status;

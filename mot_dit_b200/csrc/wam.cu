@@ -62,7 +62,8 @@ struct Dims {
 
 struct GemmPlan {
   int bn = 128, splits = 1, max_ctas = 0;
-  bool pair = false;  // normal orientation, bn 256: CTA pairs (2-SM MMA)
+  bool pair = false;    // normal orientation, bn 256: CTA pairs (2-SM MMA)
+  bool csplit = false;  // normal orientation: clusters of two, split tiles finished in column halves
 };
 
 }  // namespace
@@ -391,6 +392,7 @@ wam_status run_tc(wam_ctx* c, const CUtensorMap& A, const CUtensorMap& Bm, int r
   g.swap = swap;
   g.max_ctas = p.max_ctas;
   g.pair = p.pair;
+  g.csplit = p.csplit;
   g.ws = video ? c->ws_gemm_v : c->ws_gemm;
   g.tickets = video ? c->tk_gemm_v : c->tk_gemm;
   g.status = c->status;
@@ -1309,6 +1311,27 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
       c->p_v_o = {bn_o, 1, grid(d.dv, bn_o, false)};
       c->p_v_f1 = {256, 1, grid(d.Fv, 256, false)};
       c->p_v_f2 = {bn_f2, 1, grid(d.dv, bn_f2, false)};
+      // Cluster split for the d-wide gate-residual GEMMs when their 256-wide
+      // tiles number about half the grid and each half of the k-range is at
+      // least 24 k-blocks deep: each tile's k-range is split between the two
+      // CTAs of a cluster, which finish it in column halves (the partials
+      // crossing in shared memory, ~3 us).  At 1088 tokens FFN-down (96
+      // k-blocks): 54 tiles on 108 CTAs, 36.9 -> 26.1 us per launch alone,
+      // config-2 chunk 4.12 -> 3.91 ms.  The out-projection (24 k-blocks) is
+      // left on 128-wide whole tiles: split, it measured 1.7 us slower per
+      // launch in the chunk.  WAM_VIDEO_CSPLIT=0 (or a tile-width override)
+      // keeps the rule above.
+      const char* csv = getenv("WAM_VIDEO_CSPLIT");
+      const bool csplit_ok = !(csv && csv[0] == '0');
+      auto csplit_plan = [&](GemmPlan* p, int n_out, int K, const char* bn_var) {
+        const int tiles = ((d.Mv + 127) / 128) * (n_out / 256);
+        if (!csplit_ok || getenv(bn_var) || n_out % 256 || 2 * tiles > nsm || 4 * (2 * tiles) < 3 * vctas ||
+            K / 64 < 48)
+          return;
+        *p = GemmPlan{256, 1, 2 * tiles, false, true};
+      };
+      csplit_plan(&c->p_v_o, d.dv, d.A, "WAM_VIDEO_OPROJ_BN");
+      csplit_plan(&c->p_v_f2, d.dv, d.Fv, "WAM_VIDEO_FFN2_BN");
     }
     c->p_v_in = {128, 1, grid(d.dv, 128, false)};
     c->p_v_out = {64, 1, grid(d.Pv > 0 ? d.Pv : 64, 64, false)};
@@ -2000,7 +2023,7 @@ namespace {
 // persistent CTAs (0: all SMs), pair = CTA pairs; swapped: `ctas` = CTAs per
 // output tile.
 wam_status op_linear_bf16(const void* x, const void* w, const float* bias, float* out, int M, int N, int K, bool swap,
-                          int ctas, int bn_normal, bool pair, cudaStream_t s) {
+                          int ctas, int bn_normal, bool pair, cudaStream_t s, bool csplit = false) {
   if (K % 64) return WAM_ERR_INVALID_ARG;
   const int bn = swap ? (M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256) : bn_normal;
   if (swap && M > 256) return WAM_ERR_INVALID_ARG;
@@ -2026,6 +2049,7 @@ wam_status op_linear_bf16(const void* x, const void* w, const float* bias, float
   g.swap = swap;
   g.max_ctas = swap ? 0 : std::max(0, ctas);
   g.pair = pair;
+  g.csplit = csplit;
   const size_t tickets = tc_gemm_tickets(g);
   static thread_local float* ws = nullptr;
   static thread_local int* tk = nullptr;
@@ -2080,9 +2104,11 @@ wam_status wam_op_linear(int dtype, const void* x, const void* w, const float* b
 }
 
 wam_status wam_op_linear_tiled(const void* x, const void* w, const float* bias, float* out, int M, int N, int K, int bn,
-                               int pair, int ctas, void* stream) {
-  if (!x || !w || !bias || !out || M < 1 || N < 1 || K < 1 || ctas < 0) return WAM_ERR_INVALID_ARG;
-  return op_linear_bf16(x, w, bias, out, M, N, K, false, ctas, bn, pair != 0, (cudaStream_t)stream);
+                               int mode, int ctas, void* stream) {
+  if (!x || !w || !bias || !out || M < 1 || N < 1 || K < 1 || ctas < 0 || mode < 0 || mode > 2)
+    return WAM_ERR_INVALID_ARG;
+  if (mode == 2 && ctas % 2) return WAM_ERR_INVALID_ARG;  // clusters of two: an even grid
+  return op_linear_bf16(x, w, bias, out, M, N, K, false, ctas, bn, mode == 1, (cudaStream_t)stream, mode == 2);
 }
 
 wam_status wam_op_attention_joint(const void* q, const void* k, const void* v, void* out, int B, int H, int Lq, int Lk,

@@ -89,6 +89,34 @@ def test_video_cta_pairs(monkeypatch, batch):
     wam.close()
 
 
+@pytest.mark.parametrize("batch", [1, 2])
+def test_video_cluster_split(monkeypatch, batch):
+    """The video FFN-down on 256-wide tiles split between the two CTAs of a
+    cluster (finished in column halves, the partials crossing in shared
+    memory): the grid is set to twice its tile count so the rule picks it at
+    this size.  Bitwise equal to the same partition reduced through global
+    memory, at parity with the oracle, CEWP == sequential."""
+    # FFN width 3072: FFN-down's k-range is deep enough (48 k-blocks) for the split
+    c = _mid().replace(batch=batch, ffn_video=3072)
+    ctas = str(2 * ((c.batch * (c.l_cond + c.l_video) + 127) // 128) * (c.d_video // 256))
+    inp = inputs(c, 23)
+    monkeypatch.setenv("WAM_VIDEO_GEMM_CTAS", ctas)
+    for k in ("WAM_VIDEO_CSPLIT", "WAM_VIDEO_OPROJ_BN", "WAM_VIDEO_FFN2_BN"):
+        monkeypatch.delenv(k, raising=False)
+    wam = W.Wam(c, seed=23)
+    got = run_chunk(wam, inp, S=2, mode=W.CEWP, use_graph=True)
+    for mode, graph in ((W.SEQUENTIAL, True), (W.CEWP, False)):
+        assert np.array_equal(run_chunk(wam, inp, S=2, mode=mode, use_graph=graph), got)
+    wam.close()
+    monkeypatch.setenv("WAM_VIDEO_CSPLIT", "0")
+    monkeypatch.setenv("WAM_VIDEO_FFN2_BN", "256")
+    wam = W.Wam(c, seed=23)
+    assert np.array_equal(run_chunk(wam, inp, S=2), got)
+    wam.close()
+    ref_a0, ref_veff = oracle_chunk(c, 23, inp, S=2)
+    check_parity(got, inp, ref_a0, ref_veff, c.dtype)
+
+
 @pytest.mark.parametrize("pair", ["0", "1"])
 def test_video_fused_norm(monkeypatch, pair):
     """Opt-in fused video norm (WAM_VIDEO_FUSED_NORM=1): the QKV / FFN-up

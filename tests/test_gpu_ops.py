@@ -49,52 +49,59 @@ def test_linear_bf16(M_, N, K, swap, splits):
     assert rel_l2(got, ref) < 2e-6
 
 
-# CTA pairs: two CTAs of a cluster share each M = 256 tensor-core MMA, each
-# holding its own 128 rows of X and half of the 256 rows of W; `ctas` =
-# persistent CTAs (two per stream-K unit).
+# Cluster forms of the 256-wide video tiles: mode 1, CTA pairs sharing each
+# M = 256 tensor-core MMA (each CTA its own 128 rows of X and half of the 256
+# rows of W); mode 2, single-CTA tiles in clusters of two, a tile split
+# between the two CTAs of a cluster finished in column halves.  `ctas` =
+# persistent CTAs.
 @pytest.mark.parametrize("M_,N,K,ctas", [
-    (1088, 1536, 6144, 108),  # FFN-down shape: 5 pair rows (the last pair's rank 1 entirely past M), stream-K
+    (1088, 1536, 6144, 108),  # FFN-down shape: 5 pair rows (the last pair's rank 1 past M) / 54 tiles split in two
     (1088, 4608, 1536, 90),   # QKV shape: two whole tiles per pair
     (1088, 1536, 1536, 0),    # out-projection shape on all SMs
     (200, 512, 256, 2),       # one pair walks every tile; M ends inside rank 1's rows
     (64, 256, 64, 0),         # one k-block in all; rank 1 has no valid row
-    (300, 768, 512, 14),      # 7 pairs: pieces of uneven length, split tiles
+    (300, 768, 512, 14),      # 7 pairs: pieces of uneven length, split tiles across clusters
+    (1088, 1536, 1536, 108),  # out-projection shape, every tile split between the CTAs of one cluster
 ])
-def test_linear_cta_pairs(M_, N, K, ctas):
+def test_linear_cluster_forms(M_, N, K, ctas):
     rng = np.random.default_rng(M_ + N + K + ctas)
     x = round_bf16(rng.standard_normal((M_, K)).astype(np.float32))
     w = round_bf16((0.05 * rng.standard_normal((N, K))).astype(np.float32))
     b = rng.standard_normal(N).astype(np.float32)
     ref = x.astype(np.float64) @ w.astype(np.float64).T + b
     outs = []
-    for pair in (True, False):
+    for mode in (1, 2, 0):
         out = torch.full((M_, N), float("nan"), device=DEV)
-        W.op_linear_tiled(_bf16(x), _bf16(w), _f32(b), out, M_, N, K, bn=256, pair=pair, ctas=ctas)
+        W.op_linear_tiled(_bf16(x), _bf16(w), _f32(b), out, M_, N, K, bn=256, mode=mode, ctas=ctas)
         torch.cuda.synchronize()
         got = out.cpu().numpy()
         assert np.isfinite(got).all()
         # fp32 accumulation of K bf16 products against the exact sum
         assert rel_l2(got, ref) < 4e-6
         outs.append(got)
-    # the pair and single-CTA forms split k differently: agreement to rounding
-    assert rel_l2(outs[0], outs[1]) < 4e-6
+    # the three forms split k differently: agreement to rounding
+    assert rel_l2(outs[0], outs[2]) < 4e-6
+    # the cluster split and the global split-tile reduction add the same
+    # pieces on the same stream-K split: the same bits
+    assert np.array_equal(outs[1], outs[2])
 
 
-def test_linear_cta_pairs_repeatable():
-    """The same launch twice gives the same bits (fixed split points and
-    fixed-order partial sums, whatever the timing of the pairs)."""
+def test_linear_cluster_forms_repeatable():
+    """The same launch three times gives the same bits (fixed split points and
+    fixed-order partial sums, whatever the timing of the clusters)."""
     M_, N, K = 1088, 1536, 6144
     rng = np.random.default_rng(5)
     x = _bf16(round_bf16(rng.standard_normal((M_, K)).astype(np.float32)))
     w = _bf16(round_bf16((0.05 * rng.standard_normal((N, K))).astype(np.float32)))
     b = _f32(rng.standard_normal(N).astype(np.float32))
-    outs = []
-    for _ in range(3):
-        out = torch.empty((M_, N), device=DEV)
-        W.op_linear_tiled(x, w, b, out, M_, N, K, bn=256, pair=True, ctas=108)
-        outs.append(out)
-    torch.cuda.synchronize()
-    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    for mode in (1, 2):
+        outs = []
+        for _ in range(3):
+            out = torch.empty((M_, N), device=DEV)
+            W.op_linear_tiled(x, w, b, out, M_, N, K, bn=256, mode=mode, ctas=108)
+            outs.append(out)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
 
 # Joint action attention: (sample, head) split over a cluster of CTAs.
