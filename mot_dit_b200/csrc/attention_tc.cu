@@ -124,6 +124,10 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+}  // namespace
+WAM_KTRACE_UNIT(attn)
+namespace {
+
 struct AttnTcK {
   int H, Lq, Lk, B;
   int zq0, zk0, zv0;  // z (matrix) index of (b=0, h=0) in the Q / K / V maps
@@ -134,6 +138,7 @@ struct AttnTcK {
 __global__ void __launch_bounds__(kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const AttnTcK a) {
+  WAM_KT_BEGIN;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The 128-byte swizzle pattern is a function of the address bits: every tile
   // must start on a 1024-byte boundary.
@@ -192,6 +197,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 0) {
     if (lane == 0) {
       pdl_wait();
+      WAM_KT_WAITED();
       mbar_arrive_expect_tx(q_full, kQBytes);
       tma_load_3d(sQ, &map_q, q_full, 0, q0, a.zq0 + bh);
       int issued = 0;
@@ -400,6 +406,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  WAM_KT_END(attn, 1u);
 }
 
 }  // namespace

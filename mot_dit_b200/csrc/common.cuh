@@ -227,6 +227,51 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ------------------------------------------------ diagnostic kernel trace --
+// Builds with -DWAM_KTRACE only: WAM_KTRACE_UNIT(name) in a .cu file gives it
+// a record buffer and an extern "C" reader wam_debug_ktrace_<name>; the
+// kernels there note their entry time (WAM_KT_BEGIN) and have thread 0 of
+// every CTA append (kind, grid, block, SM, entry, exit) at its end (WAM_KT_END).
+#ifdef WAM_KTRACE
+struct KtRec {
+  unsigned long long t0, t1;
+  unsigned kind, grid_x, grid_y, block, smid, waited;  // waited: ns from entry to the dependent-launch wait's return
+};
+constexpr unsigned kKtMax = 1u << 18;
+#define WAM_KTRACE_UNIT(name)                                                                           \
+  __device__ KtRec g_kt_##name[kKtMax];                                                                 \
+  __device__ unsigned g_kt_n_##name;                                                                    \
+  __device__ __forceinline__ void kt_end_##name(unsigned long long t0, unsigned long long tw, unsigned kind) { \
+    if (threadIdx.x != 0) return;                                                                        \
+    const unsigned i = atomicAdd(&g_kt_n_##name, 1u);                                                    \
+    if (i >= kKtMax) return;                                                                             \
+    unsigned sm;                                                                                         \
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));                                                      \
+    g_kt_##name[i] = KtRec{t0, globaltimer(), kind, gridDim.x, gridDim.y, blockIdx.x + 65536u * blockIdx.y, sm, \
+                           (unsigned)(tw > t0 ? tw - t0 : 0)};                                           \
+  }                                                                                                      \
+  extern "C" int wam_debug_ktrace_##name(void* host, int cap) {                                          \
+    unsigned n = 0;                                                                                      \
+    if (cudaMemcpyFromSymbol(&n, g_kt_n_##name, 4) != cudaSuccess) return -1;                            \
+    if (n > kKtMax) n = kKtMax;                                                                          \
+    if ((int)n > cap) n = cap;                                                                           \
+    if (n && cudaMemcpyFromSymbol(host, g_kt_##name, n * sizeof(KtRec)) != cudaSuccess) return -1;       \
+    const unsigned z = 0;                                                                                \
+    cudaMemcpyToSymbol(g_kt_n_##name, &z, 4);                                                            \
+    return (int)n;                                                                                       \
+  }
+#define WAM_KT_BEGIN                            \
+  const unsigned long long kt_t0 = globaltimer(); \
+  unsigned long long kt_tw = 0
+#define WAM_KT_WAITED() (kt_tw = globaltimer())
+#define WAM_KT_END(name, kind) kt_end_##name(kt_t0, kt_tw, (kind))
+#else
+#define WAM_KTRACE_UNIT(name)
+#define WAM_KT_BEGIN
+#define WAM_KT_WAITED()
+#define WAM_KT_END(name, kind)
+#endif
+
 // ------------------------------------------------- norm + modulation -------
 // One row, one warp: h = rms(x) * (gain ? gain[n] : 1 + scale[n]) + (shift ?
 // shift[n] : 0), rms(x) = x / sqrt(mean(x^2) + 1e-6).  A lane holds up to
@@ -235,40 +280,38 @@ __device__ __forceinline__ void cp_async_wait() {
 // that normalises a row calls this, so all of them round alike.
 constexpr int kRowNormV = 12;
 
-template <bool BF16>
-__device__ __forceinline__ void norm_mod_row(const float* __restrict__ x, void* __restrict__ h, int d,
-                                             const float* __restrict__ scale, const float* __restrict__ shift,
-                                             const float* __restrict__ gain, int lane) {
+// The row's values (every load issued before any is used).
+__device__ __forceinline__ void norm_row_load(const float* __restrict__ x, int d, int lane, float4 (&v)[kRowNormV]) {
   const float4* xr = reinterpret_cast<const float4*>(x);
   const int n4 = d >> 2;
-  float4 v[kRowNormV];
-  float ss = 0.f;
 #pragma unroll
   for (int k = 0; k < kRowNormV; ++k) {
     const int i = lane + 32 * k;
     v[k] = i < n4 ? xr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+}
+// 1 / rms of the row (lane partial sums in k order, then a xor-shuffle tree).
+__device__ __forceinline__ float norm_row_rscale(const float4 (&v)[kRowNormV], int d) {
+  float ss = 0.f;
 #pragma unroll
   for (int k = 0; k < kRowNormV; ++k) ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float r = 1.0f / sqrtf(ss / (float)d + 1e-6f);
+  return 1.0f / sqrtf(ss / (float)d + 1e-6f);
+}
+// h = v * r * mul + add, with mul / add the modulation's float4 i (mul
+// already 1 + scale, or the gain).
+template <bool BF16, typename MulAdd>
+__device__ __forceinline__ void norm_row_store(const float4 (&v)[kRowNormV], float r, int d, int lane, void* __restrict__ h,
+                                               MulAdd mul_add) {
+  const int n4 = d >> 2;
 #pragma unroll
   for (int k = 0; k < kRowNormV; ++k) {
     const int i = lane + 32 * k;
     if (i >= n4) break;
+    float4 mul4, add4;
+    mul_add(i, mul4, add4);
     float y[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-    float4 mul4, add4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (gain) {
-      mul4 = __ldg(reinterpret_cast<const float4*>(gain) + i);
-    } else {
-      mul4 = __ldg(reinterpret_cast<const float4*>(scale) + i);
-      mul4.x += 1.f;
-      mul4.y += 1.f;
-      mul4.z += 1.f;
-      mul4.w += 1.f;
-    }
-    if (shift) add4 = __ldg(reinterpret_cast<const float4*>(shift) + i);
     y[0] = y[0] * r * mul4.x + add4.x;
     y[1] = y[1] * r * mul4.y + add4.y;
     y[2] = y[2] * r * mul4.z + add4.z;
@@ -282,6 +325,30 @@ __device__ __forceinline__ void norm_mod_row(const float* __restrict__ x, void* 
       reinterpret_cast<float4*>(h)[i] = make_float4(y[0], y[1], y[2], y[3]);
     }
   }
+}
+// The modulation's float4 i: (gain or 1 + scale, shift or 0).
+__device__ __forceinline__ void norm_mod_vec(const float* __restrict__ scale, const float* __restrict__ shift,
+                                             const float* __restrict__ gain, int i, float4& mul4, float4& add4) {
+  if (gain) {
+    mul4 = __ldg(reinterpret_cast<const float4*>(gain) + i);
+  } else {
+    mul4 = __ldg(reinterpret_cast<const float4*>(scale) + i);
+    mul4.x += 1.f;
+    mul4.y += 1.f;
+    mul4.z += 1.f;
+    mul4.w += 1.f;
+  }
+  add4 = shift ? __ldg(reinterpret_cast<const float4*>(shift) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+template <bool BF16>
+__device__ __forceinline__ void norm_mod_row(const float* __restrict__ x, void* __restrict__ h, int d,
+                                             const float* __restrict__ scale, const float* __restrict__ shift,
+                                             const float* __restrict__ gain, int lane) {
+  float4 v[kRowNormV];
+  norm_row_load(x, d, lane, v);
+  const float r = norm_row_rscale(v, d);
+  norm_row_store<BF16>(v, r, d, lane, h, [&](int i, float4& m, float4& a) { norm_mod_vec(scale, shift, gain, i, m, a); });
 }
 
 // GELU, tanh form: 0.5 x (1 + tanh(z)), z = sqrt(2/pi) (x + 0.044715 x^3),

@@ -231,6 +231,10 @@ __device__ unsigned long long g_gemm_tl[1024][16];
 #define WAM_TL(slot, v)
 #endif
 
+}  // namespace
+WAM_KTRACE_UNIT(gemm)
+namespace {
+
 // Failure-path test hook (wam_test_peer_wait): the last piece of a split tile
 // that is its CTA's final segment waits for g_peer_wait_extra more published
 // partials than exist, with the limit g_peer_wait_limit_ns, so that the
@@ -449,6 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap map_o, const __grid_constant__ CUtensorMap map_o2,
                    const GemmK g, const EpiArgs e) {
   using C = TileCfg<BN, SWAP, EPI, PAIR>;
+  WAM_KT_BEGIN;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The 128-byte swizzle is a function of the address bits: every tile must
   // start on a 1024-byte boundary.
@@ -569,6 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // with the fused norm the producer reads weights only: no wait for the previous kernel
         if (!C::kNB) pdl_wait();
+        WAM_KT_WAITED();
         if (!SWAP && e.na_x) {
           // the A operand is written by this launch (norm prologue): every row done
           if (!wait_count(e.na_cnt + 1, g.rows_a, g.status, abort_flag)) *abort_flag = 1;
@@ -1332,6 +1338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_dealloc(tmem, C::kTmemCols);
   }
   if (threadIdx.x == 0) WAM_TL(4, globaltimer());
+  WAM_KT_END(gemm, (unsigned)(BN * 1000 + SWAP * 100 + EPI * 10 + PAIR + 2 * g.csplit));
   if (!SWAP && e.na_x && threadIdx.x == 0) {
     // every CTA is past its rows and its wait once all have counted out here
     __threadfence();

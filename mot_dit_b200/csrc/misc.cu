@@ -16,19 +16,42 @@ namespace {
 
 constexpr int kNormWarps = 16;  // rows per CTA (config-2 chunk 4.09 -> 4.02 ms against 8)
 
+}  // namespace
+WAM_KTRACE_UNIT(misc)
+namespace {
+
 // ------------------------------------------------- norm + modulation -------
 // One warp per row (norm_mod_row, shared with the fused-norm GEMM prologue).
 template <bool BF16>
 __global__ void __launch_bounds__(32 * kNormWarps)
     norm_mod_kernel(const float* __restrict__ x, void* __restrict__ h, int M, int d, const float* __restrict__ scale,
                     const float* __restrict__ shift, const float* __restrict__ gain, int ldh) {
+  // the modulation vectors, shared by every row of the CTA
+  __shared__ float4 s_mul[kRowNormMax / 4];
+  __shared__ float4 s_add[kRowNormMax / 4];
+  WAM_KT_BEGIN;
   pdl_trigger();
   pdl_wait();
+  WAM_KT_WAITED();
   const int row = blockIdx.x * kNormWarps + (threadIdx.x >> 5);
-  if (row >= M) return;
-  norm_mod_row<BF16>(x + (size_t)row * d, BF16 ? (void*)(reinterpret_cast<__nv_bfloat16*>(h) + (size_t)row * ldh)
-                                                : (void*)(reinterpret_cast<float*>(h) + (size_t)row * ldh),
-                     d, scale, shift, gain, threadIdx.x & 31);
+  const int lane = threadIdx.x & 31;
+  const bool has_row = row < M;
+  // one round trip: the row's loads go out first, then the CTA stages the
+  // modulation vectors while they are in flight
+  float4 v[kRowNormV];
+  norm_row_load(x + (size_t)(has_row ? row : 0) * d, d, lane, v);
+  for (int i = threadIdx.x; i < (d >> 2); i += blockDim.x) norm_mod_vec(scale, shift, gain, i, s_mul[i], s_add[i]);
+  __syncthreads();
+  if (!has_row) return;
+  const float r = norm_row_rscale(v, d);
+  norm_row_store<BF16>(v, r, d, lane,
+                       BF16 ? (void*)(reinterpret_cast<__nv_bfloat16*>(h) + (size_t)row * ldh)
+                            : (void*)(reinterpret_cast<float*>(h) + (size_t)row * ldh),
+                       [&](int i, float4& m, float4& a) {
+                         m = s_mul[i];
+                         a = s_add[i];
+                       });
+  WAM_KT_END(misc, 2u);
 }
 
 // ------------------------------------------------ timestep conditioning ----
