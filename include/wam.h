@@ -312,7 +312,7 @@ wam_status wam_op_linear(int dtype, const void* dev_x, const void* dev_w, const 
                          int M, int N, int K, int swap, int splits, void* stream);
 
 /* The same product through the video expert's tile shapes (bf16 only, normal
- * orientation, fp32 out): bn = 128 or 256 output features per CTA tile.
+ * orientation, fp32 out): bn = 128, 192 or 256 output features per CTA tile.
  * mode 0: single CTAs.  mode 1 (bn 256): CTA pairs -- two CTAs of a cluster
  * share each M = 256 tensor-core MMA (the 2-SM form), each holding its own
  * 128 rows of X and half of the 256 rows of W.  mode 2: single-CTA tiles

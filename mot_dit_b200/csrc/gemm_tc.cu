@@ -1514,6 +1514,10 @@ cudaError_t prepare_tc_gemm() {
   WAM_PREP(256, false, kClassStore)
   WAM_PREP(256, false, kClassQkv)
   WAM_PREP(256, false, kClassRes)
+  WAM_PREP(192, false, kClassScalar)
+  WAM_PREP(192, false, kClassStore)
+  WAM_PREP(192, false, kClassQkv)
+  WAM_PREP(192, false, kClassRes)
 #undef WAM_PREP
   if ((e = prepare_one<256, false, kClassStore, true>()) != cudaSuccess) return e;
   if ((e = prepare_one<256, false, kClassRes, true>()) != cudaSuccess) return e;
@@ -1591,6 +1595,7 @@ cudaError_t launch_tc_gemm(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
     switch (t.bn) {
       case 64: return launch_normal<64>(t, e, s);
       case 128: return launch_normal<128>(t, e, s);
+      case 192: return launch_normal<192>(t, e, s);
       case 256: return launch_normal<256>(t, e, s);
     }
   }

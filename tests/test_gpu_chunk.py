@@ -117,6 +117,27 @@ def test_video_cluster_split(monkeypatch, batch):
     check_parity(got, inp, ref_a0, ref_veff, c.dtype)
 
 
+def test_video_qkv_192_wide(monkeypatch):
+    """Six heads (attention width 384): the video QKV runs on 192-wide tiles
+    (18 whole tiles against 15 at 256 wide), the QK-norm / RoPE epilogue
+    takes three heads a tile.  Parity with the oracle, CEWP == sequential,
+    and the 256-wide form agrees to rounding."""
+    c = _mid().replace(batch=1, n_heads=6)
+    inp = inputs(c, 29)
+    monkeypatch.delenv("WAM_VIDEO_QKV_BN", raising=False)
+    wam = W.Wam(c, seed=29)
+    got = run_chunk(wam, inp, S=2, mode=W.CEWP, use_graph=True)
+    assert np.array_equal(run_chunk(wam, inp, S=2, mode=W.SEQUENTIAL, use_graph=False), got)
+    wam.close()
+    ref_a0, ref_veff = oracle_chunk(c, 29, inp, S=2)
+    check_parity(got, inp, ref_a0, ref_veff, c.dtype)
+    monkeypatch.setenv("WAM_VIDEO_QKV_BN", "256")
+    wam = W.Wam(c, seed=29)
+    other = run_chunk(wam, inp, S=2)
+    wam.close()
+    assert rel_l2(inp["noise"] - got, inp["noise"] - other) < 1e-3
+
+
 @pytest.mark.parametrize("pair", ["0", "1"])
 def test_video_fused_norm(monkeypatch, pair):
     """Opt-in fused video norm (WAM_VIDEO_FUSED_NORM=1): the QKV / FFN-up

@@ -86,6 +86,25 @@ def test_linear_cluster_forms(M_, N, K, ctas):
     assert np.array_equal(outs[1], outs[2])
 
 
+@pytest.mark.parametrize("M_,N,K,ctas", [
+    (1088, 4608, 1536, 108),  # the video QKV shape on 192-wide tiles: two whole tiles per CTA
+    (200, 384, 256, 3),       # ragged rows, uneven stream-K pieces
+    (300, 576, 512, 0),       # all SMs: split tiles
+])
+def test_linear_192_wide(M_, N, K, ctas):
+    rng = np.random.default_rng(M_ + N + K)
+    x = round_bf16(rng.standard_normal((M_, K)).astype(np.float32))
+    w = round_bf16((0.05 * rng.standard_normal((N, K))).astype(np.float32))
+    b = rng.standard_normal(N).astype(np.float32)
+    out = torch.full((M_, N), float("nan"), device=DEV)
+    W.op_linear_tiled(_bf16(x), _bf16(w), _f32(b), out, M_, N, K, bn=192, mode=0, ctas=ctas)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    ref = x.astype(np.float64) @ w.astype(np.float64).T + b
+    assert np.isfinite(got).all()
+    assert rel_l2(got, ref) < 4e-6
+
+
 def test_linear_cluster_forms_repeatable():
     """The same launch three times gives the same bits (fixed split points and
     fixed-order partial sums, whatever the timing of the clusters)."""
