@@ -12,9 +12,10 @@
 // of stream g:
 //   S_j  = Q K_j^T      tcgen05.mma M=128 N=64 K=64, fp32 into TMEM S_g
 //   P_j  = exp2(S_j log2e / 8 - m_g)   thread = query row (64 keys), bf16
-//          into the 128B-swizzled K-major P_g tile (fence.proxy.async)
-//   O_g += P_j V_j      tcgen05.mma M=128 N=64 K=64 accumulating in TMEM, V
-//          as the MN-major B operand (the cache rows are [key][64 channels])
+//          pairs written back over the first 32 columns of S_g (tcgen05.st)
+//   O_g += P_j V_j      tcgen05.mma M=128 N=64 K=64 accumulating in TMEM, P
+//          as the A operand straight from TMEM, V as the MN-major B operand
+//          from shared memory (the cache rows are [key][64 channels])
 // m_g is raised (and O_g and the row sum rescaled in place) only when a tile's
 // maximum exceeds it by more than 2^8: exact softmax arithmetic with a stale
 // maximum, P <= 256, and in most tiles no TMEM round trip of O.  The MMA warp
@@ -38,13 +39,13 @@ constexpr int kDh = 64;
 constexpr int kStagesKV = 4;
 constexpr int kQBytes = kQ * kDh * 2;      // 16 KB
 constexpr int kKVBytes = kKT * kDh * 2;    // 8 KB (one K or V tile)
-constexpr int kPBytes = kQ * kKT * 2;      // 16 KB (one P tile)
+constexpr int kXchBytes = 3 * kQ * 4;      // stream 1's (m, l, ok) per row for the final merge
 constexpr int kThreads = 320;              // producer, MMA, two softmax warpgroups
 constexpr int kTmemCols = 256;             // S_0 [0,64), S_1 [64,128), O_0 [128,192), O_1 [192,256)
 constexpr float kRescale = 8.0f;           // log2 headroom of the stale row maximum
 constexpr int kBarBytes = 128;
 // No alignment slack: two CTAs per SM need every byte (2 x (112 KB + 1 KB reserved) <= 228 KB).
-constexpr int kSmem = kQBytes + kStagesKV * 2 * kKVBytes + 2 * kPBytes + kBarBytes;
+constexpr int kSmem = kQBytes + kStagesKV * 2 * kKVBytes + kXchBytes + kBarBytes;
 
 // Shared-memory descriptor of an MN-major bf16 operand stored as rows of 128
 // bytes (64 elements along N) with the 128-byte swizzle, consecutive K rows
@@ -63,8 +64,30 @@ __device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+// 32 lanes x 32 consecutive 32-bit columns from registers, one wait.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]: the A operand (M = 128 rows on the TMEM
+// lanes, K-major, two 16-bit elements per 32-bit column) read from tensor memory.
+__device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // 32 lanes x 64 consecutive 32-bit columns, one wait.
@@ -149,8 +172,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* sQ = smem_raw;
   uint8_t* sK = sQ + kQBytes;                  // [stage] K tiles
   uint8_t* sV = sK + kStagesKV * kKVBytes;     // [stage] V tiles
-  uint8_t* sP = sV + kStagesKV * kKVBytes;     // [stream] P tiles [128][128 B]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sP + 2 * kPBytes);
+  float* xch = reinterpret_cast<float*>(sV + kStagesKV * kKVBytes);  // [128] m_1, [128] l_1, [128] ok_1
+  uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xch) + kXchBytes);
   uint64_t* q_full = bar + 0;
   uint64_t* kv_full = bar + 1;   // [4]
   uint64_t* kv_empty = bar + 5;  // [4]
@@ -242,11 +265,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!mbar_wait(&p_full[g], t & 1, a.status, kStatusTimeoutAccum, abort_flag)) break;
         tc_fence_after();
         const int s = j % kStagesKV;
-        const uint32_t ap = smem_u32(sP + g * kPBytes), av = smem_u32(sV + s * kKVBytes);
+        const uint32_t av = smem_u32(sV + s * kKVBytes);
+        // P_j sits in the first 32 columns of S_g (16 keys = 8 columns a step);
+        // S_{j+2}, issued after this, overwrites it only once these have read it
 #pragma unroll
         for (int kk = 0; kk < kKT / 16; ++kk)
-          tc_mma_bf16(tmem + 128 + g * kDh, smem_desc_k128(ap + kk * 32), smem_desc_mn128(av + kk * 16 * 128),
-                      idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_bf16_ts(tmem + 128 + g * kDh, tmem + g * kKT + kk * 8, smem_desc_mn128(av + kk * 16 * 128),
+                         idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&pv_full[g]);
         tc_commit(&kv_empty[s]);  // K_j and V_j are read
         if (j + 2 < ntiles && !issue_s(j + 2)) break;
@@ -263,8 +288,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t t_s = t_lane + g * kKT, t_o = t_lane + 128 + g * kDh;
     const float sl2e = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
     float mref = -INFINITY, l = 0.f;  // reference maximum (scaled log2 units) and row sum of the stream
-    uint8_t* prow = sP + g * kPBytes + r * 128;
-    const int swz = r & 7;
     bool ok = true;
     int t = 0;
     for (int j = g; j < ntiles; j += 2, ++t) {
@@ -327,28 +350,23 @@ __global__ void __launch_bounds__(kThreads, 2)
           rs += v[i];
         }
       }
+      {
+        uint32_t pw[32];  // P as bf16 pairs, key 2c in the low half of column c
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        uint4 w;
-        w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-        w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-        w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-        w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-        *reinterpret_cast<uint4*>(prow + ((q ^ swz) << 4)) = w;
+        for (int c2 = 0; c2 < 32; ++c2) pw[c2] = pack_bf16(v[2 * c2], v[2 * c2 + 1]);
+        tmem_st32(t_s, pw);  // over S_j, already read into registers
       }
       l += rs;
       tc_fence_before();
-      fence_proxy_async_smem();  // P (generic-proxy stores) -> tensor-core reads
       mbar_arrive_cta(&p_full[g]);
     }
-    // The stream's last PV; then stream 1 hands (m, l) over in the idle P_1
-    // tile and stream 0 merges: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) /
+    // The stream's last PV; then stream 1 hands (m, l) over in shared memory
+    // and stream 0 merges: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) /
     // (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)), M = max(m_0, m_1).
     const int nt = (ntiles - g + 1) / 2;  // tiles of this stream
     if (ok && nt > 0) ok = mbar_wait(&pv_full[g], (nt - 1) & 1, a.status, kStatusTimeoutAccum, abort_flag);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
-    float* xch = reinterpret_cast<float*>(sP + kPBytes);  // [128] m_1, [128] l_1, [128] ok_1
     if (g == 1) {
       xch[r] = nt > 0 ? mref : -INFINITY;
       xch[kQ + r] = l;
