@@ -320,8 +320,13 @@ wam_status wam_op_linear(int dtype, const void* dev_x, const void* dev_w, const 
  * gives to the two CTAs of one cluster is finished in column halves, each
  * CTA's half-partial of the other's columns crossing in shared memory.
  * ctas = persistent CTAs (0: one per SM; even for mode 2, rounded down to
- * pairs for mode 1).  K a multiple of 64, N a multiple of 32.  Returns
- * WAM_ERR_INVALID_ARG for other shapes or values. */
+ * pairs for mode 1).  K a multiple of 64, N a multiple of 32.
+ * mode 3: the swapped orientation of the action expert (M <= 64 token rows
+ * as the MMA's N operand, bn ignored), each 128-feature tile split over
+ * ctas = 2..8 CTAs of one cluster, one equal k-range each (K / 64 a multiple
+ * of ctas, and 32 (M <= 32) or 64 a multiple of 4 ctas); the pieces are summed
+ * in rank (= k) order in shared memory, each CTA finishing its share of the
+ * token columns.  Returns WAM_ERR_INVALID_ARG for other shapes or values. */
 wam_status wam_op_linear_tiled(const void* dev_x, const void* dev_w, const float* dev_bias, float* dev_out, int M,
                                int N, int K, int bn, int mode, int ctas, void* stream);
 

@@ -323,7 +323,8 @@ def op_linear(dtype, x, w, bias, out, M, N, K, swap=False, splits=1, stream=None
 
 
 def op_linear_tiled(x, w, bias, out, M, N, K, bn=256, mode=1, ctas=0, stream=None):
-    """mode 0: single CTAs; 1: CTA pairs (2-SM MMA); 2: clusters of two, split tiles finished in halves."""
+    """mode 0: single CTAs; 1: CTA pairs (2-SM MMA); 2: clusters of two, split tiles finished in halves;
+    3: swapped (M <= 64 tokens), each tile split over a cluster of `ctas` CTAs summed in shared memory."""
     st = lib().wam_op_linear_tiled(_ptr(x), _ptr(w), _ptr(bias), _ptr(out), M, N, K, bn, int(mode), ctas,
                                    _stream(stream))
     if st:

@@ -23,6 +23,7 @@
 #include "kernels.h"
 
 namespace wam {
+WAM_KTRACE_UNIT(jattn)
 namespace {
 
 constexpr int kD = 64;      // head dim of the bf16 path
@@ -388,6 +389,7 @@ __host__ __device__ constexpr bool joint_fits(int splits, int Lq) { return (size
 __global__ void __launch_bounds__(kJThreads, 1)
     attn_joint_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                       const AttnJointK a) {
+  WAM_KT_BEGIN;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // TMA's 128-byte swizzle is a function of the address bits (tile bases on
   // 1024-byte boundaries); every CTA of the cluster sees the same layout
@@ -433,6 +435,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
   if (tid == 0)  // tiles of keys complete before the launch
     while (issued < first && min(k_end, k_begin + (issued + 1) * kTK) <= a.ready) issue(issued++);
   pdl_wait();  // the queries and the action rows are the previous kernel's
+  WAM_KT_WAITED();
   if (tid == 0)
     while (issued < first) issue(issued++);
   const __nv_bfloat16* qb = a.q + (size_t)bh * a.Lq * kD;
@@ -614,6 +617,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
           *reinterpret_cast<uint32_t*>(dst + nt * 8 + 2 * t4) = pack_bf16(o[nt][2 * r] * inv, o[nt][2 * r + 1] * inv);
       }
     }
+    WAM_KT_END(jattn, 3u);
     return;
   }
   // partial of this split -> rank 0's shared memory, once every CTA of the
@@ -632,7 +636,10 @@ __global__ void __launch_bounds__(kJThreads, 1)
     }
   }
   jt_cluster_sync();  // every partial is in rank 0's shared memory
-  if (split != 0) return;
+  if (split != 0) {
+    WAM_KT_END(jattn, 3u);
+    return;
+  }
   // merge in split order: M = max_s m_s, f_s = 2^((m_s - M) c) / sum_s 2^((m_s - M) c) l_s
   if (tid < a.Lq) {
     float M = -INFINITY;
@@ -663,6 +670,7 @@ __global__ void __launch_bounds__(kJThreads, 1)
     w.y = pack_bf16(acc.z, acc.w);
     *reinterpret_cast<uint2*>(a.out + (size_t)(b * a.Lq + row) * a.ld_out + h * kD + 4 * c4) = w;
   }
+  WAM_KT_END(jattn, 3u);
 }
 
 }  // namespace

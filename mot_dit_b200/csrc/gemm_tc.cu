@@ -113,6 +113,8 @@ struct GemmK {
   int* tickets;  // [tiles][2]: pieces arrived, pieces published
   unsigned* status;
   int csplit;    // launched as clusters of two CTAs: a tile split between them is finished in halves
+  int cred;      // swapped: launched as clusters of cred CTAs, each tile's pieces one cluster (one
+                 // equal k-range per CTA), summed in shared memory: each CTA finishes BN / cred columns
 };
 
 // First k-block of CTA c, and the CTA owning k-block x (the largest c with
@@ -165,6 +167,13 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// A liveness point split in two: each thread arrives when it is done with
+// the other CTAs of the cluster (no memory ordering), and waits before it
+// exits until every thread of the cluster has arrived.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait;" ::: "memory"); }
 // Address, in the cluster's shared window, of the same object in CTA `rank`.
 __device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
   uint32_t a;
@@ -173,6 +182,9 @@ __device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
 // Bulk copy of `bytes` from this CTA's shared memory to cluster address `dst`
 // (another CTA of the cluster), completing on the barrier at cluster address
@@ -246,6 +258,9 @@ __device__ unsigned long long g_peer_wait_limit_ns = kWaitLimitNs;
 // Bounded wait until *count >= target (a counter other CTAs increment).
 __device__ __forceinline__ bool wait_count(const int* count, int target, unsigned* status, volatile int* abort,
                                            unsigned long long limit_ns = kWaitLimitNs) {
+  // One polling thread (the rest of its CTA waits at a barrier); each poll is
+  // an L2 round trip, so no sleep between polls: a __nanosleep here delayed
+  // the split-tile reducer by ~1.7 us after the last partner had published.
   const volatile int* vc = count;
   const unsigned long long t0 = globaltimer();
   while (*vc < target) {
@@ -254,7 +269,6 @@ __device__ __forceinline__ bool wait_count(const int* count, int target, unsigne
       atomicOr(status, kStatusTimeoutPeer);
       return false;
     }
-    __nanosleep(32);
   }
   return true;
 }
@@ -481,8 +495,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acce = accf + 2;            // [2] accumulator drained (epilogue -> MMA)
   uint64_t* redb = acce + 2;            // partial tiles copied into the ring
   uint64_t* bready = redb + 1;          // fused-norm B operand written (epilogue warps -> MMA)
-  uint64_t* peer_idle = bready + 1;     // cluster split: the partner's ring may take my half-partial
-  uint64_t* peer_data = peer_idle + 1;  // cluster split: the partner's half-partial is in my ring
+  uint64_t* peer_idle = bready + 1;     // cluster split / reduce: the partners' rings may take my partials
+  uint64_t* peer_data = peer_idle + 1;  // cluster split / reduce: the partners' partials are in my ring
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(peer_data + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -492,6 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // segments; rank 1 takes the odd 128-row tile of each 256-row pair tile).
   const uint32_t rank = PAIR ? cluster_rank() : 0u;
   const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  bool cl_arrived = false;  // cluster reduce: this thread has arrived at the exit barrier
   const long long x_begin = kbound(g, unit), x_end = kbound(g, unit + 1);
 
   if (threadIdx.x == 0) {
@@ -509,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(redb, 1);
     mbar_init(bready, 1);
-    mbar_init(peer_idle, 1);
+    mbar_init(peer_idle, g.cred > 1 ? g.cred - 1 : 1);
     mbar_init(peer_data, 1);
     *abort_flag = 0;
     *last_flag = 0;
@@ -533,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if constexpr (PAIR) cluster_sync();  // the peer's barriers exist before any remote arrival
-  if (!PAIR && g.csplit) cluster_sync();  // (the same for the cluster split; g is uniform)
+  if (!PAIR && (g.csplit || g.cred > 1)) cluster_sync();  // (the same for the cluster split / reduce; g is uniform)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_trigger();  // the next kernel may start its own set-up now
@@ -806,6 +821,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                       (c_first & 1) == 0 && kbound(g, c_first) == t0 && kbound(g, c_first + 2) == t0 + g.KB;
       const int c_lo = cs ? (unit - c_first) * (BN / 2) : 0;
       const int c_hi = cs ? c_lo + BN / 2 : BN;
+      // A swapped tile whose g.cred pieces are exactly the CTAs of one cluster
+      // (each CTA one whole equal k-range): CTA rank rk finishes token columns
+      // [rk cw, rk cw + cw), the other pieces' slices of them arriving in its
+      // idle ring through the cluster's shared window.  Decided alike by all.
+      const bool cr = SWAP && !PAIR && g.cred > 1 && npieces == g.cred && c_first % g.cred == 0 &&
+                      kbound(g, c_first) == t0 && kbound(g, c_first + g.cred) == t0 + g.KB;
+      const int cw = cr ? BN / g.cred : BN, rk = cr ? unit - c_first : 0;
+      // swapped: this thread's feature's bias and gate, and for a cluster
+      // reduction with a gate-residual its residual values (when it finishes
+      // at most 16 columns), requested now so that they arrive while the
+      // MMAs run
+      const int n_sw = ta * BM + row;
+      const bool n_sw_ok = SWAP && n_sw < g.rows_a;
+      const float bias_sw = n_sw_ok ? __ldg(R.bias + n_sw) : 0.f;
+      const float gate_sw = (n_sw_ok && R.gate) ? __ldg(R.gate + n_sw) : 0.f;
+      float xo_cr[16];
+      const bool xo_pf = cr && n_sw_ok && R.kind == kEpiGateRes && cw <= 16;
+      if (xo_pf) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int m = tb * BN + rk * cw + k;
+          xo_cr[k] = k < cw && m < g.rows_b ? R.out_f32[(size_t)m * R.ld + n_sw] : 0.f;
+        }
+      }
       const int m0w = arow(ta) + quad * 32;  // normal orientation: this warp's first row
       const int tk = PAIR ? 2 * t + (int)rank : t;  // the tickets of this CTA's 128-row tile
       const int nb = tb * BN;
@@ -934,12 +973,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (threadIdx.x == 64 && x == x_end) WAM_TL(6, globaltimer());  // exchange done
         if (*abort_flag) break;
       }
+      if (cr) {
+        // My ring is idle (my one piece's MMAs are done, nothing in flight).
+        // Its front holds every piece's slice of my columns, [src rank][4-
+        // column chunk][row] float4: mine written here, the others' arriving
+        // by bulk copy; behind it I stage my slices of the others' columns the
+        // same way, one contiguous block per destination.
+        const int S = g.cred, nq = cw / 4;
+        const uint32_t slice = (uint32_t)BM * cw * 4;
+        uint8_t* stage = smem + (size_t)S * slice;
+        // epilogue thread tt < S - 1 deals with partner q(tt): tells it my ring
+        // is idle, later sends it my slice of its columns
+        const int tt = threadIdx.x - 64, qt = tt < rk ? tt : tt + 1;
+        if (threadIdx.x == 64) mbar_arrive_expect_tx(peer_data, (S - 1) * slice);  // what the others will send
+        // (relaxed: nothing to publish -- my MMAs' reads of the ring completed
+        // before the accumulator was reported ready)
+        if (tt < S - 1) mbar_arrive_cluster_relaxed(cluster_addr(peer_idle, (uint32_t)qt));  // qt may send now
+        for (int c = 0; c < BN; c += 32) {
+          float v[32];
+          tmem_ld32(t_row + c, v);
+#pragma unroll
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const int col = c + 4 * i4, q = col / cw, qq = (col % cw) >> 2;
+            uint8_t* dst = q == rk ? smem + ((size_t)(rk * nq + qq) * BM + row) * 16
+                                   : stage + ((size_t)((q < rk ? q : q - 1) * nq + qq) * BM + row) * 16;
+            *reinterpret_cast<float4*>(dst) = make_float4(v[4 * i4], v[4 * i4 + 1], v[4 * i4 + 2], v[4 * i4 + 3]);
+          }
+        }
+        release();  // the accumulator is in shared memory now
+        fence_proxy_async_smem();  // generic writes -> the bulk copies
+        epi_bar();
+        if (threadIdx.x == 64 && x == x_end) WAM_TL(10, globaltimer());  // staged
+        if (tt < S - 1) {
+          if (!mbar_wait(peer_idle, 0, g.status, kStatusTimeoutPeer, abort_flag)) {
+            *abort_flag = 1;
+          } else {
+            if (tt == 0 && x == x_end) WAM_TL(11, globaltimer());  // every partner's ring idle
+            // my slice of qt's columns (stage slot tt) into qt's ring at my rank's slot
+            bulk_copy_to_peer(cluster_addr(smem + (size_t)rk * slice, (uint32_t)qt), stage + (size_t)tt * slice, slice,
+                              cluster_addr(peer_data, (uint32_t)qt));
+            bulk_commit();
+            if (tt == 0 && x == x_end) WAM_TL(12, globaltimer());  // copy issued
+          }
+        }
+        if (!mbar_wait(peer_data, 0, g.status, kStatusTimeoutPeer, abort_flag)) *abort_flag = 1;
+        if (threadIdx.x == 64 && x == x_end) WAM_TL(13, globaltimer());  // every partner's slice arrived
+        if (tt < S - 1) bulk_wait_read<0>();  // my staging has been read out
+        // done with the other CTAs (their slices are here, mine are read out)
+        if (!cl_arrived) cluster_arrive_relaxed();
+        cl_arrived = true;
+        epi_bar();
+        if (threadIdx.x == 64 && x == x_end) WAM_TL(6, globaltimer());  // exchange done
+        if (*abort_flag) break;
+      }
       // ---- a tile shared with other CTAs (see "Split tiles" above)
       const int mine = unit - c_first;  // this CTA's piece of tile t
       // CTA holding piece p's partial (the same rank of the piece's pair)
       auto piece_cta = [&](int p) { return PAIR ? 2 * (c_first + p) + (int)rank : c_first + p; };
       bool from_smem = false;
-      if (npieces > 1 && !cs) {
+      if (npieces > 1 && !cs && !cr) {
         if (threadIdx.x == 64) {
           const int prev = atomicAdd(g.tickets + 2 * tk, 1);
           *last_flag = (prev == npieces - 1) ? 1 : 0;
@@ -1237,9 +1329,81 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = ta * BM + row;
         const int mb = tb * BN;
         const bool n_ok = n < g.rows_a;
-        const float bias = n_ok ? __ldg(R.bias + n) : 0.f;
-        const float gate = (n_ok && R.gate) ? __ldg(R.gate + n) : 0.f;
-        for (int c = 0; c < BN; c += 32) {
+        const float bias = bias_sw, gate = gate_sw;
+        if (cr && R.kind == kEpiQkv) {
+          // my token columns summed in rank order, staged [token][128 features
+          // + 1], then (token, head) items as in the whole-tile path below
+          const float4* rv = reinterpret_cast<const float4*>(smem);
+          float* stage = reinterpret_cast<float*>(sStg);
+          epi_bar();  // (the stage's previous readers are done)
+#pragma unroll
+          for (int qq = 0; qq < 8; ++qq) {
+            if (qq >= cw / 4) break;
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int p = 0; p < g.cred; ++p) {
+              const float4 t4 = rv[(size_t)(p * (cw / 4) + qq) * BM + row];
+              a.x += t4.x;
+              a.y += t4.y;
+              a.z += t4.z;
+              a.w += t4.w;
+            }
+            stage[(4 * qq + 0) * (BM + 1) + row] = a.x + bias;
+            stage[(4 * qq + 1) * (BM + 1) + row] = a.y + bias;
+            stage[(4 * qq + 2) * (BM + 1) + row] = a.z + bias;
+            stage[(4 * qq + 3) * (BM + 1) + row] = a.w + bias;
+          }
+          epi_bar();
+          const int tt = threadIdx.x - 64;
+          if (tt < 2 * cw) {
+            const int j = tt % cw, hh = tt / cw;
+            const int m = mb + rk * cw + j;
+            const int n0 = ta * BM + hh * 64;
+            if (m < g.rows_b && n0 < g.rows_a) {
+              float xv[64];
+#pragma unroll
+              for (int k = 0; k < 64; ++k) xv[k] = stage[j * (BM + 1) + hh * 64 + k];
+              const int section = n0 / R.attn_dim, head = (n0 % R.attn_dim) / 64;
+              qk_norm_rope(R, section, head, m, xv, nullptr, nullptr, 0);
+              store_head(qkv_dst(R, section, head, m), xv);
+            }
+          }
+        } else if (cr) {
+          // my token columns [rk cw, rk cw + cw): every piece's slice of them,
+          // summed in rank (= k) order, 4 columns at a time
+          const float4* rv = reinterpret_cast<const float4*>(smem);
+#pragma unroll
+          for (int qq = 0; qq < 8; ++qq) {  // cw = BN / cred <= 32
+            if (qq >= cw / 4) break;
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int p = 0; p < g.cred; ++p) {
+              const float4 t4 = rv[(size_t)(p * (cw / 4) + qq) * BM + row];
+              a.x += t4.x;
+              a.y += t4.y;
+              a.z += t4.z;
+              a.w += t4.w;
+            }
+            if (!n_ok) continue;
+            const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int e4 = 0; e4 < 4; ++e4) {
+              const int m = mb + rk * cw + 4 * qq + e4;
+              if (m >= g.rows_b) continue;
+              const float y = av[e4] + bias;
+              float* o32 = R.out_f32 + (size_t)m * R.ld + n;
+              if (R.kind == kEpiGateRes)
+                *o32 = (xo_pf && qq < 4 ? xo_cr[(4 * qq + e4) & 15] : *o32) + gate * y;
+              else if (R.kind == kEpiStoreF32)
+                *o32 = y;
+              else if (R.kind == kEpiGelu)
+                R.out_act[(size_t)m * R.ld + n] = __float2bfloat16_rn(gelu_tanh(y));
+              else if (R.kind == kEpiScaleAct)
+                R.out_act[(size_t)m * R.ld + n] = __float2bfloat16_rn(e.scale * y);
+              else
+                epi_elem(e, m, n, y, gate);
+            }
+          }
+        }
+        for (int c = 0; c < BN && !cr; c += 32) {
           float v[32];
           get(c, v);
           if (R.kind == kEpiQkv) {
@@ -1310,6 +1474,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 64) WAM_TL(8, globaltimer());
     __syncwarp();
   }
+  // the producer and MMA warps (and any thread not yet arrived) are done with
+  // the other CTAs of the cluster
+  if (!PAIR && g.cred > 1 && !cl_arrived) cluster_arrive_relaxed();
 
   // ------------------------------------------------------------- teardown
   tc_fence_before();
@@ -1328,8 +1495,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
   // A pair stays until both CTAs are done: rank 0's MMAs read the peer's
-  // shared memory, and each CTA arrives on the other's barriers.
+  // shared memory, and each CTA arrives on the other's barriers.  So does a
+  // cluster that reduces in shared memory (no CTA leaves while a partner
+  // might still copy into it, on any path).
   if constexpr (PAIR) cluster_sync();
+  if (!PAIR && g.cred > 1) cluster_wait();
   if (warp == 1) {
     tc_fence_after();
     if constexpr (PAIR)
@@ -1360,18 +1530,19 @@ cudaError_t prepare_one() {
 int g_num_sms = 0;
 int g_max_pairs = 0;  // clusters of two 227 KB CTAs the device holds at once
 
-// Launch as clusters of two CTAs (pairs of SMs), with programmatic dependent
-// launch like launch_k.
+// Launch as clusters of `cluster` CTAs, with programmatic dependent launch
+// like launch_k.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pairs(void (*kernel)(KArgs...), int pairs, size_t smem, cudaStream_t s, Args... args) {
+cudaError_t launch_clusters(void (*kernel)(KArgs...), int cluster, int clusters, size_t smem, cudaStream_t s,
+                            Args... args) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs);
+  cfg.gridDim = dim3(cluster * clusters);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.x = cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1379,6 +1550,11 @@ cudaError_t launch_pairs(void (*kernel)(KArgs...), int pairs, size_t smem, cudaS
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+// Clusters of two CTAs (pairs of SMs).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pairs(void (*kernel)(KArgs...), int pairs, size_t smem, cudaStream_t s, Args... args) {
+  return launch_clusters(kernel, 2, pairs, smem, s, args...);
 }
 
 // Output rows of one tile row (the stream-K tile): 128, or 256 for a pair.
@@ -1426,6 +1602,17 @@ cudaError_t launch_one(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
   g.tickets = t.tickets;
   g.status = t.status;
   g.csplit = (!PAIR && !SWAP && t.csplit && g.G % 2 == 0) ? 1 : 0;
+  g.cred = 0;
+  if (SWAP && !PAIR && t.cred > 1 && t.cred == t.splits) {
+    // one cluster per tile, one equal k-range per CTA, the exchange areas (S
+    // slices in, S - 1 out) fitting the operand ring
+    const int S = t.cred;
+    const long long tiles = (long long)g.tiles_a * ((t.rows_b + BN - 1) / BN);
+    if (S > 8 || g.KB % S != 0 || BN % (4 * S) != 0 || g.G != tiles * S ||
+        (size_t)C::kStages * C::kStageBytes < (size_t)(2 * S - 1) * BM * (BN / S) * 4)
+      return cudaErrorInvalidValue;
+    g.cred = S;
+  }
   // unused output maps are passed as copies of the A map
   const CUtensorMap& mo = e.map_o ? *e.map_o : *t.map_a;
   const CUtensorMap& mo2 = e.map_o2 ? *e.map_o2 : *t.map_a;
@@ -1433,6 +1620,9 @@ cudaError_t launch_one(const TcGemm& t, const EpiArgs& e, cudaStream_t s) {
     return launch_pairs(tc_gemm_kernel<BN, SWAP, EPI, true>, g.G, C::kSmem, s, *t.map_a, *t.map_b, mo, mo2, g, e);
   else if (g.csplit)  // clusters of two CTAs: grid 2 x (G / 2)
     return launch_pairs(tc_gemm_kernel<BN, SWAP, EPI, false>, g.G / 2, C::kSmem, s, *t.map_a, *t.map_b, mo, mo2, g, e);
+  else if (g.cred > 1)  // one cluster of g.cred CTAs per tile
+    return launch_clusters(tc_gemm_kernel<BN, SWAP, EPI, false>, g.cred, (int)(g.G / g.cred), C::kSmem, s, *t.map_a,
+                           *t.map_b, mo, mo2, g, e);
   else
     return launch_k(tc_gemm_kernel<BN, SWAP, EPI, false>, dim3(g.G), dim3(kThreads), C::kSmem, s, *t.map_a, *t.map_b,
                     mo, mo2, g, e);

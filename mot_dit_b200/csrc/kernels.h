@@ -141,6 +141,9 @@ struct TcGemm {
   bool csplit;               // normal, single CTAs: launch as clusters of two (even grid); a tile whose
                              // k-range stream-K splits between the two CTAs of a cluster is finished
                              // in column halves, the partials crossing in shared memory
+  int cred;                  // swapped, splits > 1: launch as clusters of `splits` CTAs (<= 8, dividing
+                             // the k-blocks and bn / 4) when cred == splits; each tile's pieces are then
+                             // summed in shared memory, each CTA finishing bn / splits token columns
   float* ws;                 // partial tiles: 2 * CTAs * 128 * bn floats (tc_gemm_ws_floats)
   int* tickets;              // two per output tile, zero on entry, left zero
   unsigned* status;

@@ -14,16 +14,19 @@
 namespace wam {
 namespace {
 
-constexpr int kNormWarps = 16;  // rows per CTA (config-2 chunk 4.09 -> 4.02 ms against 8)
+constexpr int kNormWarps = 16;      // rows per CTA (config-2 chunk 4.09 -> 4.02 ms against 8)
+constexpr int kNormWarpsSmall = 4;  // rows per CTA up to kNormSmallRows rows, so more SMs share the loads
+constexpr int kNormSmallRows = 256;
 
 }  // namespace
 WAM_KTRACE_UNIT(misc)
 namespace {
 
 // ------------------------------------------------- norm + modulation -------
-// One warp per row (norm_mod_row, shared with the fused-norm GEMM prologue).
-template <bool BF16>
-__global__ void __launch_bounds__(32 * kNormWarps)
+// One warp per row (norm_mod_row, shared with the fused-norm GEMM prologue),
+// WARPS rows per CTA.
+template <bool BF16, int WARPS>
+__global__ void __launch_bounds__(32 * WARPS)
     norm_mod_kernel(const float* __restrict__ x, void* __restrict__ h, int M, int d, const float* __restrict__ scale,
                     const float* __restrict__ shift, const float* __restrict__ gain, int ldh) {
   // the modulation vectors, shared by every row of the CTA
@@ -33,7 +36,7 @@ __global__ void __launch_bounds__(32 * kNormWarps)
   pdl_trigger();
   pdl_wait();
   WAM_KT_WAITED();
-  const int row = blockIdx.x * kNormWarps + (threadIdx.x >> 5);
+  const int row = blockIdx.x * WARPS + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const bool has_row = row < M;
   // one round trip: the row's loads go out first, then the CTA stages the
@@ -288,10 +291,14 @@ cudaError_t launch_norm_mod(const float* x, void* h, bool h_bf16, int M, int d, 
   if (ldh == 0) ldh = d;
   if (ldh < d || ldh % 4) return cudaErrorInvalidValue;
   if (d % 4 != 0 || d > 32 * 4 * kRowNormV) return cudaErrorInvalidValue;
-  dim3 grid((M + kNormWarps - 1) / kNormWarps);
-  if (h_bf16)
-    return launch_k(norm_mod_kernel<true>, grid, dim3(32 * kNormWarps), 0, s, x, h, M, d, scale, shift, gain, ldh);
-  return launch_k(norm_mod_kernel<false>, grid, dim3(32 * kNormWarps), 0, s, x, h, M, d, scale, shift, gain, ldh);
+  if (M <= kNormSmallRows) {
+    const dim3 grid((M + kNormWarpsSmall - 1) / kNormWarpsSmall), block(32 * kNormWarpsSmall);
+    if (h_bf16) return launch_k(norm_mod_kernel<true, kNormWarpsSmall>, grid, block, 0, s, x, h, M, d, scale, shift, gain, ldh);
+    return launch_k(norm_mod_kernel<false, kNormWarpsSmall>, grid, block, 0, s, x, h, M, d, scale, shift, gain, ldh);
+  }
+  const dim3 grid((M + kNormWarps - 1) / kNormWarps), block(32 * kNormWarps);
+  if (h_bf16) return launch_k(norm_mod_kernel<true, kNormWarps>, grid, block, 0, s, x, h, M, d, scale, shift, gain, ldh);
+  return launch_k(norm_mod_kernel<false, kNormWarps>, grid, block, 0, s, x, h, M, d, scale, shift, gain, ldh);
 }
 
 cudaError_t launch_temb(const TembArgs& a, cudaStream_t s) {

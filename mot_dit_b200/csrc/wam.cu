@@ -64,6 +64,7 @@ struct GemmPlan {
   int bn = 128, splits = 1, max_ctas = 0;
   bool pair = false;    // normal orientation, bn 256: CTA pairs (2-SM MMA)
   bool csplit = false;  // normal orientation: clusters of two, split tiles finished in column halves
+  int cred = 0;         // swapped: clusters of `splits` CTAs sum each tile's pieces in shared memory
 };
 
 }  // namespace
@@ -113,6 +114,8 @@ struct wam_ctx {
   // plans
   GemmPlan p_v_qkv, p_v_o, p_v_f1, p_v_f2, p_v_in, p_v_out;
   GemmPlan p_a_in, p_a_qkv, p_a_o, p_a_f1, p_a_f2, p_a_out;
+  // Euler steps j >= 1 (no video kernels beside them): splits over clusters
+  GemmPlan p_a_qkv_l, p_a_o_l, p_a_f1_l, p_a_f2_l;
   GemmPlan p_u_qkv, p_u_o, p_u_f1, p_u_f2;  // LoRA down-projections u = s x A^T
   int attn_splits = 1;
   int attn_joint_splits = 0;  // joint action attention on clusters (0: the split-KV kernel)
@@ -354,7 +357,8 @@ inline void* vcache(wam_ctx* c, int i) {
   } while (0)
 
 // ------------------------------------------------------------- planning ---
-GemmPlan plan_swap(int rows_w, int tokens, int K, int bn, bool fused_norm, int target_ctas) {
+GemmPlan plan_swap(int rows_w, int tokens, int K, int bn, bool fused_norm, int target_ctas, bool cred = false,
+                   int wide_splits = 0) {
   GemmPlan p;
   p.bn = bn;
   const int tiles = ((rows_w + 127) / 128) * ((tokens + bn - 1) / bn);
@@ -363,16 +367,35 @@ GemmPlan plan_swap(int rows_w, int tokens, int K, int bn, bool fused_norm, int t
   const int min_kb = 3;  // keep each split a few k-blocks deep
   if (s > kb / min_kb) s = kb / min_kb;
   // With 24 or more feature tiles the weights already stream from as many
-  // SMs; splitting further only adds the partial-tile hand-off (action QKV /
-  // FFN-up at 32 tokens: 4 splits 16.6 us, none 14.5 us per launch in the
-  // 10-step chunk).
-  if (tiles >= 24) s = 1;
+  // SMs; splits summed through global partials only added the hand-off
+  // (action QKV / FFN-up at 32 tokens: 4 splits 16.6 us, none 14.5 us per
+  // launch in the 10-step chunk), so such a GEMM splits only over clusters
+  // (wide_splits CTAs summing in shared memory), else not at all.
+  if (tiles >= 24) s = cred && wide_splits > 1 ? wide_splits : 1;
   // a tile takes at most splits + 1 pieces; the last one's partner partials
   // must fit its operand ring for the fast reduction
   const int cap = tc_gemm_ring_partials(bn, true, fused_norm);
   if (s > cap) s = cap;
   if (s < 1) s = 1;
   p.splits = s;
+  // Cluster reduction: a split count that divides the k-blocks and bn / 4
+  // (whole 4-column slices per CTA), at most 8 (a portable cluster), no less than
+  // half the stream-K choice (the weight stream keeps most of its SMs).  The
+  // pieces are then summed in shared memory instead of through global
+  // partials and tickets (action out-proj / FFN-down at 32 tokens: 8 splits).
+  if (cred && !fused_norm && s > 1) {
+    int S = 0;
+    for (int c = std::min({8, bn / 4, std::max(s, 2)}); c >= 2; --c)
+      if (kb % c == 0 && (bn / 4) % c == 0) {
+        S = c;
+        break;
+      }
+    if (S >= 2 && 2 * S >= std::min(s, 8)) {
+      p.splits = S;
+      p.cred = S;
+    }
+  }
+  if (tiles >= 24 && p.cred == 0) p.splits = 1;
   return p;
 }
 
@@ -393,6 +416,7 @@ wam_status run_tc(wam_ctx* c, const CUtensorMap& A, const CUtensorMap& Bm, int r
   g.max_ctas = p.max_ctas;
   g.pair = p.pair;
   g.csplit = p.csplit;
+  g.cred = p.cred;
   g.ws = video ? c->ws_gemm_v : c->ws_gemm;
   g.tickets = video ? c->tk_gemm_v : c->tk_gemm;
   g.status = c->status;
@@ -882,6 +906,13 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
   // a step that waits on the video blocks runs beside them: its attention
   // takes little shared memory per CTA so the video GEMMs keep their SMs
   c->attn_spread = ev_wait == nullptr;
+  // GEMM plans by step index alone (the same in every schedule): the first
+  // step may run beside the video expert, later ones run alone
+  const bool later = j > 0;
+  const GemmPlan* pq = later ? &c->p_a_qkv_l : &c->p_a_qkv;
+  const GemmPlan* po = later ? &c->p_a_o_l : &c->p_a_o;
+  const GemmPlan* p1 = later ? &c->p_a_f1_l : &c->p_a_f1;
+  const GemmPlan* p2 = later ? &c->p_a_f2_l : &c->p_a_f2;
   c->cur_cls = WAM_PROF_ACTION_TEMB;
   RET(temb(c, false, &io->sched[j], s));
   c->cur_cls = WAM_PROF_ACTION_IO;
@@ -891,7 +922,7 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
   }
   for (int i = 0; i < d.N; ++i) {
     const float* mod = c->mod_a + (size_t)i * 6 * d.da;
-    Lin Lq{&c->m_w_qkv_a, &c->m_ha, matp(c, blk(x, i, kQkvW)), c->h_a, 3 * d.A, d.da, i, &c->p_a_qkv, d.lh};
+    Lin Lq{&c->m_w_qkv_a, &c->m_ha, matp(c, blk(x, i, kQkvW)), c->h_a, 3 * d.A, d.da, i, pq, d.lh};
     lora(c, Lq, i, kQkvLa, &c->m_la_qkv, &c->p_u_qkv);
     RET(norm_linear(c, Lq, epi_qkv(c, false, i), mod + d.da, mod, nullptr, WAM_PROF_ACTION_QKV, s));
     if (ev_wait) CK(cudaStreamWaitEvent(s, ev_wait[i], 0));
@@ -902,17 +933,17 @@ wam_status enqueue_action_step(wam_ctx* c, cudaStream_t s, const ActionIo* io, i
     c->cur_cls = WAM_PROF_ACTION_OPROJ;
     EpiArgs eo = epi_base(kEpiGateRes, vecp(c, blk(x, i, kOB)), c->x_a, nullptr, d.da);
     eo.gate = mod + 2 * d.da;
-    Lin Lo{&c->m_w_o_a, &c->m_oa, matp(c, blk(x, i, kOW)), c->o_a, d.da, d.A, i, &c->p_a_o, d.lo};
+    Lin Lo{&c->m_w_o_a, &c->m_oa, matp(c, blk(x, i, kOW)), c->o_a, d.da, d.A, i, po, d.lo};
     lora(c, Lo, i, kOLa, &c->m_la_o, &c->p_u_o);
     RET(linear(c, false, Lo, d.Ma, eo, nullptr, s));
-    Lin L1{&c->m_w_f1_a, &c->m_ha, matp(c, blk(x, i, kF1W)), c->h_a, d.Fa, d.da, i, &c->p_a_f1, d.lh};
+    Lin L1{&c->m_w_f1_a, &c->m_ha, matp(c, blk(x, i, kF1W)), c->h_a, d.Fa, d.da, i, p1, d.lh};
     lora(c, L1, i, kF1La, &c->m_la_f1, &c->p_u_f1);
     RET(norm_linear(c, L1, epi_base(kEpiGelu, vecp(c, blk(x, i, kF1B)), nullptr, c->f_a, d.lf), mod + 4 * d.da,
                     mod + 3 * d.da, nullptr, WAM_PROF_ACTION_FFN_UP, s));
     c->cur_cls = WAM_PROF_ACTION_FFN_DOWN;
     EpiArgs e2 = epi_base(kEpiGateRes, vecp(c, blk(x, i, kF2B)), c->x_a, nullptr, d.da);
     e2.gate = mod + 5 * d.da;
-    Lin L2{&c->m_w_f2_a, &c->m_fa, matp(c, blk(x, i, kF2W)), c->f_a, d.da, d.Fa, i, &c->p_a_f2, d.lf};
+    Lin L2{&c->m_w_f2_a, &c->m_fa, matp(c, blk(x, i, kF2W)), c->f_a, d.da, d.Fa, i, p2, d.lf};
     lora(c, L2, i, kF2La, &c->m_la_f2, &c->p_u_f2);
     RET(linear(c, false, L2, d.Ma, e2, nullptr, s));
     trace_mark(c, s, WAM_TRACE_ACTION_END, i);
@@ -1374,11 +1405,38 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
       const int n = atoi(v);
       if (n > 0) actas = n;
     }
+    // Split action GEMMs sum their pieces in a cluster's shared memory;
+    // WAM_ACTION_CRED=0 keeps the same splits but sums through global
+    // partials (the stream-K tickets).
+    const char* crv = getenv("WAM_ACTION_CRED");
+    const bool cred_on = !(crv && crv[0] == '0');
     c->p_a_in = plan_swap(d.da, d.Ma, d.Kin, bn_a, false, actas);
+    // The first Euler step runs beside the video expert: its GEMMs keep the
+    // stream-K plans (the cluster plans below took SMs from the video stream,
+    // config-2 chunk 3.54 -> 3.80 ms).  Later steps run alone and use them.
     c->p_a_qkv = plan_swap(3 * d.A, d.Ma, d.da + d.r, bn_a, fn, actas);
     c->p_a_o = plan_swap(d.da, d.Ma, d.A + d.r, bn_a, false, actas);
     c->p_a_f1 = plan_swap(d.Fa, d.Ma, d.da + d.r, bn_a, fn, actas);
     c->p_a_f2 = plan_swap(d.da, d.Ma, d.Fa + d.r, bn_a, false, actas);
+    // The wide action FFN-up (24 or more feature tiles) splits each tile
+    // over a cluster of WAM_ACTION_WIDE_SPLITS CTAs (default 4; 0 or 1:
+    // unsplit): with the pieces summed in shared memory the split pays (the
+    // 10-step chunk's FFN-up 9.3 -> 5.9 us per launch at 4).  The QKV GEMM
+    // (36 tiles) takes WAM_ACTION_QKV_SPLITS (default 2: 8.6 -> 7.8 us; at 4
+    // its 144 CTAs in clusters did not all find SMs at once, 8.3 -> 12.1 us).
+    int wide = 4, wide_qkv = 2;
+    if (const char* v = getenv("WAM_ACTION_WIDE_SPLITS")) wide = atoi(v);
+    if (const char* v = getenv("WAM_ACTION_QKV_SPLITS")) wide_qkv = atoi(v);
+    c->p_a_qkv_l = plan_swap(3 * d.A, d.Ma, d.da + d.r, bn_a, fn, actas, wide_qkv > 1, wide_qkv);
+    c->p_a_o_l = plan_swap(d.da, d.Ma, d.A + d.r, bn_a, false, actas, true);
+    c->p_a_f1_l = plan_swap(d.Fa, d.Ma, d.da + d.r, bn_a, fn, actas, wide > 1, wide);
+    c->p_a_f2_l = plan_swap(d.da, d.Ma, d.Fa + d.r, bn_a, false, actas, true);
+    if (!cred_on) {
+      c->p_a_qkv_l.cred = 0;
+      c->p_a_o_l.cred = 0;
+      c->p_a_f1_l.cred = 0;
+      c->p_a_f2_l.cred = 0;
+    }
     if (d.r > 0) {
       c->p_u_qkv = plan_swap(d.r, d.Ma, d.da, bn_a, false, actas);
       c->p_u_o = plan_swap(d.r, d.Ma, d.A, bn_a, false, actas);
@@ -1405,6 +1463,10 @@ wam_status wam_init(const wam_config* cfg, uint64_t seed, wam_ctx** out) {
     need(c->p_a_o, d.da, d.Ma, d.A + d.r, true, &ws, &tiles);
     need(c->p_a_f1, d.Fa, d.Ma, d.da + d.r, true, &ws, &tiles);
     need(c->p_a_f2, d.da, d.Ma, d.Fa + d.r, true, &ws, &tiles);
+    need(c->p_a_qkv_l, 3 * d.A, d.Ma, d.da + d.r, true, &ws, &tiles);
+    need(c->p_a_o_l, d.da, d.Ma, d.A + d.r, true, &ws, &tiles);
+    need(c->p_a_f1_l, d.Fa, d.Ma, d.da + d.r, true, &ws, &tiles);
+    need(c->p_a_f2_l, d.da, d.Ma, d.Fa + d.r, true, &ws, &tiles);
     if (d.r > 0) {
       need(c->p_u_qkv, d.r, d.Ma, d.da, true, &ws, &tiles);
       need(c->p_u_o, d.r, d.Ma, d.A, true, &ws, &tiles);
@@ -2039,7 +2101,7 @@ namespace {
 // persistent CTAs (0: all SMs), pair = CTA pairs; swapped: `ctas` = CTAs per
 // output tile.
 wam_status op_linear_bf16(const void* x, const void* w, const float* bias, float* out, int M, int N, int K, bool swap,
-                          int ctas, int bn_normal, bool pair, cudaStream_t s, bool csplit = false) {
+                          int ctas, int bn_normal, bool pair, cudaStream_t s, bool csplit = false, bool cred = false) {
   if (K % 64) return WAM_ERR_INVALID_ARG;
   const int bn = swap ? (M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256) : bn_normal;
   if (swap && M > 256) return WAM_ERR_INVALID_ARG;
@@ -2066,6 +2128,7 @@ wam_status op_linear_bf16(const void* x, const void* w, const float* bias, float
   g.max_ctas = swap ? 0 : std::max(0, ctas);
   g.pair = pair;
   g.csplit = csplit;
+  g.cred = swap && cred ? g.splits : 0;
   const size_t tickets = tc_gemm_tickets(g);
   static thread_local float* ws = nullptr;
   static thread_local int* tk = nullptr;
@@ -2121,9 +2184,14 @@ wam_status wam_op_linear(int dtype, const void* x, const void* w, const float* b
 
 wam_status wam_op_linear_tiled(const void* x, const void* w, const float* bias, float* out, int M, int N, int K, int bn,
                                int mode, int ctas, void* stream) {
-  if (!x || !w || !bias || !out || M < 1 || N < 1 || K < 1 || ctas < 0 || mode < 0 || mode > 2)
+  if (!x || !w || !bias || !out || M < 1 || N < 1 || K < 1 || ctas < 0 || mode < 0 || mode > 3)
     return WAM_ERR_INVALID_ARG;
   if (mode == 2 && ctas % 2) return WAM_ERR_INVALID_ARG;  // clusters of two: an even grid
+  if (mode == 3) {  // swapped, clusters of `ctas` CTAs per tile
+    if (M > 64 || ctas < 2 || ctas > 8 || (K / 64) % ctas || (M <= 32 ? 32 : 64) % (4 * ctas))
+      return WAM_ERR_INVALID_ARG;
+    return op_linear_bf16(x, w, bias, out, M, N, K, true, ctas, 128, false, (cudaStream_t)stream, false, true);
+  }
   return op_linear_bf16(x, w, bias, out, M, N, K, false, ctas, bn, mode == 1, (cudaStream_t)stream, mode == 2);
 }
 

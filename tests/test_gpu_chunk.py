@@ -117,6 +117,37 @@ def test_video_cluster_split(monkeypatch, batch):
     check_parity(got, inp, ref_a0, ref_veff, c.dtype)
 
 
+@pytest.mark.parametrize("batch,shape", [
+    (1, dict(n_heads=8, ffn_action=1536)),
+    (2, dict(n_heads=8, ffn_action=1536)),
+    (1, dict(d_action=256, n_heads=16, ffn_action=3072)),
+])
+def test_action_cluster_reduce(monkeypatch, batch, shape):
+    """Action GEMMs split over clusters, the pieces summed in shared memory:
+    out-projection and FFN-down (the first shape: 2 and 8 CTAs per
+    128-feature tile over 8 and 24 k-blocks; at batch 2 on 64-token tiles),
+    and the wide QKV / FFN-up (the last shape: 24 feature tiles each, 4 CTAs
+    per tile; the QK-norm / RoPE and GELU epilogues).  Bitwise equal to the
+    same splits summed through global partials, CEWP == sequential, at parity
+    with the oracle."""
+    c = _mid().replace(batch=batch, **shape)
+    monkeypatch.delenv("WAM_ACTION_WIDE_SPLITS", raising=False)
+    monkeypatch.setenv("WAM_ACTION_QKV_SPLITS", "4")  # the QKV epilogue on clusters too
+    inp = inputs(c, 29)
+    monkeypatch.delenv("WAM_ACTION_CRED", raising=False)
+    wam = W.Wam(c, seed=29)
+    got = run_chunk(wam, inp, S=2, mode=W.CEWP, use_graph=True)
+    for mode, graph in ((W.SEQUENTIAL, True), (W.CEWP, False)):
+        assert np.array_equal(run_chunk(wam, inp, S=2, mode=mode, use_graph=graph), got)
+    wam.close()
+    monkeypatch.setenv("WAM_ACTION_CRED", "0")
+    wam = W.Wam(c, seed=29)
+    assert np.array_equal(run_chunk(wam, inp, S=2), got)
+    wam.close()
+    ref_a0, ref_veff = oracle_chunk(c, 29, inp, S=2)
+    check_parity(got, inp, ref_a0, ref_veff, c.dtype)
+
+
 def test_video_qkv_192_wide(monkeypatch):
     """Six heads (attention width 384): the video QKV runs on 192-wide tiles
     (18 whole tiles against 15 at 256 wide), the QK-norm / RoPE epilogue

@@ -105,6 +105,45 @@ def test_linear_192_wide(M_, N, K, ctas):
     assert rel_l2(got, ref) < 4e-6
 
 
+# Swapped orientation (the action expert's 32-token GEMMs): each 128-feature
+# tile split over a cluster of `ctas` CTAs, one equal k-range each, the pieces
+# summed in shared memory (mode 3), against the exact sum and bitwise against
+# the global split-tile reduction on the same split (op_linear, swap).
+@pytest.mark.parametrize("M_,N,K,ctas", [
+    (32, 768, 1536, 8),   # action out-projection shape: 6 tiles x 8 CTAs, 3 k-blocks each
+    (32, 768, 3072, 8),   # action FFN-down shape: 6 k-blocks each
+    (20, 300, 512, 4),    # ragged tokens and features: 3 tiles, 8-column shares
+    (64, 256, 1024, 8),   # 64 tokens: a 64-wide token tile, 8-column shares
+    (7, 130, 128, 2),     # one k-block per CTA, a second tile of 2 rows
+])
+def test_linear_swapped_cluster_reduce(M_, N, K, ctas):
+    rng = np.random.default_rng(M_ * 7 + N + K + ctas)
+    x = round_bf16(rng.standard_normal((M_, K)).astype(np.float32))
+    w = round_bf16((0.05 * rng.standard_normal((N, K))).astype(np.float32))
+    b = rng.standard_normal(N).astype(np.float32)
+    ref = x.astype(np.float64) @ w.astype(np.float64).T + b
+    got_cr = torch.full((M_, N), float("nan"), device=DEV)
+    W.op_linear_tiled(_bf16(x), _bf16(w), _f32(b), got_cr, M_, N, K, mode=3, ctas=ctas)
+    got_tk = torch.full((M_, N), float("nan"), device=DEV)
+    W.op_linear(W.BF16, _bf16(x), _bf16(w), _f32(b), got_tk, M_, N, K, swap=True, splits=ctas)
+    torch.cuda.synchronize()
+    a, t = got_cr.cpu().numpy(), got_tk.cpu().numpy()
+    assert np.isfinite(a).all()
+    assert rel_l2(a, ref) < 4e-6
+    # the same pieces added in the same (k) order: the same bits
+    assert np.array_equal(a, t)
+
+
+def test_linear_swapped_cluster_reduce_rejects_bad_shapes():
+    x = torch.zeros((32, 1536), device=DEV, dtype=torch.bfloat16)
+    w = torch.zeros((768, 1536), device=DEV, dtype=torch.bfloat16)
+    b = torch.zeros(768, device=DEV)
+    out = torch.zeros((32, 768), device=DEV)
+    for ctas in (1, 9, 5):  # outside 2..8, or not dividing the 24 k-blocks
+        with pytest.raises(W.WamError):
+            W.op_linear_tiled(x, w, b, out, 32, 768, 1536, mode=3, ctas=ctas)
+
+
 def test_linear_cluster_forms_repeatable():
     """The same launch three times gives the same bits (fixed split points and
     fixed-order partial sums, whatever the timing of the clusters)."""
