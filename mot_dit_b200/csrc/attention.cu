@@ -357,6 +357,7 @@ constexpr int kKVTile = kTK * kD * 2;  // 8 KB: one K or V tile (64 rows x 128 B
 
 struct AttnJointK {
   int H, Lq, Lk, splits, kps, ready, ld_out;
+  const int* ready_flag;  // non-null: `ready` applies only if it reads 1
   int zk0, zv0;
   const __nv_bfloat16* q;
   __nv_bfloat16* out;
@@ -432,8 +433,17 @@ __global__ void __launch_bounds__(kJThreads, 1)
   };
   const int first = min(ntiles, kJStages);
   int issued = 0;
-  if (tid == 0)  // tiles of keys complete before the launch
-    while (issued < first && min(k_end, k_begin + (issued + 1) * kTK) <= a.ready) issue(issued++);
+  if (tid == 0) {  // tiles of keys complete before the launch
+    int ready = a.ready;
+    if (a.ready_flag) {
+      int f;
+      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(f) : "l"(a.ready_flag) : "memory");
+      if (f != 1) ready = 0;
+      else  // the rows were written before the flag was set; TMA (the async proxy) reads them next
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
+    while (issued < first && min(k_end, k_begin + (issued + 1) * kTK) <= ready) issue(issued++);
+  }
   pdl_wait();  // the queries and the action rows are the previous kernel's
   WAM_KT_WAITED();
   if (tid == 0)
@@ -750,6 +760,7 @@ cudaError_t launch_attention_joint(const AttnJoint& t, cudaStream_t s) {
   k.splits = t.splits;
   k.kps = (t.Lk + t.splits - 1) / t.splits;
   k.ready = t.ready;
+  k.ready_flag = t.ready_flag;
   k.ld_out = ldo;
   k.zk0 = t.zk0;
   k.zv0 = t.zv0;

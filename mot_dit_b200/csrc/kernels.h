@@ -193,6 +193,8 @@ struct TembArgs {
   float* scratch;                    // 256 + 2d floats
   int d, n_blocks;
   bool bf16;
+  int* set_flag = nullptr;  // non-null: the first kernel, once its dependent-launch wait has returned
+                            // (every kernel before it on the stream complete), stores 1 here (release)
 };
 cudaError_t launch_temb(const TembArgs& a, cudaStream_t s);
 
@@ -228,6 +230,8 @@ struct AttnJoint {
   void* out;
   int B, H, Lq, Lk, ld_out;
   int ready;
+  const int* ready_flag = nullptr;  // non-null: the rows below `ready` are read before the dependent-launch
+                                    // wait only if this flag reads 1 (acquire), else after it
   int splits;
   bool spread = false;  // one CTA per SM (more shared memory than it needs): for launches with the GPU to themselves
   unsigned* status;

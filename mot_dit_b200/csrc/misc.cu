@@ -69,10 +69,14 @@ template <bool BF16>
 __global__ void __launch_bounds__(32 * kGemvWarps)
     gemv_kernel(const void* __restrict__ W, const float* __restrict__ x, const float* __restrict__ t, int mode,
                 const float* __restrict__ bias, float* __restrict__ y, int N, int K, const float* __restrict__ T0,
-                size_t T_stride, int n_blocks, float* __restrict__ mod) {
+                size_t T_stride, int n_blocks, float* __restrict__ mod, int* set_flag) {
   extern __shared__ float xs[];
   pdl_trigger();
   pdl_wait();
+  // every kernel before this one on the stream is complete and its writes
+  // visible: say so to later kernels that read before their own wait
+  if (set_flag && blockIdx.x == 0 && threadIdx.x == 0)
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(set_flag), "r"(1) : "memory");
   if (mode == 2) {
     const double tt = (double)t[0];
     for (int k = threadIdx.x; k < 128; k += blockDim.x) {
@@ -306,18 +310,19 @@ cudaError_t launch_temb(const TembArgs& a, cudaStream_t s) {
   if (d % 8 != 0) return cudaErrorInvalidValue;
   float* c1 = a.scratch;
   float* c = a.scratch + d;
-  auto gemv = [&](const void* W, const float* x, int mode, const float* b, float* y, int N, int K, bool mod) {
+  auto gemv = [&](const void* W, const float* x, int mode, const float* b, float* y, int N, int K, bool mod,
+                  int* flag = nullptr) {
     dim3 grid((N + kGemvWarps - 1) / kGemvWarps);
     const size_t sm = (size_t)(mode == 2 ? 256 : K) * sizeof(float);
     float* modp = mod ? a.mod : nullptr;
     if (a.bf16)
       return launch_k(gemv_kernel<true>, grid, dim3(32 * kGemvWarps), sm, s, W, x, a.t, mode, b, y, N, K, a.T0,
-                      a.T_stride, a.n_blocks, modp);
+                      a.T_stride, a.n_blocks, modp, flag);
     return launch_k(gemv_kernel<false>, grid, dim3(32 * kGemvWarps), sm, s, W, x, a.t, mode, b, y, N, K, a.T0,
-                    a.T_stride, a.n_blocks, modp);
+                    a.T_stride, a.n_blocks, modp, flag);
   };
   cudaError_t e;
-  if ((e = gemv(a.w1, nullptr, 2, a.b1, c1, d, 256, false)) != cudaSuccess) return e;
+  if ((e = gemv(a.w1, nullptr, 2, a.b1, c1, d, 256, false, a.set_flag)) != cudaSuccess) return e;
   if ((e = gemv(a.w2, c1, 1, a.b2, c, d, d, false)) != cudaSuccess) return e;
   return gemv(a.wm, c, 1, a.bm, nullptr, 6 * d, d, true);
 }
