@@ -1458,6 +1458,28 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int m = mb + c + j;
               if (m < g.rows_b) R.out_act[(size_t)m * R.ld + n] = __float2bfloat16_rn(sc * (v[j] + bias));
             }
+          } else if (n_ok && R.kind == kEpiEuler) {
+            // the step's dt once, and the 32 state values (distinct rows) all
+            // requested before any store: per-element calls reloaded the
+            // schedule and read each value after the previous store (the
+            // compiler cannot rule out aliasing), a chain of 32 round trips
+            const float dt = e.aio->sched[e.step] - e.aio->sched[e.step + 1];
+            __nv_bfloat16* const a_next = reinterpret_cast<__nv_bfloat16*>(e.a_next);
+            const int a_next_ld = e.a_next_ld;
+            float a0[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int m = mb + c + j;
+              a0[j] = m < g.rows_b ? R.out_f32[(size_t)m * R.ld + n] : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int m = mb + c + j;
+              if (m >= g.rows_b) continue;
+              const float a = a0[j] - dt * (v[j] + bias);
+              R.out_f32[(size_t)m * R.ld + n] = a;
+              if (a_next) a_next[(size_t)m * a_next_ld + n] = __float2bfloat16_rn(a);
+            }
           } else if (n_ok) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
