@@ -37,6 +37,22 @@
 // prefetched into that staging with cp.async while the MMA runs and updated in
 // place; the QKV epilogue prefetches its tokens' RoPE rows the same way.
 //
+// Clusters (no load is multicast; partner data crosses by bulk copies into
+// the partner's idle operand ring, completing on its mbarrier):
+//  - PAIR: two CTAs share each M = 256 tcgen05.mma (cta_group::2), each
+//    loading its own 128 rows of A and half of B (opt-in);
+//  - csplit (normal orientation, clusters of two): a tile whose k-range
+//    stream-K splits exactly between the two CTAs is finished in column
+//    halves, each CTA sending the other its half-partial of the other's
+//    columns;
+//  - cred (swapped, clusters of up to 8): each tile's pieces are the CTAs of
+//    one cluster, one equal k-range each; every CTA sends each partner its
+//    4-column slice of that partner's token columns and finishes its own,
+//    summing the slices in rank (= k) order -- the ticket path's order, so
+//    the result is bitwise the same.  Each CTA arrives at the cluster's exit
+//    barrier when it is done with its partners and waits there before it
+//    leaves, so none leaves while a partner may still copy into it.
+//
 // Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
 // issuer, warps 2..5 epilogue (warp w reads TMEM lanes 32*(w%4) .. +31).
 #include <cstdio>
