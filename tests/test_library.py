@@ -162,3 +162,26 @@ def test_noalloc_attention_refusals_without_a_device():
     # (at least two splits of 4224 floats each) already refuses beyond 248 pairs
     assert call(B=1025, H=1, Lq=1, Lk=128, Lc=128, splits=2) == 2
     assert call(B=248, H=1, Lq=1, Lk=128, Lc=128, splits=2, ptrs=(None, p, p, p)) == 1
+
+
+def test_linear_tiled_refusals_without_a_device():
+    """wam_op_linear_tiled refuses bad shapes and values before any CUDA call,
+    for the swapped cluster form (mode 3) among them: every path below runs on
+    a host without a GPU (the pointers are dummies that are never
+    dereferenced)."""
+    L = W.lib()
+    p = C.c_void_p(0x1000)
+
+    def call(M=32, N=768, K=1536, bn=128, mode=3, ctas=8, ptrs=(p, p, p, p)):
+        return L.wam_op_linear_tiled(*ptrs, M, N, K, bn, mode, ctas, None)
+    assert call(mode=4) == 1 and call(mode=-1) == 1      # no such form
+    assert call(ctas=-1) == 1
+    assert call(ptrs=(None, p, p, p)) == 1 and call(ptrs=(p, p, None, p)) == 1
+    assert call(M=0) == 1 and call(N=0) == 1 and call(K=0) == 1
+    assert call(mode=2, ctas=7) == 1                     # clusters of two: an even grid
+    # mode 3: 2..8 CTAs per tile, dividing the k-blocks and the token tile's 4-column slices
+    assert call(ctas=1) == 1 and call(ctas=9) == 1 and call(ctas=0) == 1
+    assert call(ctas=5) == 1                             # 24 k-blocks
+    assert call(K=1600, ctas=2) == 1                     # K/64 = 25: not a multiple of 2
+    assert call(M=65) == 1                               # at most 64 tokens
+    assert call(M=20, K=3 * 64 * 4, ctas=3) == 1         # 32 columns: 8 slices do not split in 3
